@@ -1,0 +1,403 @@
+"""Benchmark: decode-attention tokens/s on one B200 (or N, data parallel) through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+One step = one whole decode step of the hot path on one batch: append the s_q new cache rows
+of every request, then decode attention over the full cache (range planning, tensor-core
+split-KV kernel, split combine).  Inputs are seeded synthetic tensors resident in HBM before
+the timed region; the cache (0.30 GB for the default workload) is larger than the 126 MB L2,
+so no flush is done between steps.  Timing: CUDA events on the launching stream over exactly K
+steps, bracketed by a barrier and a device synchronise, max over ranks.  Rank 0 prints one
+JSON line.
+
+`--impl reference` times the fp64 CPU oracle (the correctness reference) on the host cores,
+on a bounded sample of the same workload; under torchrun only rank 0 runs it.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "decode attn tokens/s; KV-cache GB/s & TFLOPS as fraction of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def shard_requests(batch: int, rank: int, world: int):
+    """Weak scaling: every rank decodes its own full batch; returns the global request ids of
+    this rank (disjoint across ranks)."""
+    return list(range(rank * batch, (rank + 1) * batch))
+
+
+def reduce_max(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def workload_accounting(w, lengths):
+    from_oracle = None  # the byte / FLOP formulas below restate the definitions, no oracle import
+    lengths = np.asarray(lengths, dtype=np.int64)
+    if w.kind in ("mla", "gla"):
+        row = w.groups * w.d_k + w.d_rope
+    else:
+        row = w.groups * (w.d_k + w.d_v) + w.d_rope
+    cache_bytes = int(lengths.sum()) * row * 2
+    io_bytes = w.batch * w.s_q * w.h_q * ((w.d_k + w.d_rope) * 2 + w.d_v * 2 + 4)
+    vis = sum(int((lengths - w.s_q + i + 1).sum()) for i in range(w.s_q))
+    flops = vis * 2 * w.h_q * (w.d_k + w.d_rope + w.d_v)
+    del from_oracle
+    return cache_bytes, io_bytes, flops
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the GPU works (200 ms period)."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.rows.append(parts)
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in self.rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in self.rows if num(r[2]) is not None]
+        load = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in self.rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(load) if load else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(self.rows)}
+
+
+def bench_gpu(args, rank, world, local_rank):
+    import latent_kv_cache_split_b200 as lkv
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+    w = synth.workload(args.workload)
+    d = synth.make_inputs(w)
+    new = synth.new_token_rows(w)
+    lengths = d["lengths"]
+    cu = d["cu_seqlens"].to(dev)
+    q = d["q"].to(dev)
+    qr = d["q_rope"].to(dev)
+    B, S = w.batch, w.s_q
+    if w.kind in ("mla", "gla"):
+        cache = d["cache"].to(dev)
+        width = w.groups * w.d_k
+        lat, kpe = cache[:, :width], cache[:, width:]
+        new_rows = new["rows"].to(dev)
+    else:
+        k, v, kpe = d["k"].to(dev), d["v"].to(dev), d["kpe"].to(dev)
+        new_k, new_v, new_kpe = new["k"].to(dev), new["v"].to(dev), new["kpe"].to(dev)
+    out = torch.empty((B, S, w.h_q, w.d_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, S, w.h_q), dtype=torch.float32, device=dev)
+    nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+    if w.kind == "mla":
+        ws = torch.empty(lkv.mla_decode_workspace_size(B, S, w.h_q, w.d_k, nsm), dtype=torch.uint8, device=dev)
+    else:
+        kind = lkv.KIND_GQLA if w.kind == "gqla" else lkv.KIND_GLA
+        ws = torch.empty(lkv.group_decode_workspace_size(kind, B, S, w.h_q, w.groups, w.d_v, nsm),
+                         dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    launches_per_step = 3 if w.kind != "gqla" else 5   # append(s) + decode + combine
+
+    def append():
+        if w.kind in ("mla", "gla"):
+            lkv.latent_cache_append(new_rows, cache, cu, S)
+        else:
+            lkv.latent_cache_append(new_k, k, cu, S)
+            lkv.latent_cache_append(new_v, v, cu, S)
+            lkv.latent_cache_append(new_kpe, kpe, cu, S)
+
+    def decode(qq, qqr, o, l):
+        if w.kind == "mla":
+            lkv.mla_absorbed_decode(qq, qqr, lat, kpe, cu, w.scale, out=o, lse=l, workspace=ws)
+        elif w.kind == "gqla":
+            lkv.gqla_group_decode(qq, qqr, k, v, kpe, cu, w.scale, out=o, lse=l, workspace=ws)
+        else:
+            lkv.gla_group_decode(qq, qqr, lat, kpe, w.groups, cu, w.scale, out=o, lse=l, workspace=ws)
+
+    def step():
+        append()
+        decode(q, qr, out, lse)
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    sampler = ClockSampler(dev.index if dev.index is not None else 0) if rank == 0 else None
+    for _ in range(args.warmup):
+        step()
+    if lkv.check_device() != 0:
+        raise RuntimeError("device error during warm-up")
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    # ---- timed region: exactly K steps, per-step events around the decode call as well
+    ev_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_d = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    barrier()
+    t0.record(stream)
+    for i in range(args.steps):
+        ev_s[i].record(stream)
+        append()
+        ev_d[i].record(stream)
+        decode(q, qr, out, lse)
+        ev_e[i].record(stream)
+    t1.record(stream)
+    barrier()
+    total_ms = t0.elapsed_time(t1)
+    dec_ms = [ev_d[i].elapsed_time(ev_e[i]) for i in range(args.steps)]
+    if sampler:
+        time.sleep(0.2)
+        sampler.stop()
+    err = lkv.check_device()
+    if err != 0:
+        raise RuntimeError(f"device error word {err} after the timed region")
+    total_ms = reduce_max(total_ms, world, dev)
+    dec_avg_ms = reduce_max(float(np.mean(dec_ms)), world, dev)
+
+    # ---- end to end through the public API: host inputs in, host result out, every step
+    q_h = d["q"].pin_memory()
+    qr_h = d["q_rope"].pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    q_d = torch.empty_like(q)
+    qr_d = torch.empty_like(qr)
+    if w.kind in ("mla", "gla"):
+        rows_h = new["rows"].pin_memory()
+        step_in = [(rows_h, new_rows)]
+    else:
+        step_in = [(new["k"].pin_memory(), new_k), (new["v"].pin_memory(), new_v),
+                   (new["kpe"].pin_memory(), new_kpe)]
+    h2d = q_h.numel() * 2 + qr_h.numel() * 2 + sum(h.numel() * h.element_size() for h, _ in step_in)
+    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+    e2e_steps = max(3, min(args.steps, 200))
+
+    def e2e_step():
+        q_d.copy_(q_h, non_blocking=True)
+        qr_d.copy_(qr_h, non_blocking=True)
+        for h, dd in step_in:
+            dd.copy_(h, non_blocking=True)
+        append()
+        decode(q_d, qr_d, out, lse)
+        out_h.copy_(out, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    barrier()
+    e2e_ms = reduce_max(e0.elapsed_time(e1), world, dev) / e2e_steps
+
+    tokens = B * S * world
+    cache_bytes, io_bytes, flops = workload_accounting(w, lengths)
+    res = None
+    if rank == 0:
+        peaks, how = load_peaks()
+        ms = total_ms / args.steps
+        alg_bytes = cache_bytes + io_bytes
+        dec_s = dec_avg_ms * 1e-3
+        gbs = alg_bytes / dec_s / 1e9
+        tfl = flops / dec_s / 1e12
+        t_hbm = alg_bytes / (peaks["hbm_gbs"] * 1e9)
+        t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+        bound = "hbm" if t_hbm >= t_tc else "tensor"
+        achieved = gbs if bound == "hbm" else tfl
+        peak = peaks["hbm_gbs"] if bound == "hbm" else peaks["bf16_tflops"]
+        res = {
+            "metric": METRIC,
+            "value": tokens / (ms * 1e-3),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded Gaussian, shapes of the pages' MLA/GQLA decode workloads)",
+            "config": {"workload": w.name, "kind": w.kind, "batch_per_gpu": B, "s_q": S, "h_q": w.h_q,
+                       "groups": w.groups, "d_k": w.d_k, "d_v": w.d_v, "d_rope": w.d_rope,
+                       "seqlen": w.seqlen, "cache_gb_per_gpu": round(cache_bytes / 1e9, 4),
+                       "l2": "inputs larger than L2 (cache >> 126 MB); no flush",
+                       "parallelism": f"dp{world}"},
+            "decode_kernel_ms": dec_avg_ms,
+            "kv_gbs": gbs,
+            "tflops": tfl,
+            "roofline": {"bound": bound, "achieved": achieved, "peak": peak,
+                         "unit": "GB/s" if bound == "hbm" else "TFLOP/s", "frac": achieved / peak,
+                         "traffic": None, "peak_source": f"{how} (MEASURED_PEAKS.json burst)",
+                         "roofline_ms": max(t_hbm, t_tc) * 1e3,
+                         "frac_of_step_roofline": max(t_hbm, t_tc) * 1e3 / ms,
+                         "kernel": "decode_tc_kernel + split combine (one lkv_*_decode call)",
+                         "algorithmic_bytes": alg_bytes, "algorithmic_flops": flops},
+            "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+                    "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": sampler.summary() if sampler else None,
+        }
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return res
+
+
+def cpu_baseline(w, budget_s: float):
+    """The oracle as it stands on the host cores, on a bounded sample of the workload."""
+    import oracle
+    d = synth.make_inputs(w)
+    cu = d["cu_seqlens"].numpy().astype(np.int64)
+    order = list(range(w.batch))
+    t0 = time.perf_counter()
+    done = 0
+    for b in order:
+        if w.kind == "mla":
+            c = d["cache"]
+            oracle.mla_absorbed_decode(d["q"], d["q_rope"], c[:, :w.d_k], c[:, w.d_k:], cu, w.scale, requests=[b])
+        elif w.kind == "gqla":
+            oracle.gqla_group_decode(d["q"], d["q_rope"], d["k"], d["v"], d["kpe"], cu, w.scale, requests=[b])
+        else:
+            width = w.groups * w.d_k
+            c = d["cache"]
+            oracle.gla_group_decode(d["q"], d["q_rope"], c[:, :width], c[:, width:], w.groups, cu, w.scale,
+                                    requests=[b])
+        done += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done * w.s_q / dt, "unit": "tokens/s", "cores": os.cpu_count(),
+            "kind": "oracle", "sample": f"{done} of {w.batch} requests of {w.name} (fp64 numpy oracle)",
+            "seconds": dt}
+
+
+def bench_reference(args, rank, world):
+    if rank != 0:
+        return None
+    w = synth.workload(args.workload)
+    budget = max(1.0, 150.0 / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        cpu_baseline(w, budget)
+    vals = [cpu_baseline(w, budget) for _ in range(args.steps)]
+    v = float(np.mean([x["value"] for x in vals]))
+    cb = dict(vals[-1])
+    cb["value"] = v
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * w.batch * w.s_q / v,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "batch_per_gpu": w.batch, "s_q": w.s_q,
+                                        "seqlen": w.seqlen, "parallelism": f"dp{world}"},
+        "cpu_baseline": cb,
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="mla_b64_l4096", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="lkv", choices=["lkv", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", str(args.gpus)))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus and "WORLD_SIZE" in os.environ:
+        raise SystemExit("--gpus must match the launcher's world size")
+    if args.impl == "reference":
+        res = bench_reference(args, rank, world)
+    else:
+        res = bench_gpu(args, rank, world, local_rank)
+        if rank == 0 and world == 1:
+            res["cpu_baseline"] = cpu_baseline(synth.workload(args.workload), args.cpu_budget)
+        elif rank == 0:
+            res["cpu_baseline"] = None
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,202 @@
+/*
+ * lkv.h -- C ABI of the B200 (sm_100a) latent / grouped KV-cache decode-attention library.
+ *
+ * One decode step for a batch of requests: every request b has a contiguous run of
+ * L_b cached tokens starting at row cu_seqlens[b] of the cache arrays; its s_q (1 or 2)
+ * newest tokens are already the last s_q rows of that run.  Query token i of request b
+ * attends to rows 0 .. L_b - s_q + i of its run (causal inside the new tokens).  For query
+ * head h of group j = h / (h_q / G):
+ *
+ *   s[t]  = scale * ( q[b,i,h,:] . K_j[t,:]  +  q_rope[b,i,h,:] . k_rope[t,:] )
+ *   lse   = ln sum_t exp(s[t])
+ *   out   = sum_t exp(s[t] - lse) * V_j[t,:]
+ *
+ * Forms (sources: "GQLA: Group-Query Latent Attention for Hardware-Adaptive Large Language
+ * Model Decoding", section 2 "Methodology"; "Grouped Latent Attention" article, section "GLA"):
+ *   - MLA absorbed path (section 2, "MQA absorbed path"): G = 1, K = V = the latent c_KV
+ *     (width r_kv), plus one RoPE key of width d_R shared by all heads.  The query carries
+ *     W_UK already (q_nope_abs); the output is in latent space.
+ *   - GQLA GQA path (section 2, "GQA path"): the latent expanded once into g groups of
+ *     keys K_j and values V_j (width d_h each) plus the shared RoPE key.
+ *   - GLA: n_lat latent groups of width r_g; group j's heads use latent group j as both
+ *     K_j and V_j; one RoPE key shared by all groups.
+ *
+ * Conventions for every entry point:
+ *   - All pointers are device pointers unless stated; the caller allocates every buffer,
+ *     including the workspace.  The library allocates no device memory in these calls.
+ *   - Calls are asynchronous on `stream` (cudaStream_t; NULL = legacy default stream).
+ *   - Argument errors are detected on the host before anything is launched and returned
+ *     as LKV_ERR_INVALID_ARG / LKV_ERR_UNSUPPORTED / LKV_ERR_WORKSPACE.  These checks make
+ *     no CUDA call.
+ *   - Faults found on the device (a bounded wait that gave up, a cache length below s_q,
+ *     a destination row past the cache) never trap: the kernel records a site code in a
+ *     device error word, skips the bad access and unwinds.  lkv_check_device() reads it.
+ *   - "bf16" means bf16 storage with fp32 accumulation; lse is always fp32, natural log.
+ *   - Row strides are in elements and must keep every row 16-byte aligned.
+ */
+#ifndef LKV_H
+#define LKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* lkv_stream_t; /* same type as cudaStream_t */
+
+typedef enum {
+  LKV_OK = 0,
+  LKV_ERR_INVALID_ARG = 1, /* null pointer, bad size, stride or alignment; nothing launched */
+  LKV_ERR_UNSUPPORTED = 2, /* well formed but outside the implemented shapes / dtypes */
+  LKV_ERR_WORKSPACE = 3,   /* workspace null or smaller than the *_workspace_size value */
+  LKV_ERR_CUDA = 4,        /* a CUDA runtime call failed (launch, attribute, tensor map) */
+  LKV_ERR_DEVICE = 5       /* lkv_check_device: a kernel recorded a device-side failure */
+} lkv_status;
+
+typedef enum { LKV_BF16 = 0, LKV_FP32 = 1 } lkv_dtype;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int lkv_version(void);
+
+/* Static description of a status code.  Never NULL. */
+const char* lkv_status_string(int status);
+
+/*
+ * Work partition used by the decode kernels (host-only, no CUDA call).  The tiles of all
+ * (request, unit) pairs are laid end to end and cut into `ranges` equal runs, one per
+ * persistent CTA (MLA: per CTA pair).  A unit is one query token of a request for MLA,
+ * one group of a request for GQLA / GLA.  Returns the number of ranges, or -1 on bad input.
+ *   kind: 0 = MLA absorbed, 1 = GQLA, 2 = GLA.  num_sms: SMs available on the device.
+ */
+int lkv_plan_ranges(int kind, int batch, int s_q, int groups, int num_sms);
+
+/*
+ * Host-only view of the same partition (no CUDA call): for host-side cu_seqlens_host [batch+1]
+ * and `num_ranges` ranges, writes one record of 8 int32 per segment, in processing order:
+ *   (range, request, unit, tile_lo, tile_hi, complete, slot, unit_id)
+ * tiles are 64 keys; slot is -1 for a segment that covers its whole unit, else the partial
+ * slot (0 = first segment of its range, 1 = last).  Returns the number of segments (records
+ * past max_out are counted but not written), or -1 on bad input.
+ */
+int lkv_plan_segments(int kind, const int32_t* cu_seqlens_host, int batch, int s_q, int groups,
+                      int num_ranges, int32_t* out, int max_out);
+
+/* Bytes of workspace the decode entry points need (host-only, no CUDA call); 0 on bad input.
+ * The workspace holds fp32 partial outputs / LSEs for units that straddle a range boundary
+ * and the record of which unit each partial belongs to.  Its contents need no initialisation
+ * and are fully rewritten by every call. */
+size_t lkv_mla_decode_workspace_size(int batch, int s_q, int h_q, int r_kv, int num_sms);
+size_t lkv_group_decode_workspace_size(int kind, int batch, int s_q, int h_q, int groups,
+                                       int d_v, int num_sms);
+
+/*
+ * MLA absorbed decode (MQA over the shared latent).
+ *   q_nope_abs [batch, s_q, h_q, r_kv]  contiguous, query with W_UK folded in
+ *   q_rope     [batch, s_q, h_q, d_rope] contiguous
+ *   ckv        [cache_rows, r_kv]  row stride ckv_row_stride (elements)
+ *   kpe        [cache_rows, d_rope] row stride kpe_row_stride (ckv and kpe may interleave in
+ *              one [cache_rows, r_kv + d_rope] array: kpe = ckv + r_kv, same stride)
+ *   cu_seqlens [batch + 1] int32, device; cu_seqlens[batch] <= cache_rows;
+ *              every L_b = cu_seqlens[b+1] - cu_seqlens[b] >= s_q (checked on the device: a shorter
+ *              request is recorded as LKV_SITE_BAD_LENGTH and its outputs are not written)
+ *   out        [batch, s_q, h_q, r_kv] (bf16 for LKV_BF16, fp32 for LKV_FP32)
+ *   lse        [batch, s_q, h_q] fp32
+ * Implemented: LKV_BF16 with r_kv = 512, d_rope = 64, h_q = 128 (tcgen05 kernel, CTA pairs);
+ *              LKV_FP32 with r_kv + d_rope <= 1024, r_kv <= 512 (CUDA-core kernel).
+ * s_q must be 1 or 2.  workspace_bytes >= lkv_mla_decode_workspace_size(...).
+ */
+lkv_status lkv_mla_absorbed_decode(const void* q_nope_abs, const void* q_rope, const void* ckv,
+                                   int64_t ckv_row_stride, const void* kpe,
+                                   int64_t kpe_row_stride, int64_t cache_rows,
+                                   const int32_t* cu_seqlens, int batch, int s_q, int h_q,
+                                   int r_kv, int d_rope, float scale, int dtype, void* out,
+                                   float* lse, void* workspace, size_t workspace_bytes,
+                                   lkv_stream_t stream);
+
+/*
+ * GQLA grouped decode (GQA path over g expanded key/value groups).
+ *   q      [batch, s_q, h_q, d_h], q_rope [batch, s_q, h_q, d_rope] contiguous
+ *   k, v   [cache_rows, g, d_h] with row strides k_row_stride / v_row_stride (elements per
+ *          cache row, >= g*d_h); kpe [cache_rows, d_rope] row stride kpe_row_stride
+ *   out    [batch, s_q, h_q, d_h]; lse [batch, s_q, h_q]
+ * Implemented: LKV_BF16 with d_h = 128, d_rope = 64, h_q / g <= 64, s_q * h_q / g <= 128;
+ *              LKV_FP32 with d_h + d_rope <= 1024, d_h <= 512.
+ */
+lkv_status lkv_gqla_group_decode(const void* q, const void* q_rope, const void* k,
+                                 int64_t k_row_stride, const void* v, int64_t v_row_stride,
+                                 const void* kpe, int64_t kpe_row_stride, int64_t cache_rows,
+                                 const int32_t* cu_seqlens, int batch, int s_q, int h_q, int g,
+                                 int d_h, int d_rope, float scale, int dtype, void* out,
+                                 float* lse, void* workspace, size_t workspace_bytes,
+                                 lkv_stream_t stream);
+
+/*
+ * GLA grouped-latent decode.
+ *   q      [batch, s_q, h_q, r_g], q_rope [batch, s_q, h_q, d_rope] contiguous
+ *   clat   [cache_rows, n_lat * r_g] row stride clat_row_stride; group j = columns
+ *          j*r_g .. (j+1)*r_g - 1; kpe [cache_rows, d_rope] row stride kpe_row_stride
+ *   out    [batch, s_q, h_q, r_g]; lse [batch, s_q, h_q]
+ * Implemented: LKV_BF16 with r_g = 256, d_rope = 64, s_q * h_q / n_lat <= 128;
+ *              LKV_FP32 with r_g + d_rope <= 1024, r_g <= 512.
+ */
+lkv_status lkv_gla_group_decode(const void* q, const void* q_rope, const void* clat,
+                                int64_t clat_row_stride, const void* kpe, int64_t kpe_row_stride,
+                                int64_t cache_rows, const int32_t* cu_seqlens, int batch, int s_q,
+                                int h_q, int n_lat, int r_g, int d_rope, float scale, int dtype,
+                                void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                lkv_stream_t stream);
+
+/*
+ * Cache append: copy the s_q new rows of every request into the cache.
+ * Row b*s_q + i of new_rows goes to cache row cu_seqlens[b] + L_b - s_q + i (the new tokens
+ * are the tail of each request's run; source: GQLA explainer, section 2 -- the cache holds
+ * the latent and RoPE key per token, or the expanded groups on the GQA path).
+ *   new_rows  [batch*s_q rows] of row_bytes each, row stride new_row_stride_bytes
+ *   cache     [cache_rows rows], row stride cache_row_stride_bytes
+ * row_bytes, both strides and both pointers must be multiples of 16.  A request with
+ * L_b < s_q or a destination past cache_rows is skipped and recorded in the device error word.
+ */
+lkv_status lkv_latent_cache_append(const void* new_rows, int64_t new_row_stride_bytes,
+                                   void* cache, int64_t cache_row_stride_bytes,
+                                   int64_t cache_rows, int64_t row_bytes,
+                                   const int32_t* cu_seqlens, int batch, int s_q,
+                                   lkv_stream_t stream);
+
+/*
+ * Merge attention results computed over disjoint key sets (split-KV combine):
+ *   lse[r] = ln sum_p exp(lse_parts[p, r]);  out[r, :] = sum_p exp(lse_parts[p, r] - lse[r]) * o_parts[p, r, :]
+ *   o_parts [n_parts, rows, d_v] fp32, lse_parts [n_parts, rows] fp32 (a part with lse = -inf
+ *   holds no keys and is ignored); out [rows, d_v] in out_dtype; lse [rows] fp32 (may be NULL).
+ * d_v must be a multiple of 4 and at most 1024.
+ */
+lkv_status lkv_merge_partials(const float* o_parts, const float* lse_parts, int n_parts,
+                              int64_t rows, int d_v, int out_dtype, void* out, float* lse,
+                              lkv_stream_t stream);
+
+/*
+ * Synchronise the current device and read the device error word (0 = none).  Returns
+ * LKV_ERR_DEVICE if it is set, LKV_ERR_CUDA if synchronisation itself failed, else LKV_OK.
+ * clear != 0 resets the word to 0 afterwards.  code_out may be NULL.
+ */
+lkv_status lkv_check_device(int32_t* code_out, int clear);
+
+/*
+ * Failure-detection self test: launches one CTA that waits on an mbarrier no thread
+ * arrives at, with the given limit.  The wait gives up, records LKV_SITE_SELFTEST in the
+ * device error word and the kernel returns; the context stays usable.
+ */
+lkv_status lkv_selftest_wait_timeout(uint64_t limit_ns, lkv_stream_t stream);
+
+/* Site codes stored in the device error word. */
+#define LKV_SITE_SELFTEST 1
+#define LKV_SITE_BAD_LENGTH 2     /* a request with L_b < s_q (append or decode)      */
+#define LKV_SITE_BAD_ROW 3        /* a cache row past cache_rows                      */
+#define LKV_SITE_WAIT_BASE 100    /* + kernel-specific wait site: a bounded wait gave up */
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LKV_H */

@@ -1,0 +1,254 @@
+"""Python binding for liblkv.so: B200 (sm_100a) decode attention over a latent / grouped KV cache.
+
+Argument marshalling only: every function passes device pointers, sizes and the current
+CUDA stream to the C ABI (include/lkv.h) and raises on a non-OK status.  PyTorch supplies
+device memory and streams; all computation runs in the library's CUDA kernels.  There is no
+fallback: if liblkv.so is missing the import fails.
+
+Functions (same names as the C entry points without the ``lkv_`` prefix):
+    mla_absorbed_decode, gqla_group_decode, gla_group_decode, latent_cache_append,
+    merge_partials, check_device, selftest_wait_timeout, plan_ranges,
+    mla_decode_workspace_size, group_decode_workspace_size
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblkv.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build it with `python latent_kv_cache_split_b200/build.py` "
+        "(the CUDA library is required; there is no fallback)")
+_lib = ctypes.CDLL(LIB_PATH)
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE = range(6)
+BF16, FP32 = 0, 1
+KIND_MLA, KIND_GQLA, KIND_GLA = 0, 1, 2
+
+_vp, _i64, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+
+
+def _sig(name, res, *args):
+    f = getattr(_lib, name)
+    f.restype = res
+    f.argtypes = list(args)
+    return f
+
+
+_lib_version = _sig("lkv_version", _i32)
+_status_string = _sig("lkv_status_string", ctypes.c_char_p, _i32)
+_plan = _sig("lkv_plan_ranges", _i32, _i32, _i32, _i32, _i32, _i32)
+_mla_ws = _sig("lkv_mla_decode_workspace_size", _sz, _i32, _i32, _i32, _i32, _i32)
+_grp_ws = _sig("lkv_group_decode_workspace_size", _sz, _i32, _i32, _i32, _i32, _i32, _i32, _i32)
+_mla = _sig("lkv_mla_absorbed_decode", _i32, _vp, _vp, _vp, _i64, _vp, _i64, _i64, _vp,
+            _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp)
+_gqla = _sig("lkv_gqla_group_decode", _i32, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _i64, _i64,
+             _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp)
+_gla = _sig("lkv_gla_group_decode", _i32, _vp, _vp, _vp, _i64, _vp, _i64, _i64, _vp,
+            _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp)
+_append = _sig("lkv_latent_cache_append", _i32, _vp, _i64, _vp, _i64, _i64, _i64, _vp,
+               _i32, _i32, _vp)
+_merge = _sig("lkv_merge_partials", _i32, _vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _vp)
+_check = _sig("lkv_check_device", _i32, ctypes.POINTER(ctypes.c_int32), _i32)
+_selftest = _sig("lkv_selftest_wait_timeout", _i32, ctypes.c_uint64, _vp)
+_segments = _sig("lkv_plan_segments", _i32, _i32, _vp, _i32, _i32, _i32, _i32, _vp, _i32)
+
+EXPORTED = ["lkv_version", "lkv_status_string", "lkv_plan_ranges", "lkv_mla_decode_workspace_size",
+            "lkv_group_decode_workspace_size", "lkv_mla_absorbed_decode", "lkv_gqla_group_decode",
+            "lkv_gla_group_decode", "lkv_latent_cache_append", "lkv_merge_partials",
+            "lkv_check_device", "lkv_selftest_wait_timeout", "lkv_plan_segments"]
+
+
+class LkvError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_status_string(status).decode()} (status {status})")
+
+
+def _ck(status: int, where: str):
+    if status != OK:
+        raise LkvError(status, where)
+
+
+def version() -> int:
+    return _lib_version()
+
+
+def status_string(status: int) -> str:
+    return _status_string(status).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("query / output tensors must be contiguous")
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _row_stride(t: torch.Tensor) -> int:
+    if t.dim() < 2 or t.stride(-1) != 1:
+        raise ValueError("cache rows must have unit stride in the last dimension")
+    return t.stride(0)
+
+
+def _num_sms(device) -> int:
+    return torch.cuda.get_device_properties(device).multi_processor_count
+
+
+def plan_ranges(kind: int, batch: int, s_q: int, groups: int, num_sms: int) -> int:
+    return _plan(kind, batch, s_q, groups, num_sms)
+
+
+def plan_segments(kind: int, cu_seqlens_host, s_q: int, groups: int, num_ranges: int):
+    """Segments the decode kernels process, as a list of
+    (range, request, unit, tile_lo, tile_hi, complete, slot, unit_id) tuples (host only)."""
+    import numpy as np
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens_host, dtype=np.int32))
+    B = cu.size - 1
+    n = _segments(kind, cu.ctypes.data, B, s_q, groups, num_ranges, None, 0)
+    if n < 0:
+        raise ValueError("bad partition arguments")
+    buf = np.zeros((max(n, 1), 8), dtype=np.int32)
+    _segments(kind, cu.ctypes.data, B, s_q, groups, num_ranges, buf.ctypes.data, n)
+    return [tuple(int(x) for x in row) for row in buf[:n]]
+
+
+def mla_decode_workspace_size(batch, s_q, h_q, r_kv, num_sms) -> int:
+    return _mla_ws(batch, s_q, h_q, r_kv, num_sms)
+
+
+def group_decode_workspace_size(kind, batch, s_q, h_q, groups, d_v, num_sms) -> int:
+    return _grp_ws(kind, batch, s_q, h_q, groups, d_v, num_sms)
+
+
+def _alloc_ws(nbytes, device):
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def mla_absorbed_decode(q_nope_abs, q_rope, ckv, kpe, cu_seqlens, scale, out=None, lse=None,
+                        workspace=None, stream=None):
+    """MLA absorbed decode.  q_nope_abs [B,s_q,h_q,r_kv], q_rope [B,s_q,h_q,d_R], ckv [rows,r_kv]
+    and kpe [rows,d_R] (unit inner stride; may be column slices of one interleaved cache),
+    cu_seqlens int32 [B+1].  Returns (out [B,s_q,h_q,r_kv], lse [B,s_q,h_q] fp32)."""
+    B, s_q, h_q, r_kv = q_nope_abs.shape
+    d_r = q_rope.shape[-1]
+    dev = q_nope_abs.device
+    if out is None:
+        out = torch.empty((B, s_q, h_q, r_kv), dtype=q_nope_abs.dtype, device=dev)
+    if lse is None:
+        lse = torch.empty((B, s_q, h_q), dtype=torch.float32, device=dev)
+    if workspace is None and q_nope_abs.dtype == torch.bfloat16:
+        workspace = _alloc_ws(mla_decode_workspace_size(B, s_q, h_q, r_kv, _num_sms(dev)), dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _contig(q_nope_abs, q_rope, out, lse)
+    _ck(_mla(_ptr(q_nope_abs), _ptr(q_rope), _ptr(ckv), _row_stride(ckv),
+             _ptr(kpe), _row_stride(kpe), ckv.shape[0], _ptr(cu_seqlens), B, s_q, h_q, r_kv, d_r,
+             float(scale), _dtype_code(q_nope_abs), _ptr(out), _ptr(lse), _ptr(workspace),
+             ws_bytes, _stream(stream)), "lkv_mla_absorbed_decode")
+    return out, lse
+
+
+def gqla_group_decode(q, q_rope, k, v, kpe, cu_seqlens, scale, out=None, lse=None,
+                      workspace=None, stream=None):
+    """GQLA grouped decode.  q [B,s_q,h_q,d_h], k / v [rows,g,d_h], kpe [rows,d_R]."""
+    B, s_q, h_q, d_h = q.shape
+    g = k.shape[1]
+    d_r = q_rope.shape[-1]
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, s_q, h_q, d_h), dtype=q.dtype, device=dev)
+    if lse is None:
+        lse = torch.empty((B, s_q, h_q), dtype=torch.float32, device=dev)
+    if workspace is None and q.dtype == torch.bfloat16:
+        workspace = _alloc_ws(group_decode_workspace_size(KIND_GQLA, B, s_q, h_q, g, d_h, _num_sms(dev)), dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    if k.stride(2) != 1 or k.stride(1) != d_h or v.stride(2) != 1 or v.stride(1) != d_h:
+        raise ValueError("k and v must be [rows, g, d_h] with contiguous groups")
+    _contig(q, q_rope, out, lse)
+    _ck(_gqla(_ptr(q), _ptr(q_rope), _ptr(k), k.stride(0), _ptr(v),
+              v.stride(0), _ptr(kpe), _row_stride(kpe), k.shape[0], _ptr(cu_seqlens), B, s_q, h_q,
+              g, d_h, d_r, float(scale), _dtype_code(q), _ptr(out), _ptr(lse), _ptr(workspace),
+              ws_bytes, _stream(stream)), "lkv_gqla_group_decode")
+    return out, lse
+
+
+def gla_group_decode(q, q_rope, clat, kpe, n_lat, cu_seqlens, scale, out=None, lse=None,
+                     workspace=None, stream=None):
+    """GLA decode.  q [B,s_q,h_q,r_g], clat [rows, n_lat*r_g], kpe [rows,d_R]."""
+    B, s_q, h_q, r_g = q.shape
+    d_r = q_rope.shape[-1]
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, s_q, h_q, r_g), dtype=q.dtype, device=dev)
+    if lse is None:
+        lse = torch.empty((B, s_q, h_q), dtype=torch.float32, device=dev)
+    if workspace is None and q.dtype == torch.bfloat16:
+        workspace = _alloc_ws(group_decode_workspace_size(KIND_GLA, B, s_q, h_q, n_lat, r_g, _num_sms(dev)), dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _contig(q, q_rope, out, lse)
+    _ck(_gla(_ptr(q), _ptr(q_rope), _ptr(clat), _row_stride(clat),
+             _ptr(kpe), _row_stride(kpe), clat.shape[0], _ptr(cu_seqlens), B, s_q, h_q, n_lat, r_g,
+             d_r, float(scale), _dtype_code(q), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes,
+             _stream(stream)), "lkv_gla_group_decode")
+    return out, lse
+
+
+def latent_cache_append(new_rows, cache, cu_seqlens, s_q, stream=None):
+    """Write row b*s_q+i of new_rows [B*s_q, ...] to cache row cu[b] + L_b - s_q + i."""
+    n = new_rows.shape[0]
+    B = cu_seqlens.numel() - 1
+    if n != B * s_q:
+        raise ValueError("new_rows must hold batch * s_q rows")
+    row_bytes = new_rows[0].numel() * new_rows.element_size()
+    _ck(_append(_ptr(new_rows), new_rows.stride(0) * new_rows.element_size(), _ptr(cache),
+                cache.stride(0) * cache.element_size(), cache.shape[0], row_bytes,
+                _ptr(cu_seqlens), B, s_q, _stream(stream)), "lkv_latent_cache_append")
+    return cache
+
+
+def merge_partials(o_parts, lse_parts, out_dtype=torch.bfloat16, out=None, lse=None, stream=None):
+    """Merge [n_parts, rows, d_v] fp32 partial outputs with their [n_parts, rows] lse."""
+    n, rows, d_v = o_parts.shape
+    dev = o_parts.device
+    if out is None:
+        out = torch.empty((rows, d_v), dtype=out_dtype, device=dev)
+    if lse is None:
+        lse = torch.empty((rows,), dtype=torch.float32, device=dev)
+    _contig(o_parts, lse_parts, out, lse)
+    _ck(_merge(_ptr(o_parts), _ptr(lse_parts), n, rows, d_v,
+               _dtype_code(out), _ptr(out), _ptr(lse), _stream(stream)), "lkv_merge_partials")
+    return out, lse
+
+
+def check_device(clear: bool = True) -> int:
+    """Synchronise and return the device error word (0 = no failure recorded)."""
+    code = ctypes.c_int32(0)
+    st = _check(ctypes.byref(code), 1 if clear else 0)
+    if st not in (OK, ERR_DEVICE):
+        raise LkvError(st, "lkv_check_device")
+    return code.value
+
+
+def selftest_wait_timeout(limit_ns: int, stream=None):
+    _ck(_selftest(int(limit_ns), _stream(stream)), "lkv_selftest_wait_timeout")

@@ -1,0 +1,181 @@
+"""The C-ABI library on the CPU: it loads, exports every symbol include/lkv.h declares, and its
+host-only logic (planning, workspace sizing, argument validation) behaves -- no GPU needed."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lkv():
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("lkv_build", os.path.join(ROOT, "latent_kv_cache_split_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    import latent_kv_cache_split_b200 as L
+    return L
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "lkv.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(lkv_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(lkv):
+    names = _declared()
+    assert len(names) >= 12
+    lib = ctypes.CDLL(lkv.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(lkv.EXPORTED) == names
+
+
+def test_version_and_status_strings(lkv):
+    assert lkv.version() >= 100
+    for s in range(6):
+        assert lkv.status_string(s)
+    assert lkv.status_string(99) == "unknown status"
+
+
+@pytest.mark.parametrize("kind,B,s_q,G,want", [
+    (0, 64, 1, 1, 64),      # MLA B=64: one range per request, no split
+    (0, 128, 1, 1, 74),     # varlen MLA: one range per CTA pair
+    (0, 128, 2, 1, 74),
+    (0, 8, 1, 1, 74),       # long context: split across every pair
+    (1, 64, 2, 8, 148),     # GQLA 512 units
+    (2, 8, 1, 2, 148),      # GLA-2 long context
+    (1, 8, 1, 8, 148),
+])
+def test_plan_ranges(lkv, kind, B, s_q, G, want):
+    assert lkv.plan_ranges(kind, B, s_q, G, 148) == want
+
+
+def test_plan_rejects_bad_input(lkv):
+    assert lkv.plan_ranges(5, 1, 1, 1, 148) == -1
+    assert lkv.plan_ranges(0, 0, 1, 1, 148) == -1
+    assert lkv.plan_ranges(0, 1, 1, 1, 1) == -1
+
+
+def test_workspace_sizes(lkv):
+    mla = lkv.mla_decode_workspace_size(64, 1, 128, 512, 148)
+    P = 64
+    assert mla >= 2 * P * 128 * 512 * 4 + 2 * P * 128 * 4 + 2 * P * 4
+    g = lkv.group_decode_workspace_size(1, 64, 2, 128, 8, 128, 148)
+    assert g >= 2 * 148 * 32 * 128 * 4
+    assert lkv.group_decode_workspace_size(3, 1, 1, 128, 8, 128, 148) == 0
+    assert lkv.group_decode_workspace_size(1, 1, 1, 128, 7, 128, 148) == 0
+
+
+def _check_partition(segs, cu, kind, s_q, G, P):
+    """Every tile of every unit is covered exactly once; slot rules hold."""
+    B = len(cu) - 1
+    upr = s_q if kind == 0 else G
+    covered = {}
+    by_range = {}
+    for (p, b, k, lo, hi, complete, slot, uid) in segs:
+        assert uid == b * upr + k
+        L = cu[b + 1] - cu[b]
+        keys = (L - s_q + k + 1) if kind == 0 else L
+        nt = -(-keys // 64)
+        assert 0 <= lo < hi <= nt
+        assert complete == int(lo == 0 and hi == nt)
+        for t in range(lo, hi):
+            assert (b, k, t) not in covered
+            covered[(b, k, t)] = p
+        by_range.setdefault(p, []).append((b, k, lo, hi, complete, slot))
+    for b in range(B):
+        L = cu[b + 1] - cu[b]
+        for k in range(upr):
+            keys = (L - s_q + k + 1) if kind == 0 else L
+            for t in range(-(-keys // 64)):
+                assert (b, k, t) in covered
+    sizes = []
+    for p, lst in by_range.items():
+        sizes.append(sum(hi - lo for (_, _, lo, hi, _, _) in lst))
+        for idx, (b, k, lo, hi, complete, slot) in enumerate(lst):
+            if complete:
+                assert slot == -1
+            else:
+                assert slot == (0 if idx == 0 else 1)
+                assert idx in (0, len(lst) - 1)
+    assert max(sizes) - min(sizes) <= 1 if len(sizes) == P else True
+
+
+@pytest.mark.parametrize("kind,s_q,G,P", [(0, 1, 1, 74), (0, 2, 1, 74), (1, 2, 8, 148), (2, 1, 2, 148),
+                                         (0, 1, 1, 3), (1, 1, 4, 5)])
+def test_partition_covers_every_tile_once(lkv, kind, s_q, G, P):
+    rng = np.random.default_rng(kind * 10 + s_q + P)
+    for trial in range(4):
+        B = int(rng.integers(1, 40))
+        lengths = rng.integers(s_q, 3000, size=B)
+        cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+        segs = lkv.plan_segments(kind, cu, s_q, G, P)
+        _check_partition(segs, cu.tolist(), kind, s_q, G, P)
+
+
+def test_partition_uniform_lengths_never_split(lkv):
+    cu = np.arange(65, dtype=np.int32) * 4096
+    segs = lkv.plan_segments(0, cu, 1, 1, 64)
+    assert len(segs) == 64 and all(s[5] == 1 for s in segs)
+
+
+def test_partition_tiny_requests_and_short_lengths(lkv):
+    cu = np.array([0, 1, 2, 3, 67], dtype=np.int32)
+    segs = lkv.plan_segments(0, cu, 1, 1, 74)
+    _check_partition(segs, cu.tolist(), 0, 1, 1, 74)
+    # L_b < s_q: that request contributes no tiles
+    cu = np.array([0, 1, 5], dtype=np.int32)
+    segs = lkv.plan_segments(0, cu, 2, 1, 4)
+    assert all(s[1] == 1 for s in segs)
+
+
+def _fake(n):
+    return ctypes.c_void_p(n)
+
+
+def test_validation_errors_need_no_gpu(lkv):
+    """Malformed calls are rejected before any CUDA call, so this runs on a CPU-only host."""
+    L = lkv
+    P16 = _fake(1 << 20)
+    cu = _fake(1 << 21)
+    args = dict(q=P16, qr=P16, ckv=P16, cs=576, kpe=P16, ks=576, rows=1000, cu=cu, B=2, s_q=1,
+                h=128, r=512, dr=64, scale=0.04, dt=0, out=P16, lse=P16, ws=P16, wsb=1 << 30, st=None)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return L._mla(a["q"], a["qr"], a["ckv"], a["cs"], a["kpe"], a["ks"], a["rows"], a["cu"],
+                      a["B"], a["s_q"], a["h"], a["r"], a["dr"], a["scale"], a["dt"], a["out"],
+                      a["lse"], a["ws"], a["wsb"], a["st"])
+    assert call(q=None) == L.ERR_INVALID_ARG
+    assert call(s_q=3) == L.ERR_UNSUPPORTED
+    assert call(B=0) == L.ERR_INVALID_ARG
+    assert call(dt=7) == L.ERR_INVALID_ARG
+    assert call(r=256) == L.ERR_UNSUPPORTED          # bf16 tensor-core path is r_kv = 512 only
+    assert call(h=64) == L.ERR_UNSUPPORTED
+    assert call(q=_fake((1 << 20) + 2)) == L.ERR_INVALID_ARG   # not 16-byte aligned
+    assert call(cs=500) == L.ERR_INVALID_ARG          # row stride shorter than r_kv
+    assert call(cs=580) == L.ERR_INVALID_ARG          # 1160-byte rows are not 16-byte aligned
+    assert call(scale=float("nan")) == L.ERR_INVALID_ARG
+    assert call(rows=1 << 31) == L.ERR_UNSUPPORTED
+    assert call(dt=1, r=2000, cs=2064) == L.ERR_UNSUPPORTED    # fp32 path limit
+    # GQLA: h_q not a multiple of g; unsupported head width
+    g = L._gqla(P16, P16, P16, 1024, P16, 1024, P16, 64, 1000, cu, 2, 2, 128, 3, 128, 64, 0.07, 0,
+                P16, P16, P16, 1 << 30, None)
+    assert g == L.ERR_INVALID_ARG
+    g = L._gqla(P16, P16, P16, 1024, P16, 1024, P16, 64, 1000, cu, 2, 2, 128, 8, 96, 64, 0.07, 0,
+                P16, P16, P16, 1 << 30, None)
+    assert g == L.ERR_UNSUPPORTED
+    g = L._gla(P16, P16, P16, 512, P16, 64, 1000, cu, 2, 1, 128, 2, 128, 64, 0.05, 0, P16, P16,
+               P16, 1 << 30, None)
+    assert g == L.ERR_UNSUPPORTED
+    # append: misaligned row size
+    assert L._append(P16, 24, P16, 24, 10, 24, cu, 1, 1, None) == L.ERR_INVALID_ARG
+    assert L._merge(P16, P16, 0, 4, 8, 0, P16, P16, None) == L.ERR_INVALID_ARG
+    assert L._merge(P16, P16, 2, 4, 6, 0, P16, P16, None) == L.ERR_INVALID_ARG
+    assert L._selftest(0, None) == L.ERR_INVALID_ARG

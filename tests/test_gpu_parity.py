@@ -1,0 +1,95 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle, element by element, on
+identical seeded inputs.  Small cases span several 64-key tiles, ragged tails, single-key
+requests and range splits; the full-size cases use the benchmark's own launch configuration
+and check every output (or every output of sampled requests where the oracle would be slow)."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from gpu_util import compare, run_lib, run_oracle, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def L(gpu):
+    import latent_kv_cache_split_b200 as lib
+    return lib
+
+
+def _run(L, gpu, w, lengths=None, requests=None, extra_rows=0):
+    d = synth.make_inputs(w, extra_rows=extra_rows, lengths=lengths)
+    out, lse = run_lib(L, to_dev(d, gpu))
+    torch.cuda.synchronize()
+    assert L.check_device() == 0
+    ref_out, ref_lse = run_oracle(d, requests=requests)
+    return compare(out, lse, ref_out, ref_lse, fp32=(w.dtype == "fp32"), requests=requests,
+                   label=w.name)
+
+
+def test_tiny_fp32_mla_full(L, gpu):
+    _run(L, gpu, synth.workload("tiny_fp32_mla"))
+
+
+@pytest.mark.parametrize("kind", ["mla", "gqla", "gla"])
+def test_fp32_path_all_forms(L, gpu, kind):
+    base = {"mla": "tiny_fp32_mla", "gqla": "gqla_g8_sq2_l8192", "gla": "long_gla2"}[kind]
+    w = synth.workload(base, dtype="fp32", batch=2, seqlen=None, len_lo=0, len_hi=0, input_std=1.0)
+    if kind == "gqla":
+        w = w.with_(h_q=16, groups=4, d_k=32, d_v=32, d_rope=16)
+    if kind == "gla":
+        w = w.with_(h_q=8, groups=2, d_k=48, d_v=48, d_rope=16)
+    _run(L, gpu, w, lengths=[77, 300])
+
+
+@pytest.mark.parametrize("s_q,lengths", [(1, [130, 64, 1]), (2, [2, 65, 200]), (1, [4096, 63, 129, 5000])])
+def test_mla_small_ragged(L, gpu, s_q, lengths):
+    w = synth.workload("mla_b64_l4096", batch=len(lengths), s_q=s_q, seqlen=None)
+    _run(L, gpu, w, lengths=lengths)
+
+
+def test_mla_b64_l4096_full(L, gpu):
+    """The benchmark workload, every output checked."""
+    _run(L, gpu, synth.workload("mla_b64_l4096"))
+
+
+@pytest.mark.parametrize("s_q", [1, 2])
+def test_mla_unscaled_stress(L, gpu, s_q):
+    w = synth.workload("mla_b64_l4096", batch=4, s_q=s_q, seqlen=1000, input_std=1.0)
+    _run(L, gpu, w)
+
+
+@pytest.mark.parametrize("s_q,lengths", [(2, [130, 7]), (1, [1, 200, 64]), (2, [8192, 2])])
+def test_gqla_small(L, gpu, s_q, lengths):
+    w = synth.workload("gqla_g8_sq2_l8192", batch=len(lengths), s_q=s_q, seqlen=None)
+    _run(L, gpu, w, lengths=lengths)
+
+
+def test_gqla_b64_l8192_sampled(L, gpu):
+    _run(L, gpu, synth.workload("gqla_g8_sq2_l8192"), requests=[0, 17, 42, 63])
+
+
+def test_gqla_unscaled_stress(L, gpu):
+    w = synth.workload("gqla_g8_sq2_l8192", batch=3, seqlen=700, input_std=1.0)
+    _run(L, gpu, w)
+
+
+@pytest.mark.parametrize("s_q,lengths", [(1, [300, 65]), (2, [129, 64, 3])])
+def test_gla_small(L, gpu, s_q, lengths):
+    w = synth.workload("long_gla2", batch=len(lengths), s_q=s_q, seqlen=None)
+    _run(L, gpu, w, lengths=lengths)
+
+
+@pytest.mark.parametrize("name,requests", [("long_gla2", [0, 5]), ("long_mla", [3]),
+                                           ("long_gqla_g8", [6])])
+def test_long_context_sampled(L, gpu, name, requests):
+    _run(L, gpu, synth.workload(name), requests=requests)
+
+
+@pytest.mark.parametrize("name", ["varlen_mla_sq1", "varlen_mla_sq2"])
+def test_varlen_sampled(L, gpu, name):
+    w = synth.workload(name)
+    lengths = synth.draw_lengths(np.random.default_rng(w.seed), w.batch, w.len_lo, w.len_hi)
+    pick = sorted({int(np.argmin(lengths)), int(np.argmax(lengths)), 0, 1, 31, 64, 100, 127})
+    _run(L, gpu, w, requests=pick)
