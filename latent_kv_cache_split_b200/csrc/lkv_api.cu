@@ -39,8 +39,8 @@ unsigned long long wait_limit_ns() {
 }
 
 constexpr size_t tc_smem_bytes(int mode) {
-  return 1024 + static_cast<size_t>(kStages) * kStageBytes +
-         (mode == MODE_MLA ? 128 * kXRow * sizeof(float) : 0);
+  return mode == MODE_MLA ? ModeCfg<MODE_MLA>::kSmemBytes
+                          : (mode == MODE_GQLA ? ModeCfg<MODE_GQLA>::kSmemBytes : ModeCfg<MODE_GLA>::kSmemBytes);
 }
 
 // Per-device one-time set-up: SM count, error-word address, kernel attributes.

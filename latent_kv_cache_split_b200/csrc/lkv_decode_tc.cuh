@@ -5,24 +5,28 @@
 //   warp 0      TMA producer: streams 64-token key/value tiles of the cache into a ring of
 //               shared-memory stages (2-D tiles of 64 rows x 64 bf16, 128-byte swizzle).
 //   warp 1      TMEM owner and UMMA issuer (one thread): S = Q K^T into TMEM, then
-//               O += P V into TMEM, with Q and P read from TMEM (A operand) and K, V from
-//               the shared-memory stage (B operand; V is read MN-major from the very same
-//               tile that served as K where K = V).
-//   warps 4..7  softmax / epilogue: thread r owns row r (TMEM lane r): loads the unit's
-//               query into TMEM, reads S, masks, runs the online softmax in the exp2 domain,
-//               writes P (bf16) into TMEM, rescales O when the running max moves, and at the
-//               end of a segment writes out / lse (or fp32 partials).
+//               O += P V into TMEM.  The non-RoPE part of Q and P are A operands read from
+//               TMEM; the RoPE part of Q is an A operand in shared memory; K and V are B
+//               operands in the stage (V is read MN-major from the very same swizzled tile
+//               that served as K where K = V).
+//   warps 4..7  softmax / epilogue: thread r owns row r (TMEM lane r): stages the unit's
+//               query, reads S, masks, runs the online softmax in the exp2 domain, writes P
+//               (bf16) into TMEM, rescales O when the running max moves, and at the end of a
+//               segment writes out / lse (or fp32 partials).
 //
-// TMEM columns: O [0, DV) | S [DV, DV+64) | P [DV+64, DV+96) | Q [DV+96, DV+96+QK/2).
+// TMEM columns: O [0, DV) | S [DV, DV+64) | P0, P1 [DV+64, DV+128) | Q [DV+128, ...).
+// P is double buffered so the softmax of tile n+1 never waits for the PV of tile n.
 //
 // MLA absorbed path (h_q = 128 heads share the latent, GQLA explainer section 2): the
 // 128 x 512 fp32 output accumulator alone fills a whole TMEM, so a CTA pair splits it:
 // rank 0 owns value columns 0..255 and computes the partial scores over latent columns
 // 0..255 plus the 64 RoPE columns; rank 1 owns value columns 256..511 and the partial
 // scores over latent columns 256..511.  The two partial score tiles are exchanged through
-// distributed shared memory and summed (identically on both CTAs, so both derive the same
-// P), and each CTA accumulates its own half of O.  Each CTA streams only the cache columns
-// it needs, so the pair reads every cache byte once.
+// distributed shared memory and summed (in the same order on both CTAs, so both derive the
+// same P), and each CTA accumulates its own half of O.  Each CTA streams only the cache
+// columns it needs, so the pair reads every cache byte once.  The softmax runs one tile
+// behind the score stream: tile n's partial scores are sent before tile n-1 is finished,
+// which hides the exchange latency.
 //
 // GQLA (g groups of expanded K_j, V_j) and GLA (latent groups, K_j = V_j) run one unit per
 // CTA: rows = heads of the group x new tokens (<= 128), padded to the M = 128 UMMA shape.
@@ -41,9 +45,10 @@ namespace lkv {
 constexpr int kBoxBytes = 64 * 64 * 2;  // one TMA box: 64 rows x 64 bf16
 constexpr int kMaxBoxes = 5;
 constexpr int kStageBytes = kMaxBoxes * kBoxBytes;  // 40 KB
-constexpr int kStages = 4;
+constexpr int kQropeBytes = 128 * 128;             // 128 rows x 64 bf16, swizzled
 constexpr int kTcThreads = 256;
-constexpr int kXRow = 68;  // floats per exchange row (64 + 4 padding against bank conflicts)
+constexpr int kXRow = 68;                          // floats per exchange row (64 + padding)
+constexpr int kXBufBytes = 128 * kXRow * 4;
 constexpr int kTmemCols = 512;
 
 enum DecodeMode { MODE_MLA = 0, MODE_GQLA = 1, MODE_GLA = 2 };
@@ -73,31 +78,36 @@ struct TcParams {
   unsigned long long wait_limit_ns;
 };
 
+template <int kMode>
+struct ModeCfg {
+  static constexpr bool kPair = (kMode == MODE_MLA);
+  static constexpr int kDV = (kMode == MODE_GQLA) ? 128 : 256;  // value columns per CTA
+  static constexpr int kStages = kPair ? 3 : 5;
+  static constexpr int kNope = (kMode == MODE_GQLA) ? 2 : 4;    // non-RoPE Q boxes (in TMEM)
+  static constexpr int kRopeBox = (kMode == MODE_GQLA) ? 2 : 4; // stage box holding k_rope
+  static constexpr int kVBox0 = (kMode == MODE_GQLA) ? 3 : 0;   // first stage box holding V
+  static constexpr int kNV = kDV / 64;
+  static constexpr uint32_t S0 = kDV, P0 = kDV + 64, Q0 = kDV + 128;
+  static constexpr size_t kSmemBytes =
+      1024 + static_cast<size_t>(kStages) * kStageBytes + kQropeBytes + (kPair ? 2 * kXBufBytes : 0);
+  __device__ static bool has_rope(uint32_t rank) { return !kPair || rank == 0; }
+  __device__ static int n_stage_boxes(uint32_t rank) { return kPair ? (rank == 0 ? 5 : 4) : 5; }
+};
+static_assert(ModeCfg<MODE_MLA>::Q0 + 32 * ModeCfg<MODE_MLA>::kNope <= kTmemCols, "TMEM budget");
+static_assert(ModeCfg<MODE_GLA>::Q0 + 32 * ModeCfg<MODE_GLA>::kNope <= kTmemCols, "TMEM budget");
+static_assert(ModeCfg<MODE_MLA>::kSmemBytes <= 232448, "shared memory budget");
+static_assert(ModeCfg<MODE_GLA>::kSmemBytes <= 232448, "shared memory budget");
+
+template <int kStagesT>
 struct __align__(16) TcSmem {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  uint64_t s_full, s_free, p_full, o_done, o_free, q_ready, x_full, x_free, drain;
+  uint64_t full[kStagesT];
+  uint64_t empty[kStagesT];
+  uint64_t s_full, s_free, o_free, q_ready, drain;
+  uint64_t p_full[2], o_done[2], x_full[2], x_free[2];
   uint32_t tmem_base;
   uint32_t abort;
   long long t_begin, t_end, unit_t0;
   int b0, k0;
-};
-
-// Per-mode constants.  rank is the CTA's rank in its pair (MLA) and 0 otherwise.
-template <int kMode>
-struct ModeCfg {
-  static constexpr int kDV = (kMode == MODE_GQLA) ? 128 : 256;  // value columns per CTA
-  __device__ static int n_qk_boxes(int rank) {
-    return kMode == MODE_MLA ? (rank == 0 ? 5 : 4) : (kMode == MODE_GQLA ? 3 : 5);
-  }
-  __device__ static int n_nope_boxes(int rank) {
-    return kMode == MODE_GQLA ? 2 : 4;
-  }
-  __device__ static int n_stage_boxes(int rank) {
-    return kMode == MODE_MLA ? (rank == 0 ? 5 : 4) : 5;
-  }
-  __device__ static int v_box0() { return kMode == MODE_GQLA ? 3 : 0; }
-  __device__ static constexpr int n_v_boxes() { return kDV / 64; }
 };
 
 __device__ __forceinline__ uint32_t tm_addr(uint32_t base, uint32_t lane_base, uint32_t col) {
@@ -112,15 +122,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                      const TcParams p) {
   using Cfg = ModeCfg<kMode>;
   constexpr int DV = Cfg::kDV;
-  constexpr uint32_t S0 = DV, P0 = DV + 64, Q0 = DV + 96;
-  constexpr bool kPair = (kMode == MODE_MLA);
+  constexpr int KS = Cfg::kStages;
+  constexpr bool kPair = Cfg::kPair;
+  constexpr uint32_t S0 = Cfg::S0, P0 = Cfg::P0, Q0 = Cfg::Q0;
 
   extern __shared__ __align__(1024) uint8_t dsmem_raw[];
-  __shared__ TcSmem sm;
+  __shared__ TcSmem<KS> sm;
   uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
   const uint32_t stage_base = smem_u32(dsm);
-  float* xbuf = reinterpret_cast<float*>(dsm + kStages * kStageBytes);  // MLA only
+  uint8_t* qrope_smem = dsm + KS * kStageBytes;
+  const uint32_t qrope_base = smem_u32(qrope_smem);
+  float* xbuf = reinterpret_cast<float*>(qrope_smem + kQropeBytes);  // MLA only: [2][128][kXRow]
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -140,24 +153,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < KS; ++s) {
       mbar_init(smem_u32(&sm.full[s]), 1);
       mbar_init(smem_u32(&sm.empty[s]), 1);
     }
     mbar_init(smem_u32(&sm.s_full), 1);
     mbar_init(smem_u32(&sm.s_free), n_sm_threads);
-    mbar_init(smem_u32(&sm.p_full), n_sm_threads);
-    mbar_init(smem_u32(&sm.o_done), 1);
     mbar_init(smem_u32(&sm.o_free), n_sm_threads);
     mbar_init(smem_u32(&sm.q_ready), n_sm_threads);
-    mbar_init(smem_u32(&sm.x_full), 128);
-    mbar_init(smem_u32(&sm.x_free), 128);
     mbar_init(smem_u32(&sm.drain), 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&sm.p_full[b]), n_sm_threads);
+      mbar_init(smem_u32(&sm.o_done[b]), 1);
+      mbar_init(smem_u32(&sm.x_full[b]), 128);
+      mbar_init(smem_u32(&sm.x_free[b]), 128);
+    }
     sm.abort = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
-    // range start (all lanes), published by lane 0
     bool malformed = false;
     SegCursor c = locate_range(sa, range, &malformed);
     if (lane == 0) {
@@ -207,8 +221,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool ok = true;
       while (ok && cur.next(sa, sg)) {
         for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
-          const int st = static_cast<int>(n % kStages);
-          const uint32_t par = static_cast<uint32_t>(((n / kStages) & 1) ^ 1);
+          const int st = static_cast<int>(n % KS);
+          const uint32_t par = static_cast<uint32_t>(((n / KS) & 1) ^ 1);
           if (!mbar_wait(smem_u32(&sm.empty[st]), par, wc, LKV_WAIT(W_EMPTY))) {
             ok = false;
             break;
@@ -236,85 +250,72 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
       // never leave copies in flight into a CTA that is about to exit
-      const long long inflight = n < kStages ? n : kStages;
-      for (long long m = n - inflight; m < n; ++m) {
-        WaitCtl dc{&sm.abort, p.err, p.wait_limit_ns};
-        uint32_t zero = 0;
-        dc.abort = &zero;  // drain ignores the abort flag but keeps the time limit
-        mbar_wait(smem_u32(&sm.full[m % kStages]), static_cast<uint32_t>((m / kStages) & 1), dc,
-                  LKV_WAIT(W_DRAIN));
-      }
+      const long long inflight = n < KS ? n : KS;
+      uint32_t zero = 0;
+      const WaitCtl dc{&zero, p.err, p.wait_limit_ns};  // ignores the abort flag, keeps the limit
+      for (long long m = n - inflight; m < n; ++m)
+        mbar_wait(smem_u32(&sm.full[m % KS]), static_cast<uint32_t>((m / KS) & 1), dc, LKV_WAIT(W_DRAIN));
     }
   } else if (warp == 1) {
     // ============================================================ UMMA issuer
     if (lane == 0) {
-      const int nqk = Cfg::n_qk_boxes(rank);
+      const bool rope = Cfg::has_rope(rank);
       const uint32_t id_qk = idesc_bf16(128, kTileN, 0, 0);
       const uint32_t id_pv = idesc_bf16(128, DV, 0, 1);
-      const uint32_t vb0 = Cfg::v_box0() * kBoxBytes;
       SegCursor cur = cur0;
       Segment sg;
       long long n = 0;   // global tile counter
       int seg = 0;       // segments started
       bool ok = true;
-      // pending PV (tile n-1)
-      bool pend = false, pend_first = false;
+      bool pend = false, pend_first = false;   // PV of tile pend_n not yet issued
       int pend_seg = 0;
       long long pend_n = 0;
       auto issue_pv = [&]() -> bool {
-        const int st = static_cast<int>(pend_n % kStages);
-        if (!mbar_wait(smem_u32(&sm.p_full), static_cast<uint32_t>(pend_n & 1), wc, LKV_WAIT(W_PFULL)))
+        const int pb = static_cast<int>(pend_n & 1);
+        if (!mbar_wait(smem_u32(&sm.p_full[pb]), static_cast<uint32_t>((pend_n >> 1) & 1), wc,
+                       LKV_WAIT(W_PFULL)))
           return false;
-        if (pend_first && pend_seg > 0) {
-          if (!mbar_wait(smem_u32(&sm.o_free), static_cast<uint32_t>((pend_seg - 1) & 1), wc,
-                         LKV_WAIT(W_OFREE)))
-            return false;
-        }
+        if (pend_first && pend_seg > 0 &&
+            !mbar_wait(smem_u32(&sm.o_free), static_cast<uint32_t>((pend_seg - 1) & 1), wc, LKV_WAIT(W_OFREE)))
+          return false;
         tc_fence_after();
-        const uint32_t vbase = stage_base + st * kStageBytes + vb0;
+        const uint32_t vbase = stage_base + static_cast<uint32_t>(pend_n % KS) * kStageBytes + Cfg::kVBox0 * kBoxBytes;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           const uint64_t bd = sdesc_sw128(vbase + kk * 2048, kBoxBytes, 1024);
-          umma_ts(tbase, tbase + P0 + kk * 8, bd, id_pv, (pend_first && kk == 0) ? 0u : 1u);
+          umma_ts(tbase, tbase + P0 + 32 * pb + kk * 8, bd, id_pv, (pend_first && kk == 0) ? 0u : 1u);
         }
-        umma_commit(smem_u32(&sm.o_done));
-        umma_commit(smem_u32(&sm.empty[st]));
+        umma_commit(smem_u32(&sm.o_done[pb]));
+        umma_commit(smem_u32(&sm.empty[pend_n % KS]));
         pend = false;
         return true;
       };
       while (ok && cur.next(sa, sg)) {
         for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
-          const int st = static_cast<int>(n % kStages);
-          if (!mbar_wait(smem_u32(&sm.full[st]), static_cast<uint32_t>((n / kStages) & 1), wc,
-                         LKV_WAIT(W_FULL))) {
+          const int st = static_cast<int>(n % KS);
+          if (!mbar_wait(smem_u32(&sm.full[st]), static_cast<uint32_t>((n / KS) & 1), wc, LKV_WAIT(W_FULL)) ||
+              (n > 0 && !mbar_wait(smem_u32(&sm.s_free), static_cast<uint32_t>((n - 1) & 1), wc, LKV_WAIT(W_SFREE))) ||
+              (t == sg.tile_lo &&
+               !mbar_wait(smem_u32(&sm.q_ready), static_cast<uint32_t>(seg & 1), wc, LKV_WAIT(W_QREADY)))) {
             ok = false;
             break;
-          }
-          if (n > 0 && !mbar_wait(smem_u32(&sm.s_free), static_cast<uint32_t>((n - 1) & 1), wc,
-                                  LKV_WAIT(W_SFREE))) {
-            ok = false;
-            break;
-          }
-          const bool first = (t == sg.tile_lo);
-          if (first) {
-            // the previous segment's last PV goes first: its epilogue precedes the new Q
-            if (pend && !issue_pv()) {
-              ok = false;
-              break;
-            }
-            if (!mbar_wait(smem_u32(&sm.q_ready), static_cast<uint32_t>(seg & 1), wc,
-                           LKV_WAIT(W_QREADY))) {
-              ok = false;
-              break;
-            }
           }
           tc_fence_after();
           const uint32_t kb = stage_base + st * kStageBytes;
-          for (int bx = 0; bx < nqk; ++bx) {
+#pragma unroll
+          for (int bx = 0; bx < Cfg::kNope; ++bx) {
 #pragma unroll
             for (int kk = 0; kk < 4; ++kk) {
               const uint64_t bd = sdesc_sw128(kb + bx * kBoxBytes + kk * 32, 16, 1024);
               umma_ts(tbase + S0, tbase + Q0 + bx * 32 + kk * 8, bd, id_qk, (bx | kk) ? 1u : 0u);
+            }
+          }
+          if (rope) {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = sdesc_sw128(qrope_base + kk * 32, 16, 1024);
+              const uint64_t bd = sdesc_sw128(kb + Cfg::kRopeBox * kBoxBytes + kk * 32, 16, 1024);
+              umma_ss(tbase + S0, ad, bd, id_qk, 1u);
             }
           }
           umma_commit(smem_u32(&sm.s_full));
@@ -323,7 +324,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             break;
           }
           pend = true;
-          pend_first = first;
+          pend_first = (t == sg.tile_lo);
           pend_seg = seg;
           pend_n = n;
         }
@@ -332,9 +333,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (ok && pend) issue_pv();
       // all tcgen05 work of this thread done before TMEM is released
       umma_commit(smem_u32(&sm.drain));
-      WaitCtl dc{&sm.abort, p.err, p.wait_limit_ns};
       uint32_t zero = 0;
-      dc.abort = &zero;
+      const WaitCtl dc{&zero, p.err, p.wait_limit_ns};
       mbar_wait(smem_u32(&sm.drain), 0, dc, LKV_WAIT(W_DRAIN));
     }
   } else if (warp >= 4 && (warp - 4) < n_sm_warps) {
@@ -342,15 +342,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int r = tid - 128;                 // row == TMEM lane
     const uint32_t lb = static_cast<uint32_t>((warp & 3) * 32);
     const bool row_ok = r < p.R;
-    const int nqk = Cfg::n_qk_boxes(rank);
-    const int nnope = Cfg::n_nope_boxes(rank);
     const uint32_t peer = rank ^ 1u;
-    const uint32_t x_remote = kPair ? map_to_peer(smem_u32(xbuf + r * kXRow), peer) : 0u;
-    const uint32_t xfull_remote = kPair ? map_to_peer(smem_u32(&sm.x_full), peer) : 0u;
-    const uint32_t xfree_remote = kPair ? map_to_peer(smem_u32(&sm.x_free), peer) : 0u;
+    uint32_t x_remote[2] = {0u, 0u}, xfull_remote[2] = {0u, 0u}, xfree_remote[2] = {0u, 0u};
+    if (kPair) {
+      for (int b = 0; b < 2; ++b) {
+        x_remote[b] = map_to_peer(smem_u32(xbuf + (b * 128 + r) * kXRow), peer);
+        xfull_remote[b] = map_to_peer(smem_u32(&sm.x_full[b]), peer);
+        xfree_remote[b] = map_to_peer(smem_u32(&sm.x_free[b]), peer);
+      }
+    }
     const int col_base = kPair ? 256 * static_cast<int>(rank) : 0;
 
-    // (query token, head) of this row in a unit
     // every lane of a softmax warp takes the same branch after a wait (tcgen05.ld/st are
     // warp-collective), so a wait that gives up in one lane ends the loop in all of them
     auto wait_all = [&](uint32_t bar, uint32_t par, int site) -> bool {
@@ -359,6 +361,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     auto wait_all_cl = [&](uint32_t bar, uint32_t par, int site) -> bool {
       return __all_sync(0xffffffffu, mbar_wait<true>(bar, par, wc, site)) != 0;
     };
+    // (query token, head) of this row in a unit
     auto row_map = [&](const Segment& sg, int& i, int& h) {
       if (kPair) {
         i = sg.k;
@@ -368,16 +371,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         h = sg.k * p.hpg + (r % p.hpg);
       }
     };
+    // Stage the unit's query: non-RoPE part into TMEM (A operand), RoPE part into the
+    // swizzled shared-memory A operand.
     auto load_q = [&](const Segment& sg) {
       int i, h;
       row_map(sg, i, h);
       const size_t qrow = (static_cast<size_t>(sg.b) * p.s_q + i) * p.h_q + h;
-      for (int bx = 0; bx < nqk; ++bx) {
+#pragma unroll 1
+      for (int bx = 0; bx < Cfg::kNope; ++bx) {
         uint32_t w[32];
         if (row_ok) {
-          const uint4* src = (bx < nnope)
-                                 ? reinterpret_cast<const uint4*>(p.q_nope + qrow * p.dq + col_base + 64 * bx)
-                                 : reinterpret_cast<const uint4*>(p.q_rope + qrow * 64);
+          const uint4* src = reinterpret_cast<const uint4*>(p.q_nope + qrow * p.dq + col_base + 64 * bx);
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
             const uint4 x = __ldg(src + v);
@@ -392,158 +396,114 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tmem_st32(tm_addr(tbase, lb, Q0 + bx * 32), w);
       }
+      if (Cfg::has_rope(rank)) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + qrow * 64);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 x = row_ok ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(qrope_smem + r * 128 + ((c ^ (r & 7)) << 4)) = x;
+        }
+        fence_proxy_async_smem();
+      }
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.q_ready));
     };
 
-    SegCursor cur = cur0;
-    Segment sg, nxt;
-    bool have = cur.next(sa, sg);
-    bool ok = true;
-    long long n = 0;
-    int seg = 0;
-    if (have) load_q(sg);
-    while (ok && have) {
-      bool have_next = false;
+    float m_run = -INFINITY, l_run = 0.f;
+    // Softmax of one tile whose full scores are in s[]; writes P(n); runs the segment
+    // epilogue after the unit's last tile of this range.
+    auto process = [&](float (&s)[64], const Segment& sg, int t, long long n) -> bool {
       int qi, qh;
       row_map(sg, qi, qh);
+      if (t == sg.tile_lo) {
+        m_run = -INFINITY;
+        l_run = 0.f;
+      }
       const int lim = kPair ? sg.keys : (sg.L - p.s_q + qi + 1);  // keys visible to this row
-      float m_run = -INFINITY, l_run = 0.f;
-      for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
-        if (!wait_all(smem_u32(&sm.s_full), static_cast<uint32_t>(n & 1), LKV_WAIT(W_SFULL))) {
-          ok = false;
-          break;
+      const int key0 = t * kTileN;
+      float mx = -INFINITY;
+      if (key0 + kTileN <= lim) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          s[c] *= p.sl2;
+          mx = fmaxf(mx, s[c]);
         }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 64; ++c) {
+          s[c] = (key0 + c < lim) ? s[c] * p.sl2 : -INFINITY;
+          mx = fmaxf(mx, s[c]);
+        }
+      }
+      // lazy rescale: keep the running max unless the tile max exceeds it by 2^8
+      bool rescale = false;
+      float m_new = m_run;
+      if (mx > m_run + 8.f) {
+        m_new = mx;
+        rescale = (m_run != -INFINITY);
+      }
+      const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.f;
+      const float msub = (m_new == -INFINITY) ? 0.f : m_new;
+      uint32_t pw[32];
+      float sum = 0.f;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float e0 = ex2_approx(s[2 * c] - msub);
+        const float e1 = ex2_approx(s[2 * c + 1] - msub);
+        sum += e0 + e1;
+        pw[c] = pack_bf16x2(e0, e1);
+      }
+      l_run = l_run * alpha + sum;
+      m_run = m_new;
+      const int pb = static_cast<int>(n & 1);
+      // P buffer pb was last read by PV(n-2)
+      if (n >= 2 && !wait_all(smem_u32(&sm.o_done[pb]), static_cast<uint32_t>(((n - 2) >> 1) & 1), LKV_WAIT(W_ODONE)))
+        return false;
+      if (__any_sync(0xffffffffu, rescale) && t != sg.tile_lo) {
+        // O holds this segment's tiles up to n-1: wait for PV(n-1), then scale in place
+        if (!wait_all(smem_u32(&sm.o_done[pb ^ 1]), static_cast<uint32_t>(((n - 1) >> 1) & 1), LKV_WAIT(W_ODONE)))
+          return false;
         tc_fence_after();
-        float sv[64];
-        {
-          uint32_t a[32];
-          tmem_ld32(tm_addr(tbase, lb, S0), a);
-          uint32_t b2[32];
-          tmem_ld32(tm_addr(tbase, lb, S0 + 32), b2);
+#pragma unroll 1
+        for (int c = 0; c < DV; c += 32) {
+          uint32_t o[32];
+          tmem_ld32(tm_addr(tbase, lb, c), o);
           tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            sv[c] = __uint_as_float(a[c]);
-            sv[32 + c] = __uint_as_float(b2[c]);
-          }
+          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          tmem_st32(tm_addr(tbase, lb, c), o);
         }
-        tc_fence_before();
-        mbar_arrive(smem_u32(&sm.s_free));
-        if (t == sg.tile_hi - 1) {
-          // QK of this tile is done, so the Q columns are free: stage the next unit's query
-          have_next = cur.next(sa, nxt);
-          if (have_next) load_q(nxt);
-        }
-        if (kPair) {
-          // exchange partial scores with the peer CTA
-          if (n > 0 && !wait_all_cl(smem_u32(&sm.x_free), static_cast<uint32_t>((n - 1) & 1),
-                                    LKV_WAIT(W_XFREE))) {
-            ok = false;
-            break;
-          }
-#pragma unroll
-          for (int c = 0; c < 64; c += 4) st_cluster_v4(x_remote + c * 4, sv[c], sv[c + 1], sv[c + 2], sv[c + 3]);
-          mbar_arrive_remote(xfull_remote);
-          if (!wait_all_cl(smem_u32(&sm.x_full), static_cast<uint32_t>(n & 1), LKV_WAIT(W_XFULL))) {
-            ok = false;
-            break;
-          }
-          const float4* xr = reinterpret_cast<const float4*>(xbuf + r * kXRow);
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float4 x = xr[c];
-            sv[4 * c] += x.x;
-            sv[4 * c + 1] += x.y;
-            sv[4 * c + 2] += x.z;
-            sv[4 * c + 3] += x.w;
-          }
-          mbar_arrive_remote(xfree_remote);
-        }
-        // scale, mask, tile max (exp2 domain)
-        const int key0 = t * kTileN;
-        float mx = -INFINITY;
-        if (key0 + kTileN <= lim) {
-#pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            sv[c] *= p.sl2;
-            mx = fmaxf(mx, sv[c]);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            sv[c] = (key0 + c < lim) ? sv[c] * p.sl2 : -INFINITY;
-            mx = fmaxf(mx, sv[c]);
-          }
-        }
-        // lazy rescale: keep the running max unless the tile max exceeds it by 2^8
-        bool rescale = false;
-        float m_new = m_run;
-        if (mx > m_run + 8.f) {
-          m_new = mx;
-          rescale = (m_run != -INFINITY);
-        }
-        const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.f;
-        const float msub = (m_new == -INFINITY) ? 0.f : m_new;
-        uint32_t pw[32];
-        float sum = 0.f;
-#pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float e0 = ex2_approx(sv[2 * c] - msub);
-          const float e1 = ex2_approx(sv[2 * c + 1] - msub);
-          sum += e0 + e1;
-          pw[c] = pack_bf16x2(e0, e1);
-        }
-        l_run = l_run * alpha + sum;
-        m_run = m_new;
-        // the previous PV must be done before P is overwritten or O rescaled
-        if (n > 0 && !wait_all(smem_u32(&sm.o_done), static_cast<uint32_t>((n - 1) & 1),
-                               LKV_WAIT(W_ODONE))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        if (rescale && t != sg.tile_lo) {
-          for (int c = 0; c < DV; c += 32) {
-            uint32_t o[32];
-            tmem_ld32(tm_addr(tbase, lb, c), o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-            tmem_st32(tm_addr(tbase, lb, c), o);
-          }
-        }
-        tmem_st32(tm_addr(tbase, lb, P0), pw);
-        if (key0 + kTileN > sg.keys) {
-          // Rows past the unit's last key belong to another request or to unwritten cache:
-          // their P is 0, but 0 * NaN would still poison O, so clear those V rows first.
-          const int first = sg.keys - key0;
-          const int per_box = (kTileN - first) * 8;  // 16-byte chunks per V box
-          uint8_t* vb = dsm + (n % kStages) * kStageBytes + Cfg::v_box0() * kBoxBytes;
-          for (int idx = r; idx < per_box * Cfg::n_v_boxes(); idx += n_sm_threads) {
-            const int bx = idx / per_box, rem = idx % per_box;
-            *reinterpret_cast<uint4*>(vb + bx * kBoxBytes + (first + rem / 8) * 128 + (rem % 8) * 16) =
-                make_uint4(0u, 0u, 0u, 0u);
-          }
-          fence_proxy_async_smem();
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(smem_u32(&sm.p_full));
       }
-      if (!ok) break;
+      tc_fence_after();
+      tmem_st32(tm_addr(tbase, lb, P0 + 32 * pb), pw);
+      if (key0 + kTileN > sg.keys) {
+        // Rows past the unit's last key belong to another request or to unwritten cache:
+        // their P is 0, but 0 * NaN would still poison O, so clear those V rows first.
+        const int first = sg.keys - key0;
+        const int per_box = (kTileN - first) * 8;  // 16-byte chunks per V box
+        uint8_t* vb = dsm + (n % KS) * kStageBytes + Cfg::kVBox0 * kBoxBytes;
+        for (int idx = r; idx < per_box * Cfg::kNV; idx += n_sm_threads) {
+          const int bx = idx / per_box, rem = idx % per_box;
+          *reinterpret_cast<uint4*>(vb + bx * kBoxBytes + (first + rem / 8) * 128 + (rem % 8) * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_proxy_async_smem();
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(smem_u32(&sm.p_full[pb]));
+      if (t != sg.tile_hi - 1) return true;
       // ---------------------------------------------------------- segment epilogue
-      if (!wait_all(smem_u32(&sm.o_done), static_cast<uint32_t>((n - 1) & 1), LKV_WAIT(W_ODONE))) {
-        ok = false;
-        break;
-      }
+      if (!wait_all(smem_u32(&sm.o_done[pb]), static_cast<uint32_t>((n >> 1) & 1), LKV_WAIT(W_ODONE)))
+        return false;
       tc_fence_after();
       const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
       const float lse_v = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
       const size_t orow = (static_cast<size_t>(sg.b) * p.s_q + qi) * p.h_q + qh;
       if (sg.complete) {
         __nv_bfloat16* dst = p.out + orow * p.dv_total + col_base;
+#pragma unroll 1
         for (int c = 0; c < DV; c += 32) {
           uint32_t o[32];
           tmem_ld32(tm_addr(tbase, lb, c), o);
@@ -565,6 +525,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       } else {
         const size_t prow = static_cast<size_t>(2 * range + sg.slot) * p.rmax + r;
         float* dst = p.part_o + prow * p.dv_total + col_base;
+#pragma unroll 1
         for (int c = 0; c < DV; c += 32) {
           uint32_t o[32];
           tmem_ld32(tm_addr(tbase, lb, c), o);
@@ -582,9 +543,115 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(smem_u32(&sm.o_free));
-      ++seg;
-      have = have_next;
-      if (have) sg = nxt;
+      return true;
+    };
+
+    SegCursor cur = cur0;
+    Segment sgA, nx;
+    bool haveA = cur.next(sa, sgA);
+    int tA = haveA ? sgA.tile_lo : 0;
+    long long nA = 0;
+    // tile waiting for the peer's partial scores (MLA only)
+    float prev[64];
+    Segment sgB;
+    int tB = 0;
+    long long nB = 0;
+    bool haveB = false;
+    bool ok = true;
+    if (haveA) load_q(sgA);
+    while (ok && (haveA || haveB)) {
+      float cs[64];
+      bool gotA = false;
+      Segment sgAc;
+      int tAc = 0;
+      long long nAc = 0;
+      if (haveA) {
+        if (!wait_all(smem_u32(&sm.s_full), static_cast<uint32_t>(nA & 1), LKV_WAIT(W_SFULL))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        {
+          uint32_t a[32], b2[32];
+          tmem_ld32(tm_addr(tbase, lb, S0), a);
+          tmem_ld32(tm_addr(tbase, lb, S0 + 32), b2);
+          tmem_wait_ld();
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            cs[c] = __uint_as_float(a[c]);
+            cs[32 + c] = __uint_as_float(b2[c]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(smem_u32(&sm.s_free));
+        const bool last = (tA == sgA.tile_hi - 1);
+        bool have_nx = false;
+        if (last) {
+          // QK of this tile is done, so the query operands are free: stage the next unit's
+          have_nx = cur.next(sa, nx);
+          if (have_nx) load_q(nx);
+        }
+        if (kPair) {
+          const int xb = static_cast<int>(nA & 1);
+          if (nA >= 2 && !wait_all_cl(smem_u32(&sm.x_free[xb]), static_cast<uint32_t>(((nA - 2) >> 1) & 1),
+                                      LKV_WAIT(W_XFREE))) {
+            ok = false;
+            break;
+          }
+#pragma unroll
+          for (int c = 0; c < 64; c += 4) st_cluster_v4(x_remote[xb] + c * 4, cs[c], cs[c + 1], cs[c + 2], cs[c + 3]);
+          mbar_arrive_remote(xfull_remote[xb]);
+        }
+        gotA = true;
+        sgAc = sgA;
+        tAc = tA;
+        nAc = nA;
+        ++nA;
+        ++tA;
+        if (last) {
+          haveA = have_nx;
+          if (haveA) {
+            sgA = nx;
+            tA = sgA.tile_lo;
+          }
+        }
+      }
+      if (kPair) {
+        if (haveB) {
+          const int xb = static_cast<int>(nB & 1);
+          if (!wait_all_cl(smem_u32(&sm.x_full[xb]), static_cast<uint32_t>((nB >> 1) & 1), LKV_WAIT(W_XFULL))) {
+            ok = false;
+            break;
+          }
+          const float4* xr = reinterpret_cast<const float4*>(xbuf + (xb * 128 + r) * kXRow);
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const float4 x = xr[c];
+            prev[4 * c] += x.x;
+            prev[4 * c + 1] += x.y;
+            prev[4 * c + 2] += x.z;
+            prev[4 * c + 3] += x.w;
+          }
+          mbar_arrive_remote(xfree_remote[xb]);
+          if (!process(prev, sgB, tB, nB)) {
+            ok = false;
+            break;
+          }
+        }
+        haveB = gotA;
+        if (gotA) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) prev[c] = cs[c];
+          sgB = sgAc;
+          tB = tAc;
+          nB = nAc;
+        }
+      } else if (gotA) {
+        if (!process(cs, sgAc, tAc, nAc)) {
+          ok = false;
+          break;
+        }
+      }
     }
   }
 
