@@ -149,6 +149,34 @@ lkv_status lkv_gla_group_decode(const void* q, const void* q_rope, const void* c
                                 lkv_stream_t stream);
 
 /*
+ * GQLA grouped decode that allocates nothing and takes no workspace.
+ *
+ * No counterpart on the source pages.  It serves callers that cannot allocate device memory
+ * on the decode path: hosts without a device allocator of their own, and serving loops that
+ * reserve all device memory up front and must not call cudaMalloc (which may also synchronise
+ * the device) per step.  Arguments and results are those of lkv_gqla_group_decode without the
+ * workspace.  The split-KV partials go to one fixed device array inside the library of
+ * LKV_STATIC_SCRATCH_BYTES (8 MiB), which every GPU that loads the library keeps until the
+ * process exits.
+ *   - A shape whose workspace (lkv_group_decode_workspace_size) exceeds that size is rejected
+ *     with LKV_ERR_WORKSPACE before anything is launched.
+ *   - All calls on a device share the array and it keeps the last call's contents.  The kernel
+ *     writes everything it later reads, so nothing needs clearing, but two calls that overlap
+ *     on the GPU (e.g. unordered streams) race on it.
+ *   - The first call on a device looks up the array's device address with that device
+ *     current; make that first call before any stream capture begins.
+ *   - It calls no cudaMalloc, no cudaFree and no allocating library routine.
+ */
+#define LKV_STATIC_SCRATCH_BYTES (8u << 20)
+lkv_status lkv_gqla_group_decode_noalloc(const void* q, const void* q_rope, const void* k,
+                                         int64_t k_row_stride, const void* v,
+                                         int64_t v_row_stride, const void* kpe,
+                                         int64_t kpe_row_stride, int64_t cache_rows,
+                                         const int32_t* cu_seqlens, int batch, int s_q, int h_q,
+                                         int g, int d_h, int d_rope, float scale, int dtype,
+                                         void* out, float* lse, lkv_stream_t stream);
+
+/*
  * Cache append: copy the s_q new rows of every request into the cache.
  * Row b*s_q + i of new_rows goes to cache row cu_seqlens[b] + L_b - s_q + i (the new tokens
  * are the tail of each request's run; source: GQLA explainer, section 2 -- the cache holds

@@ -51,6 +51,8 @@ _gqla = _sig("lkv_gqla_group_decode", _i32, _vp, _vp, _vp, _i64, _vp, _i64, _vp,
              _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp)
 _gla = _sig("lkv_gla_group_decode", _i32, _vp, _vp, _vp, _i64, _vp, _i64, _i64, _vp,
             _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp)
+_gqla_noalloc = _sig("lkv_gqla_group_decode_noalloc", _i32, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _i64,
+                     _i64, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp)
 _append = _sig("lkv_latent_cache_append", _i32, _vp, _i64, _vp, _i64, _i64, _i64, _vp,
                _i32, _i32, _vp)
 _merge = _sig("lkv_merge_partials", _i32, _vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _vp)
@@ -61,7 +63,8 @@ _segments = _sig("lkv_plan_segments", _i32, _i32, _vp, _i32, _i32, _i32, _i32, _
 EXPORTED = ["lkv_version", "lkv_status_string", "lkv_plan_ranges", "lkv_mla_decode_workspace_size",
             "lkv_group_decode_workspace_size", "lkv_mla_absorbed_decode", "lkv_gqla_group_decode",
             "lkv_gla_group_decode", "lkv_latent_cache_append", "lkv_merge_partials",
-            "lkv_check_device", "lkv_selftest_wait_timeout", "lkv_plan_segments"]
+            "lkv_check_device", "lkv_selftest_wait_timeout", "lkv_plan_segments",
+            "lkv_gqla_group_decode_noalloc"]
 
 
 class LkvError(RuntimeError):
@@ -190,6 +193,30 @@ def gqla_group_decode(q, q_rope, k, v, kpe, cu_seqlens, scale, out=None, lse=Non
               v.stride(0), _ptr(kpe), _row_stride(kpe), k.shape[0], _ptr(cu_seqlens), B, s_q, h_q,
               g, d_h, d_r, float(scale), _dtype_code(q), _ptr(out), _ptr(lse), _ptr(workspace),
               ws_bytes, _stream(stream)), "lkv_gqla_group_decode")
+    return out, lse
+
+
+def gqla_group_decode_noalloc(q, q_rope, k, v, kpe, cu_seqlens, scale, out=None, lse=None,
+                              stream=None):
+    """GQLA grouped decode without a workspace: for callers that cannot allocate device memory
+    per call.  The library keeps one fixed 8 MiB device scratch array per GPU instead; calls
+    that overlap on the GPU race on it, and shapes needing more scratch raise LkvError
+    (ERR_WORKSPACE).  `out` and `lse` are still caller-provided (allocated here if omitted)."""
+    B, s_q, h_q, d_h = q.shape
+    g = k.shape[1]
+    d_r = q_rope.shape[-1]
+    dev = q.device
+    if out is None:
+        out = torch.empty((B, s_q, h_q, d_h), dtype=q.dtype, device=dev)
+    if lse is None:
+        lse = torch.empty((B, s_q, h_q), dtype=torch.float32, device=dev)
+    if k.stride(2) != 1 or k.stride(1) != d_h or v.stride(2) != 1 or v.stride(1) != d_h:
+        raise ValueError("k and v must be [rows, g, d_h] with contiguous groups")
+    _contig(q, q_rope, out, lse)
+    _ck(_gqla_noalloc(_ptr(q), _ptr(q_rope), _ptr(k), k.stride(0), _ptr(v), v.stride(0), _ptr(kpe),
+                      _row_stride(kpe), k.shape[0], _ptr(cu_seqlens), B, s_q, h_q, g, d_h, d_r,
+                      float(scale), _dtype_code(q), _ptr(out), _ptr(lse), _stream(stream)),
+        "lkv_gqla_group_decode_noalloc")
     return out, lse
 
 

@@ -513,6 +513,32 @@ lkv_status lkv_gla_group_decode(const void* q, const void* q_rope, const void* c
   return run_tc(L, *d, s);
 }
 
+// Fixed scratch for lkv_gqla_group_decode_noalloc.  In host code this name is only a
+// stand-in for the device symbol; its device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_lkv_static_scratch[LKV_STATIC_SCRATCH_BYTES];
+static void* g_static_scratch_addr[kMaxDevices] = {};
+
+lkv_status lkv_gqla_group_decode_noalloc(const void* q, const void* q_rope, const void* k,
+                                         int64_t k_row_stride, const void* v,
+                                         int64_t v_row_stride, const void* kpe,
+                                         int64_t kpe_row_stride, int64_t cache_rows,
+                                         const int32_t* cu_seqlens, int batch, int s_q, int h_q,
+                                         int g, int d_h, int d_rope, float scale, int dtype,
+                                         void* out, float* lse, lkv_stream_t stream) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LKV_ERR_CUDA;
+  if (!g_static_scratch_addr[dev]) {
+    // once per device, with that device current (first call; before any stream capture)
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_lkv_static_scratch) != cudaSuccess || !ptr) return LKV_ERR_CUDA;
+    g_static_scratch_addr[dev] = ptr;
+  }
+  // the regular entry point rejects a shape whose workspace exceeds the array (LKV_ERR_WORKSPACE)
+  return lkv_gqla_group_decode(q, q_rope, k, k_row_stride, v, v_row_stride, kpe, kpe_row_stride,
+                               cache_rows, cu_seqlens, batch, s_q, h_q, g, d_h, d_rope, scale, dtype,
+                               out, lse, g_static_scratch_addr[dev], LKV_STATIC_SCRATCH_BYTES, stream);
+}
+
 lkv_status lkv_latent_cache_append(const void* new_rows, int64_t new_row_stride_bytes,
                                    void* cache, int64_t cache_row_stride_bytes,
                                    int64_t cache_rows, int64_t row_bytes,
