@@ -76,7 +76,7 @@ int lkv_plan_ranges(int kind, int batch, int s_q, int groups, int num_sms);
  * Host-only view of the same partition (no CUDA call): for host-side cu_seqlens_host [batch+1]
  * and `num_ranges` ranges, writes one record of 8 int32 per segment, in processing order:
  *   (range, request, unit, tile_lo, tile_hi, complete, slot, unit_id)
- * tiles are 64 keys; slot is -1 for a segment that covers its whole unit, else the partial
+ * tiles are 64 keys (MLA, GLA) or 128 keys (GQLA); slot is -1 for a segment that covers its whole unit, else the partial
  * slot (0 = first segment of its range, 1 = last).  Returns the number of segments (records
  * past max_out are counted but not written), or -1 on bad input.
  */

@@ -209,6 +209,7 @@ int lkv_plan_segments(int kind, const int32_t* cu_seqlens_host, int batch, int s
   a.units_per_req = kind == 0 ? s_q : groups;
   a.per_query_units = kind == 0 ? 1 : 0;
   a.P = num_ranges;
+  a.tile = kind == 0 ? ModeCfg<MODE_MLA>::kTile : (kind == 1 ? ModeCfg<MODE_GQLA>::kTile : ModeCfg<MODE_GLA>::kTile);
   int n = 0;
   for (int p = 0; p < num_ranges; ++p) {
     SegCursor c = locate_range_host(a, p);
@@ -300,8 +301,9 @@ lkv_status lkv_mla_absorbed_decode(const void* q_nope_abs, const void* q_rope, c
   if (!workspace || !al16(workspace) || workspace_bytes < w.total) return LKV_ERR_WORKSPACE;
   TcLaunch L;
   L.mode = MODE_MLA;
-  if (!make_tmap_bf16(&L.map_a, ckv, r_kv, cache_rows, ckv_row_stride * 2, 64, kTileN) ||
-      !make_tmap_bf16(&L.map_r, kpe, d_rope, cache_rows, kpe_row_stride * 2, 64, kTileN))
+  constexpr int TN = ModeCfg<MODE_MLA>::kTile;
+  if (!make_tmap_bf16(&L.map_a, ckv, r_kv, cache_rows, ckv_row_stride * 2, 64, TN) ||
+      !make_tmap_bf16(&L.map_r, kpe, d_rope, cache_rows, kpe_row_stride * 2, 64, TN))
     return LKV_ERR_CUDA;
   L.map_v = L.map_a;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -392,9 +394,10 @@ lkv_status lkv_gqla_group_decode(const void* q, const void* q_rope, const void* 
   TcLaunch L;
   L.mode = MODE_GQLA;
   const uint64_t width = static_cast<uint64_t>(g) * d_h;
-  if (!make_tmap_bf16(&L.map_a, k, width, cache_rows, k_row_stride * 2, 64, kTileN) ||
-      !make_tmap_bf16(&L.map_v, v, width, cache_rows, v_row_stride * 2, 64, kTileN) ||
-      !make_tmap_bf16(&L.map_r, kpe, d_rope, cache_rows, kpe_row_stride * 2, 64, kTileN))
+  constexpr int TN = ModeCfg<MODE_GQLA>::kTile;
+  if (!make_tmap_bf16(&L.map_a, k, width, cache_rows, k_row_stride * 2, 64, TN) ||
+      !make_tmap_bf16(&L.map_v, v, width, cache_rows, v_row_stride * 2, 64, TN) ||
+      !make_tmap_bf16(&L.map_r, kpe, d_rope, cache_rows, kpe_row_stride * 2, 64, TN))
     return LKV_ERR_CUDA;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   TcParams& p = L.p;
@@ -481,8 +484,8 @@ lkv_status lkv_gla_group_decode(const void* q, const void* q_rope, const void* c
   TcLaunch L;
   L.mode = MODE_GLA;
   if (!make_tmap_bf16(&L.map_a, clat, static_cast<uint64_t>(n_lat) * r_g, cache_rows,
-                      clat_row_stride * 2, 64, kTileN) ||
-      !make_tmap_bf16(&L.map_r, kpe, d_rope, cache_rows, kpe_row_stride * 2, 64, kTileN))
+                      clat_row_stride * 2, 64, ModeCfg<MODE_GLA>::kTile) ||
+      !make_tmap_bf16(&L.map_r, kpe, d_rope, cache_rows, kpe_row_stride * 2, 64, ModeCfg<MODE_GLA>::kTile))
     return LKV_ERR_CUDA;
   L.map_v = L.map_a;
   uint8_t* ws = static_cast<uint8_t*>(workspace);

@@ -2,8 +2,9 @@
 //
 // One persistent CTA (MLA: one CTA pair, a thread-block cluster of 2) per work range
 // (lkv_sched.cuh).  Per CTA, 8 warps:
-//   warp 0      TMA producer: streams 64-token key/value tiles of the cache into a ring of
-//               shared-memory stages (2-D tiles of 64 rows x 64 bf16, 128-byte swizzle).
+//   warp 0      TMA producer: streams key/value tiles of the cache (64 keys for MLA / GLA,
+//               128 for GQLA) into a ring of shared-memory stages (2-D boxes of tile rows x
+//               64 bf16, 128-byte swizzle).
 //   warp 1      TMEM owner and UMMA issuer (one thread): S = Q K^T into TMEM, then
 //               O += P V into TMEM.  The non-RoPE part of Q and P are A operands read from
 //               TMEM; the RoPE part of Q is an A operand in shared memory; K and V are B
@@ -14,7 +15,7 @@
 //               (bf16) into TMEM, rescales O when the running max moves, and at the end of a
 //               segment writes out / lse (or fp32 partials).
 //
-// TMEM columns: O [0, DV) | S [DV, DV+64) | P0, P1 [DV+64, DV+128) | Q [DV+128, ...).
+// TMEM columns: O [0, DV) | S [DV, DV+T) | P0, P1 [DV+T, DV+2T) | Q [DV+2T, ...) for T keys/tile.
 // P is double buffered so the softmax of tile n+1 never waits for the PV of tile n.
 //
 // MLA absorbed path (h_q = 128 heads share the latent, GQLA explainer section 2): the
@@ -42,13 +43,12 @@
 
 namespace lkv {
 
-constexpr int kBoxBytes = 64 * 64 * 2;  // one TMA box: 64 rows x 64 bf16
-constexpr int kMaxBoxes = 5;
-constexpr int kStageBytes = kMaxBoxes * kBoxBytes;  // 40 KB
 constexpr int kQropeBytes = 128 * 128;             // 128 rows x 64 bf16, swizzled
 constexpr int kTcThreads = 256;
-constexpr int kXRow = 68;                          // floats per exchange row (64 + padding)
-constexpr int kXBufBytes = 128 * kXRow * 4;
+// MLA pair message per tile: 128 rows x 64 fp16 of exp2(partial score - partial tile max)
+// (values in (0, 1], so fp16 keeps 11 significant bits where bf16 would keep 8), then the 128
+// partial tile maxima (fp32).
+constexpr int kMsgBytes = 128 * 128 + 128 * 4;
 constexpr int kTmemCols = 512;
 
 enum DecodeMode { MODE_MLA = 0, MODE_GQLA = 1, MODE_GLA = 2 };
@@ -81,29 +81,50 @@ struct TcParams {
 template <int kMode>
 struct ModeCfg {
   static constexpr bool kPair = (kMode == MODE_MLA);
+  // Keys per tile.  GQLA runs 128-key tiles so that every QK UMMA is N = 128 (one issuing
+  // thread then keeps the tensor pipe at full rate); MLA and GLA keep 64-key tiles because a
+  // 128-column S tile would not fit next to their 256-column O accumulator and resident Q.
+  static constexpr int kTile = (kMode == MODE_GQLA) ? 128 : 64;
+  static constexpr int kBoxBytes = kTile * 128;                 // one TMA box: kTile rows x 64 bf16
+  // GQLA keeps K (+ k_rope) and V in separate rings: a K slot is refilled as soon as its QK
+  // is done, while V waits for its PV.  Where K = V (MLA, GLA) one ring holds the tile.
+  static constexpr bool kSplitKV = (kMode == MODE_GQLA);
+  static constexpr int kStageBytes = (kSplitKV ? 3 : 5) * kBoxBytes;  // K ring (or whole tile)
+  static constexpr int kVStageBytes = 2 * kBoxBytes;                  // V ring (GQLA)
   static constexpr int kDV = (kMode == MODE_GQLA) ? 128 : 256;  // value columns per CTA
-  static constexpr int kStages = kPair ? 3 : 5;
+  static constexpr int kStages = (kMode == MODE_GQLA) ? 2 : (kPair ? 3 : 5);
+  static constexpr int kVStages = kSplitKV ? 3 : 1;
   static constexpr int kNope = (kMode == MODE_GQLA) ? 2 : 4;    // non-RoPE Q boxes (in TMEM)
   static constexpr int kRopeBox = (kMode == MODE_GQLA) ? 2 : 4; // stage box holding k_rope
-  static constexpr int kVBox0 = (kMode == MODE_GQLA) ? 3 : 0;   // first stage box holding V
+  static constexpr int kVBox0 = 0;                              // first V box (V ring or stage)
   static constexpr int kNV = kDV / 64;
-  static constexpr uint32_t S0 = kDV, P0 = kDV + 64, Q0 = kDV + 128;
-  static constexpr size_t kSmemBytes =
-      1024 + static_cast<size_t>(kStages) * kStageBytes + kQropeBytes + (kPair ? 2 * kXBufBytes : 0);
+  static constexpr int kPCols = kTile / 2;                      // bf16 P per buffer
+  static constexpr uint32_t S0 = kDV, P0 = kDV + kTile, Q0 = kDV + 2 * kTile;
+  static constexpr size_t kRingBytes =
+      static_cast<size_t>(kStages) * kStageBytes + (kSplitKV ? static_cast<size_t>(kVStages) * kVStageBytes : 0);
+  static constexpr size_t kSmemBytes = 1024 + kRingBytes + kQropeBytes + (kPair ? 4 * kMsgBytes : 0);
   __device__ static bool has_rope(uint32_t rank) { return !kPair || rank == 0; }
-  __device__ static int n_stage_boxes(uint32_t rank) { return kPair ? (rank == 0 ? 5 : 4) : 5; }
+  __device__ static int n_stage_boxes(uint32_t rank) { return kPair ? (rank == 0 ? 5 : 4) : (kSplitKV ? 3 : 5); }
 };
 static_assert(ModeCfg<MODE_MLA>::Q0 + 32 * ModeCfg<MODE_MLA>::kNope <= kTmemCols, "TMEM budget");
 static_assert(ModeCfg<MODE_GLA>::Q0 + 32 * ModeCfg<MODE_GLA>::kNope <= kTmemCols, "TMEM budget");
+static_assert(ModeCfg<MODE_GQLA>::Q0 + 32 * ModeCfg<MODE_GQLA>::kNope <= kTmemCols, "TMEM budget");
+static_assert(ModeCfg<MODE_MLA>::kTile == 64, "the score exchange rows hold 64 keys");
 static_assert(ModeCfg<MODE_MLA>::kSmemBytes <= 232448, "shared memory budget");
 static_assert(ModeCfg<MODE_GLA>::kSmemBytes <= 232448, "shared memory budget");
+static_assert(ModeCfg<MODE_GQLA>::kSmemBytes <= 232448, "shared memory budget");
 
-template <int kStagesT>
+// Advance a shared-memory descriptor by a byte offset (start-address field, 16-byte units).
+__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
+
+template <int kStagesT, int kVStagesT>
 struct __align__(16) TcSmem {
   uint64_t full[kStagesT];
   uint64_t empty[kStagesT];
+  uint64_t vfull[kVStagesT];
+  uint64_t vempty[kVStagesT];
   uint64_t s_full, s_free, o_free, q_ready, drain;
-  uint64_t p_full[2], o_done[2], x_full[2], x_free[2];
+  uint64_t p_full[2], o_done[2], x_full[2], x_free[2], x_ready[2], x_read[2];
   uint32_t tmem_base;
   uint32_t abort;
   long long t_begin, t_end, unit_t0;
@@ -123,17 +144,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   using Cfg = ModeCfg<kMode>;
   constexpr int DV = Cfg::kDV;
   constexpr int KS = Cfg::kStages;
+  constexpr int TN = Cfg::kTile;
+  constexpr int kBoxBytes = Cfg::kBoxBytes;
+  constexpr int kStageBytes = Cfg::kStageBytes;
   constexpr bool kPair = Cfg::kPair;
   constexpr uint32_t S0 = Cfg::S0, P0 = Cfg::P0, Q0 = Cfg::Q0;
 
   extern __shared__ __align__(1024) uint8_t dsmem_raw[];
-  __shared__ TcSmem<KS> sm;
+  constexpr int VS = Cfg::kVStages;
+  constexpr bool kSplit = Cfg::kSplitKV;
+  __shared__ TcSmem<KS, VS> sm;
   uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsmem_raw) + 1023) &
                                             ~static_cast<uintptr_t>(1023));
   const uint32_t stage_base = smem_u32(dsm);
-  uint8_t* qrope_smem = dsm + KS * kStageBytes;
+  uint8_t* vring = dsm + KS * kStageBytes;                 // GQLA V ring
+  const uint32_t vring_base = smem_u32(vring);
+  uint8_t* qrope_smem = dsm + Cfg::kRingBytes;
   const uint32_t qrope_base = smem_u32(qrope_smem);
-  float* xbuf = reinterpret_cast<float*>(qrope_smem + kQropeBytes);  // MLA only: [2][128][kXRow]
+  uint8_t* sbuf = qrope_smem + kQropeBytes;  // MLA only: 2 outgoing messages, then 2 incoming
+  uint8_t* rbuf = sbuf + 2 * kMsgBytes;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -147,6 +176,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   sa.cu = p.cu;
   sa.B = p.B;
   sa.s_q = p.s_q;
+  sa.tile = TN;
   sa.units_per_req = kPair ? p.s_q : p.G;
   sa.per_query_units = kPair ? 1 : 0;
   sa.P = p.P;
@@ -157,6 +187,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(smem_u32(&sm.full[s]), 1);
       mbar_init(smem_u32(&sm.empty[s]), 1);
     }
+    for (int s = 0; s < VS; ++s) {
+      mbar_init(smem_u32(&sm.vfull[s]), 1);
+      mbar_init(smem_u32(&sm.vempty[s]), 1);
+    }
     mbar_init(smem_u32(&sm.s_full), 1);
     mbar_init(smem_u32(&sm.s_free), n_sm_threads);
     mbar_init(smem_u32(&sm.o_free), n_sm_threads);
@@ -165,8 +199,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&sm.p_full[b]), n_sm_threads);
       mbar_init(smem_u32(&sm.o_done[b]), 1);
-      mbar_init(smem_u32(&sm.x_full[b]), 128);
-      mbar_init(smem_u32(&sm.x_free[b]), 128);
+      mbar_init(smem_u32(&sm.x_full[b]), 1);      // armed by this CTA, filled by the peer's copy
+      mbar_init(smem_u32(&sm.x_free[b]), 1);      // the peer has read our message b
+      mbar_init(smem_u32(&sm.x_ready[b]), 128);   // all rows of outgoing message b written
+      mbar_init(smem_u32(&sm.x_read[b]), 128);    // all rows of incoming message b read
     }
     sm.abort = 0;
     fence_mbar_init();
@@ -217,7 +253,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint32_t bytes = nbox * kBoxBytes;
       SegCursor cur = cur0;
       Segment sg;
-      long long n = 0;
+      long long n = 0, nv = 0;   // K (or whole) tiles and V tiles issued
       bool ok = true;
       while (ok && cur.next(sa, sg)) {
         for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
@@ -230,7 +266,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t fb = smem_u32(&sm.full[st]);
           mbar_arrive_expect_tx(fb, bytes);
           const uint32_t dst = stage_base + st * kStageBytes;
-          const int row = sg.cu_b + t * kTileN;
+          const int row = sg.cu_b + t * TN;
           if (kMode == MODE_MLA) {
             const int c0 = 256 * static_cast<int>(rank);
             for (int bx = 0; bx < 4; ++bx) tma_load_2d(dst + bx * kBoxBytes, &map_a, fb, c0 + 64 * bx, row);
@@ -240,8 +276,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tma_load_2d(dst, &map_a, fb, c0, row);
             tma_load_2d(dst + kBoxBytes, &map_a, fb, c0 + 64, row);
             tma_load_2d(dst + 2 * kBoxBytes, &map_r, fb, 0, row);
-            tma_load_2d(dst + 3 * kBoxBytes, &map_v, fb, c0, row);
-            tma_load_2d(dst + 4 * kBoxBytes, &map_v, fb, c0 + 64, row);
+            // V goes to its own ring slot, freed only by the PV of this tile
+            const int vs = static_cast<int>(n % VS);
+            if (!mbar_wait(smem_u32(&sm.vempty[vs]), static_cast<uint32_t>(((n / VS) & 1) ^ 1), wc,
+                           LKV_WAIT(W_EMPTY))) {
+              ok = false;
+              ++n;  // this tile's K copies are in flight: the drain below must wait for them
+              break;
+            }
+            const uint32_t vb = smem_u32(&sm.vfull[vs]);
+            mbar_arrive_expect_tx(vb, Cfg::kVStageBytes);
+            const uint32_t vdst = vring_base + vs * Cfg::kVStageBytes;
+            tma_load_2d(vdst, &map_v, vb, c0, row);
+            tma_load_2d(vdst + kBoxBytes, &map_v, vb, c0 + 64, row);
+            ++nv;
           } else {
             const int c0 = 256 * sg.k;
             for (int bx = 0; bx < 4; ++bx) tma_load_2d(dst + bx * kBoxBytes, &map_a, fb, c0 + 64 * bx, row);
@@ -255,22 +303,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const WaitCtl dc{&zero, p.err, p.wait_limit_ns};  // ignores the abort flag, keeps the limit
       for (long long m = n - inflight; m < n; ++m)
         mbar_wait(smem_u32(&sm.full[m % KS]), static_cast<uint32_t>((m / KS) & 1), dc, LKV_WAIT(W_DRAIN));
+      if (kSplit) {
+        // V copies: issued for every tile whose K was issued, except possibly the last one when
+        // its vempty wait gave up; wait only for those actually issued (counted by nv)
+        const long long vin = nv < VS ? nv : VS;
+        for (long long m = nv - vin; m < nv; ++m)
+          mbar_wait(smem_u32(&sm.vfull[m % VS]), static_cast<uint32_t>((m / VS) & 1), dc, LKV_WAIT(W_DRAIN));
+      }
     }
   } else if (warp == 1) {
     // ============================================================ UMMA issuer
     if (lane == 0) {
       const bool rope = Cfg::has_rope(rank);
-      const uint32_t id_qk = idesc_bf16(128, kTileN, 0, 0);
+      const uint32_t id_qk = idesc_bf16(128, TN, 0, 0);
       const uint32_t id_pv = idesc_bf16(128, DV, 0, 1);
+      const uint64_t qrope_desc = sdesc_sw128(qrope_base, 16, 1024);
       SegCursor cur = cur0;
       Segment sg;
       long long n = 0;   // global tile counter
       int seg = 0;       // segments started
       bool ok = true;
-      bool pend = false, pend_first = false;   // PV of tile pend_n not yet issued
-      int pend_seg = 0;
-      long long pend_n = 0;
+      // PVs trail their QKs: by one tile, or by two in the MLA pair (its softmax runs one tile
+      // behind the score stream, so P(n-1) is only ready after S(n) has been read).
+      constexpr int kLag = kPair ? 2 : 1;
+      long long pq_n[2] = {0, 0};
+      int pq_seg[2] = {0, 0};
+      bool pq_first[2] = {false, false};
+      int pq_len = 0, pq_head = 0;
       auto issue_pv = [&]() -> bool {
+        const long long pend_n = pq_n[pq_head];
+        const bool pend_first = pq_first[pq_head];
+        const int pend_seg = pq_seg[pq_head];
         const int pb = static_cast<int>(pend_n & 1);
         if (!mbar_wait(smem_u32(&sm.p_full[pb]), static_cast<uint32_t>((pend_n >> 1) & 1), wc,
                        LKV_WAIT(W_PFULL)))
@@ -278,16 +341,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (pend_first && pend_seg > 0 &&
             !mbar_wait(smem_u32(&sm.o_free), static_cast<uint32_t>((pend_seg - 1) & 1), wc, LKV_WAIT(W_OFREE)))
           return false;
+        if (kSplit && !mbar_wait(smem_u32(&sm.vfull[pend_n % VS]), static_cast<uint32_t>((pend_n / VS) & 1), wc,
+                                 LKV_WAIT(W_FULL)))
+          return false;
         tc_fence_after();
-        const uint32_t vbase = stage_base + static_cast<uint32_t>(pend_n % KS) * kStageBytes + Cfg::kVBox0 * kBoxBytes;
+        const uint32_t vaddr = kSplit ? vring_base + static_cast<uint32_t>(pend_n % VS) * Cfg::kVStageBytes
+                                      : stage_base + static_cast<uint32_t>(pend_n % KS) * kStageBytes;
+        const uint64_t vdesc = sdesc_sw128(vaddr + Cfg::kVBox0 * kBoxBytes, kBoxBytes, 1024);
+        const uint32_t pa = tbase + P0 + Cfg::kPCols * pb;
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t bd = sdesc_sw128(vbase + kk * 2048, kBoxBytes, 1024);
-          umma_ts(tbase, tbase + P0 + 32 * pb + kk * 8, bd, id_pv, (pend_first && kk == 0) ? 0u : 1u);
-        }
+        for (int kk = 0; kk < TN / 16; ++kk)
+          umma_ts(tbase, pa + kk * 8, desc_add(vdesc, kk * 2048), id_pv, (pend_first && kk == 0) ? 0u : 1u);
         umma_commit(smem_u32(&sm.o_done[pb]));
-        umma_commit(smem_u32(&sm.empty[pend_n % KS]));
-        pend = false;
+        umma_commit(kSplit ? smem_u32(&sm.vempty[pend_n % VS]) : smem_u32(&sm.empty[pend_n % KS]));
+        pq_head ^= 1;
+        --pq_len;
         return true;
       };
       while (ok && cur.next(sa, sg)) {
@@ -301,36 +369,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t kb = stage_base + st * kStageBytes;
+          const uint64_t kdesc = sdesc_sw128(stage_base + st * kStageBytes, 16, 1024);
 #pragma unroll
           for (int bx = 0; bx < Cfg::kNope; ++bx) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t bd = sdesc_sw128(kb + bx * kBoxBytes + kk * 32, 16, 1024);
-              umma_ts(tbase + S0, tbase + Q0 + bx * 32 + kk * 8, bd, id_qk, (bx | kk) ? 1u : 0u);
-            }
+            for (int kk = 0; kk < 4; ++kk)
+              umma_ts(tbase + S0, tbase + Q0 + bx * 32 + kk * 8, desc_add(kdesc, bx * kBoxBytes + kk * 32), id_qk,
+                      (bx | kk) ? 1u : 0u);
           }
           if (rope) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t ad = sdesc_sw128(qrope_base + kk * 32, 16, 1024);
-              const uint64_t bd = sdesc_sw128(kb + Cfg::kRopeBox * kBoxBytes + kk * 32, 16, 1024);
-              umma_ss(tbase + S0, ad, bd, id_qk, 1u);
-            }
+            for (int kk = 0; kk < 4; ++kk)
+              umma_ss(tbase + S0, desc_add(qrope_desc, kk * 32), desc_add(kdesc, Cfg::kRopeBox * kBoxBytes + kk * 32),
+                      id_qk, 1u);
           }
           umma_commit(smem_u32(&sm.s_full));
-          if (pend && !issue_pv()) {
+          if (kSplit) umma_commit(smem_u32(&sm.empty[st]));  // the K slot is free once QK is done
+          if (pq_len == kLag && !issue_pv()) {
             ok = false;
             break;
           }
-          pend = true;
-          pend_first = (t == sg.tile_lo);
-          pend_seg = seg;
-          pend_n = n;
+          const int tail = (pq_head + pq_len) & 1;
+          pq_n[tail] = n;
+          pq_first[tail] = (t == sg.tile_lo);
+          pq_seg[tail] = seg;
+          ++pq_len;
         }
         ++seg;
       }
-      if (ok && pend) issue_pv();
+      while (ok && pq_len > 0) ok = issue_pv();
       // all tcgen05 work of this thread done before TMEM is released
       umma_commit(smem_u32(&sm.drain));
       uint32_t zero = 0;
@@ -343,10 +410,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t lb = static_cast<uint32_t>((warp & 3) * 32);
     const bool row_ok = r < p.R;
     const uint32_t peer = rank ^ 1u;
-    uint32_t x_remote[2] = {0u, 0u}, xfull_remote[2] = {0u, 0u}, xfree_remote[2] = {0u, 0u};
+    uint32_t rbuf_remote[2] = {0u, 0u}, xfull_remote[2] = {0u, 0u}, xfree_remote[2] = {0u, 0u};
     if (kPair) {
       for (int b = 0; b < 2; ++b) {
-        x_remote[b] = map_to_peer(smem_u32(xbuf + (b * 128 + r) * kXRow), peer);
+        rbuf_remote[b] = map_to_peer(smem_u32(rbuf + b * kMsgBytes), peer);
         xfull_remote[b] = map_to_peer(smem_u32(&sm.x_full[b]), peer);
         xfree_remote[b] = map_to_peer(smem_u32(&sm.x_free[b]), peer);
       }
@@ -411,56 +478,92 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     };
 
     float m_run = -INFINITY, l_run = 0.f;
-    // Softmax of one tile whose full scores are in s[]; writes P(n); runs the segment
-    // epilogue after the unit's last tile of this range.
-    auto process = [&](float (&s)[64], const Segment& sg, int t, long long n) -> bool {
-      int qi, qh;
-      row_map(sg, qi, qh);
+    // Grouped modes: softmax of one tile whose scores are in s[] -> P bits in pw[], the running
+    // max / sum updated; `alpha` rescales O when the running max moved.
+    auto softmax_tile = [&](float (&s)[TN], const Segment& sg, int t, int qi, uint32_t (&pw)[TN / 2],
+                            bool& rescale, float& alpha) {
       if (t == sg.tile_lo) {
         m_run = -INFINITY;
         l_run = 0.f;
       }
-      const int lim = kPair ? sg.keys : (sg.L - p.s_q + qi + 1);  // keys visible to this row
-      const int key0 = t * kTileN;
-      float mx = -INFINITY;
-      if (key0 + kTileN <= lim) {
+      const int lim = sg.L - p.s_q + qi + 1;  // keys visible to this row
+      const int key0 = t * TN;
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (key0 + TN <= lim) {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
+        for (int c = 0; c < TN; ++c) {
           s[c] *= p.sl2;
-          mx = fmaxf(mx, s[c]);
+          m4[c & 3] = fmaxf(m4[c & 3], s[c]);
         }
       } else {
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
+        for (int c = 0; c < TN; ++c) {
           s[c] = (key0 + c < lim) ? s[c] * p.sl2 : -INFINITY;
-          mx = fmaxf(mx, s[c]);
+          m4[c & 3] = fmaxf(m4[c & 3], s[c]);
         }
       }
+      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       // lazy rescale: keep the running max unless the tile max exceeds it by 2^8
-      bool rescale = false;
+      rescale = false;
       float m_new = m_run;
       if (mx > m_run + 8.f) {
         m_new = mx;
         rescale = (m_run != -INFINITY);
       }
-      const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.f;
+      alpha = rescale ? ex2_approx(m_run - m_new) : 1.f;
       const float msub = (m_new == -INFINITY) ? 0.f : m_new;
-      uint32_t pw[32];
-      float sum = 0.f;
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float e0 = ex2_approx(s[2 * c] - msub);
-        const float e1 = ex2_approx(s[2 * c + 1] - msub);
-        sum += e0 + e1;
+      for (int c = 0; c < TN / 2; ++c) {
+        const uint32_t h = ex2_f16x2(s[2 * c] - msub, s[2 * c + 1] - msub);
+        const float e0 = f16_lo(h), e1 = f16_hi(h);
+        s4[c & 3] += e0 + e1;
         pw[c] = pack_bf16x2(e0, e1);
       }
-      l_run = l_run * alpha + sum;
+      l_run = l_run * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
       m_run = m_new;
+    };
+    // MLA pair: P = E_own * E_peer * 2^(t_own + t_peer - M) where E = exp2(partial - t) (fp16) of
+    // each CTA's half of the contraction and t its partial tile max (t_own + t_peer bounds the
+    // tile max of the full score).  Products of two floats commute, so both CTAs get the same P.
+    auto combine_tile = [&](const uint32_t (&eo)[32], const uint32_t (&ep)[32], float t_o, float t_p,
+                            const Segment& sg, int t, uint32_t (&pw)[TN / 2], bool& rescale, float& alpha) {
+      if (t == sg.tile_lo) {
+        m_run = -INFINITY;
+        l_run = 0.f;
+      }
+      const float T = t_o + t_p;  // -inf when every key of this tile is masked for the row
+      rescale = false;
+      float m_new = m_run;
+      if (T > m_run + 8.f) {
+        m_new = T;
+        rescale = (m_run != -INFINITY);
+      }
+      alpha = rescale ? ex2_approx(m_run - m_new) : 1.f;
+      const float f = (T == -INFINITY) ? 0.f : ex2_approx(T - m_new);
+      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float e0 = f16_lo(eo[c]) * f16_lo(ep[c]) * f;
+        const float e1 = f16_hi(eo[c]) * f16_hi(ep[c]) * f;
+        s4[c & 3] += e0 + e1;
+        pw[c] = pack_bf16x2(e0, e1);
+      }
+      l_run = l_run * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+      m_run = m_new;
+    };
+    // Common tail of a tile: publish P(n) (after the PV that last read its buffer), rescale O if
+    // the running max moved, and run the segment epilogue after the unit's last tile here.
+    auto finish_tile = [&](uint32_t (&pw)[TN / 2], bool rescale, float alpha, const Segment& sg, int t,
+                           long long n) -> bool {
+      int qi, qh;
+      row_map(sg, qi, qh);
+      const int key0 = t * TN;
       const int pb = static_cast<int>(n & 1);
       // P buffer pb was last read by PV(n-2)
       if (n >= 2 && !wait_all(smem_u32(&sm.o_done[pb]), static_cast<uint32_t>(((n - 2) >> 1) & 1), LKV_WAIT(W_ODONE)))
         return false;
-      if (__any_sync(0xffffffffu, rescale) && t != sg.tile_lo) {
+      if (__any_sync(0xffffffffu, rescale ? 1 : 0) && t != sg.tile_lo) {
         // O holds this segment's tiles up to n-1: wait for PV(n-1), then scale in place
         if (!wait_all(smem_u32(&sm.o_done[pb ^ 1]), static_cast<uint32_t>(((n - 1) >> 1) & 1), LKV_WAIT(W_ODONE)))
           return false;
@@ -476,13 +579,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
       tc_fence_after();
-      tmem_st32(tm_addr(tbase, lb, P0 + 32 * pb), pw);
-      if (key0 + kTileN > sg.keys) {
+#pragma unroll
+      for (int c = 0; c < TN / 2; c += 32) {
+        uint32_t w[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j) w[j] = pw[c + j];
+        tmem_st32(tm_addr(tbase, lb, P0 + Cfg::kPCols * pb + c), w);
+      }
+      if (key0 + TN > sg.keys) {
         // Rows past the unit's last key belong to another request or to unwritten cache:
         // their P is 0, but 0 * NaN would still poison O, so clear those V rows first.
         const int first = sg.keys - key0;
-        const int per_box = (kTileN - first) * 8;  // 16-byte chunks per V box
-        uint8_t* vb = dsm + (n % KS) * kStageBytes + Cfg::kVBox0 * kBoxBytes;
+        const int per_box = (TN - first) * 8;  // 16-byte chunks per V box
+        if (kSplit && !wait_all(smem_u32(&sm.vfull[n % VS]), static_cast<uint32_t>((n / VS) & 1), LKV_WAIT(W_FULL)))
+          return false;  // the copy must land before it is overwritten
+        uint8_t* vb = (kSplit ? vring + (n % VS) * Cfg::kVStageBytes : dsm + (n % KS) * kStageBytes) +
+                      Cfg::kVBox0 * kBoxBytes;
         for (int idx = r; idx < per_box * Cfg::kNV; idx += n_sm_threads) {
           const int bx = idx / per_box, rem = idx % per_box;
           *reinterpret_cast<uint4*>(vb + bx * kBoxBytes + (first + rem / 8) * 128 + (rem % 8) * 16) =
@@ -551,37 +663,38 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool haveA = cur.next(sa, sgA);
     int tA = haveA ? sgA.tile_lo : 0;
     long long nA = 0;
-    // tile waiting for the peer's partial scores (MLA only)
-    float prev[64];
+    // MLA: tile whose own half has been sent and whose peer half is awaited
+    uint32_t eprev[32];
+    float tprev = -INFINITY;
     Segment sgB;
     int tB = 0;
     long long nB = 0;
     bool haveB = false;
+    long long nconsumed = 0;  // incoming messages read (MLA)
     bool ok = true;
     if (haveA) load_q(sgA);
     while (ok && (haveA || haveB)) {
-      float cs[64];
+      float cs[TN];
       bool gotA = false;
       Segment sgAc;
       int tAc = 0;
       long long nAc = 0;
+      uint32_t ecur[32];
+      float tcur = -INFINITY;
       if (haveA) {
         if (!wait_all(smem_u32(&sm.s_full), static_cast<uint32_t>(nA & 1), LKV_WAIT(W_SFULL))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        {
-          uint32_t a[32], b2[32];
-          tmem_ld32(tm_addr(tbase, lb, S0), a);
-          tmem_ld32(tm_addr(tbase, lb, S0 + 32), b2);
-          tmem_wait_ld();
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            cs[c] = __uint_as_float(a[c]);
-            cs[32 + c] = __uint_as_float(b2[c]);
-          }
+        for (int c = 0; c < TN; c += 32) {
+          uint32_t a[32];
+          tmem_ld32(tm_addr(tbase, lb, S0 + c), a);
+#pragma unroll
+          for (int j = 0; j < 32; ++j) cs[c + j] = __uint_as_float(a[j]);
         }
+        tmem_wait_ld();
         tc_fence_before();
         mbar_arrive(smem_u32(&sm.s_free));
         const bool last = (tA == sgA.tile_hi - 1);
@@ -591,16 +704,52 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           have_nx = cur.next(sa, nx);
           if (have_nx) load_q(nx);
         }
-        if (kPair) {
+        if constexpr (kPair) {
+          // own half: mask, partial tile max, E = exp2(partial - max) in bf16
           const int xb = static_cast<int>(nA & 1);
+          if (r == 0) mbar_arrive_expect_tx(smem_u32(&sm.x_full[xb]), kMsgBytes);  // the peer's half of nA
+          const int lim = sgA.keys, key0 = tA * TN;
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          if (key0 + TN <= lim) {
+#pragma unroll
+            for (int c = 0; c < TN; ++c) {
+              cs[c] *= p.sl2;
+              m4[c & 3] = fmaxf(m4[c & 3], cs[c]);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < TN; ++c) {
+              cs[c] = (key0 + c < lim) ? cs[c] * p.sl2 : -INFINITY;
+              m4[c & 3] = fmaxf(m4[c & 3], cs[c]);
+            }
+          }
+          tcur = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          const float tsub = (tcur == -INFINITY) ? 0.f : tcur;
+#pragma unroll
+          for (int c = 0; c < 32; ++c) ecur[c] = ex2_f16x2(cs[2 * c] - tsub, cs[2 * c + 1] - tsub);
+          // our outgoing buffer xb (and the peer's incoming one) are free once message nA-2 was read
           if (nA >= 2 && !wait_all_cl(smem_u32(&sm.x_free[xb]), static_cast<uint32_t>(((nA - 2) >> 1) & 1),
                                       LKV_WAIT(W_XFREE))) {
             ok = false;
             break;
           }
+          uint8_t* msg = sbuf + xb * kMsgBytes;
 #pragma unroll
-          for (int c = 0; c < 64; c += 4) st_cluster_v4(x_remote[xb] + c * 4, cs[c], cs[c + 1], cs[c + 2], cs[c + 3]);
-          mbar_arrive_remote(xfull_remote[xb]);
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(msg + r * 128 + ((c ^ (r & 7)) << 4)) =
+                make_uint4(ecur[4 * c], ecur[4 * c + 1], ecur[4 * c + 2], ecur[4 * c + 3]);
+          reinterpret_cast<float*>(msg + 128 * 128)[r] = tcur;
+          fence_proxy_async_smem();
+          mbar_arrive(smem_u32(&sm.x_ready[xb]));
+          bool sent = true;
+          if (r == 0) {
+            sent = mbar_wait(smem_u32(&sm.x_ready[xb]), static_cast<uint32_t>((nA >> 1) & 1), wc, LKV_WAIT(W_XFULL));
+            if (sent) bulk_copy_to_peer(rbuf_remote[xb], smem_u32(msg), kMsgBytes, xfull_remote[xb]);
+          }
+          if (!__shfl_sync(0xffffffffu, sent ? 1 : 0, 0)) {
+            ok = false;
+            break;
+          }
         }
         gotA = true;
         sgAc = sgA;
@@ -616,24 +765,41 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       }
-      if (kPair) {
+      if constexpr (kPair) {
         if (haveB) {
           const int xb = static_cast<int>(nB & 1);
           if (!wait_all_cl(smem_u32(&sm.x_full[xb]), static_cast<uint32_t>((nB >> 1) & 1), LKV_WAIT(W_XFULL))) {
             ok = false;
             break;
           }
-          const float4* xr = reinterpret_cast<const float4*>(xbuf + (xb * 128 + r) * kXRow);
+          const uint8_t* msg = rbuf + xb * kMsgBytes;
+          uint32_t ep[32];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float4 x = xr[c];
-            prev[4 * c] += x.x;
-            prev[4 * c + 1] += x.y;
-            prev[4 * c + 2] += x.z;
-            prev[4 * c + 3] += x.w;
+          for (int c = 0; c < 8; ++c) {
+            const uint4 x = *reinterpret_cast<const uint4*>(msg + r * 128 + ((c ^ (r & 7)) << 4));
+            ep[4 * c] = x.x;
+            ep[4 * c + 1] = x.y;
+            ep[4 * c + 2] = x.z;
+            ep[4 * c + 3] = x.w;
           }
-          mbar_arrive_remote(xfree_remote[xb]);
-          if (!process(prev, sgB, tB, nB)) {
+          const float tpeer = reinterpret_cast<const float*>(msg + 128 * 128)[r];
+          ++nconsumed;
+          mbar_arrive(smem_u32(&sm.x_read[xb]));
+          bool freed = true;
+          if (r == 0) {
+            // every row of the incoming message has been read: the peer may reuse both buffers
+            freed = mbar_wait(smem_u32(&sm.x_read[xb]), static_cast<uint32_t>((nB >> 1) & 1), wc, LKV_WAIT(W_XFREE));
+            if (freed) mbar_arrive_remote(xfree_remote[xb]);
+          }
+          if (!__shfl_sync(0xffffffffu, freed ? 1 : 0, 0)) {
+            ok = false;
+            break;
+          }
+          uint32_t pw[TN / 2];
+          bool rescale;
+          float alpha;
+          combine_tile(eprev, ep, tprev, tpeer, sgB, tB, pw, rescale, alpha);
+          if (!finish_tile(pw, rescale, alpha, sgB, tB, nB)) {
             ok = false;
             break;
           }
@@ -641,16 +807,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         haveB = gotA;
         if (gotA) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) prev[c] = cs[c];
+          for (int c = 0; c < 32; ++c) eprev[c] = ecur[c];
+          tprev = tcur;
           sgB = sgAc;
           tB = tAc;
           nB = nAc;
         }
       } else if (gotA) {
-        if (!process(cs, sgAc, tAc, nAc)) {
+        int qi, qh;
+        row_map(sgAc, qi, qh);
+        uint32_t pw[TN / 2];
+        bool rescale;
+        float alpha;
+        softmax_tile(cs, sgAc, tAc, qi, pw, rescale, alpha);
+        if (!finish_tile(pw, rescale, alpha, sgAc, tAc, nAc)) {
           ok = false;
           break;
         }
+      }
+    }
+    if (kPair && !ok && r == 0) {
+      // After giving up, the peer may still have up to two messages on their way into this
+      // CTA's shared memory (it sends message m once message m-2 was read here).  Let them
+      // land (bounded) before the CTA can exit; every message is armed exactly once.
+      uint32_t zero = 0;
+      const WaitCtl dc{&zero, p.err, p.wait_limit_ns};
+      for (long long m = nconsumed; m < nconsumed + 2; ++m) {
+        if (m >= nA) mbar_arrive_expect_tx(smem_u32(&sm.x_full[m & 1]), kMsgBytes);
+        mbar_wait<true>(smem_u32(&sm.x_full[m & 1]), static_cast<uint32_t>((m >> 1) & 1), dc, LKV_WAIT(W_DRAIN));
       }
     }
   }

@@ -3,7 +3,7 @@
 // A "unit" is one query token of a request (MLA absorbed path: all h_q heads attend to the
 // shared latent, one unit per new token) or one group of a request (GQLA / GLA: the rows of
 // a unit are the group's heads for every new token).  Each unit needs ceil(keys / 64) key
-// tiles.  All tiles of all units are laid end to end (request-major, then unit) and the
+// tiles (64 or 128 keys, per kernel).  All tiles of all units are laid end to end (request-major, then unit) and the
 // sequence is cut into P equal ranges, one per persistent CTA (per CTA pair for MLA).  A
 // range is processed as "segments": maximal runs of its tiles that belong to one unit.  A
 // segment that covers its unit entirely writes the final output; the first or last segment
@@ -20,11 +20,10 @@
 
 namespace lkv {
 
-constexpr int kTileN = 64;  // keys per tile
-
 struct SchedArgs {
   const int* cu;         // [B+1]
   int B, s_q;
+  int tile;              // keys per tile
   int units_per_req;     // MLA: s_q ; grouped: G
   int per_query_units;   // 1: unit k is query token k (MLA); 0: unit k is group k
   int P;                 // number of ranges
@@ -35,18 +34,18 @@ __host__ __device__ __forceinline__ int unit_keys(const SchedArgs& a, int L, int
   if (L < a.s_q) return 0;
   return a.per_query_units ? (L - a.s_q + k + 1) : L;
 }
-__host__ __device__ __forceinline__ long long ceil_tiles(int keys) {
-  return (static_cast<long long>(keys) + kTileN - 1) / kTileN;
+__host__ __device__ __forceinline__ long long ceil_tiles(int keys, int tile) {
+  return (static_cast<long long>(keys) + tile - 1) / tile;
 }
 __host__ __device__ __forceinline__ long long request_tiles(const SchedArgs& a, int b) {
   const int L = LKV_LDG(a.cu + b + 1) - LKV_LDG(a.cu + b);
   if (L < a.s_q) return 0;
   if (a.per_query_units) {
     long long t = 0;
-    for (int k = 0; k < a.units_per_req; ++k) t += ceil_tiles(L - a.s_q + k + 1);
+    for (int k = 0; k < a.units_per_req; ++k) t += ceil_tiles(L - a.s_q + k + 1, a.tile);
     return t;
   }
-  return a.units_per_req * ceil_tiles(L);
+  return a.units_per_req * ceil_tiles(L, a.tile);
 }
 
 struct Segment {
@@ -72,7 +71,7 @@ struct SegCursor {
       const int cu_b = LKV_LDG(a.cu + b);
       const int L = LKV_LDG(a.cu + b + 1) - cu_b;
       const int keys = unit_keys(a, L, k);
-      const long long nt = ceil_tiles(keys);
+      const long long nt = ceil_tiles(keys, a.tile);
       const long long lo = (t_begin > unit_t0 ? t_begin : unit_t0) - unit_t0;
       const long long hi_g = unit_t0 + nt < t_end ? unit_t0 + nt : t_end;
       const long long hi = hi_g - unit_t0;
@@ -151,7 +150,7 @@ __device__ __forceinline__ SegCursor locate_range(const SchedArgs& a, int p, boo
     // walk units inside the request until the one containing t_begin
     const int L = LKV_LDG(a.cu + fb + 1) - LKV_LDG(a.cu + fb);
     for (int k = 0; k < a.units_per_req; ++k) {
-      const long long nt = ceil_tiles(unit_keys(a, L, k));
+      const long long nt = ceil_tiles(unit_keys(a, L, k), a.tile);
       if (c.unit_t0 + nt > c.t_begin) {
         c.k = k;
         break;
@@ -181,7 +180,7 @@ inline SegCursor locate_range_host(const SchedArgs& a, int p) {
       c.unit_t0 = acc;
       const int L = a.cu[b + 1] - a.cu[b];
       for (int k = 0; k < a.units_per_req; ++k) {
-        const long long nt = ceil_tiles(unit_keys(a, L, k));
+        const long long nt = ceil_tiles(unit_keys(a, L, k), a.tile);
         if (c.unit_t0 + nt > c.t_begin) {
           c.k = k;
           break;

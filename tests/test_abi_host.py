@@ -75,6 +75,7 @@ def test_workspace_sizes(lkv):
 def _check_partition(segs, cu, kind, s_q, G, P):
     """Every tile of every unit is covered exactly once; slot rules hold."""
     B = len(cu) - 1
+    T = 128 if kind == 1 else 64
     upr = s_q if kind == 0 else G
     covered = {}
     by_range = {}
@@ -82,7 +83,7 @@ def _check_partition(segs, cu, kind, s_q, G, P):
         assert uid == b * upr + k
         L = cu[b + 1] - cu[b]
         keys = (L - s_q + k + 1) if kind == 0 else L
-        nt = -(-keys // 64)
+        nt = -(-keys // T)
         assert 0 <= lo < hi <= nt
         assert complete == int(lo == 0 and hi == nt)
         for t in range(lo, hi):
@@ -93,7 +94,7 @@ def _check_partition(segs, cu, kind, s_q, G, P):
         L = cu[b + 1] - cu[b]
         for k in range(upr):
             keys = (L - s_q + k + 1) if kind == 0 else L
-            for t in range(-(-keys // 64)):
+            for t in range(-(-keys // T)):
                 assert (b, k, t) in covered
     sizes = []
     for p, lst in by_range.items():
