@@ -103,8 +103,13 @@ struct ModeCfg {
   static constexpr size_t kRingBytes =
       static_cast<size_t>(kStages) * kStageBytes + (kSplitKV ? static_cast<size_t>(kVStages) * kVStageBytes : 0);
   static constexpr size_t kSmemBytes = 1024 + kRingBytes + kQropeBytes + (kPair ? 4 * kMsgBytes : 0);
-  __device__ static bool has_rope(uint32_t rank) { return !kPair || rank == 0; }
-  __device__ static int n_stage_boxes(uint32_t rank) { return kPair ? (rank == 0 ? 5 : 4) : (kSplitKV ? 3 : 5); }
+  // QK K-steps per CTA.  In the MLA pair rank 0 takes latent columns [0, 224) plus the 64
+  // RoPE columns and rank 1 takes latent columns [224, 512): 18 K-steps each.  The part of a
+  // CTA's query that is not in TMEM (RoPE, or latent columns 224..255 for rank 1) sits in
+  // shared memory, and the stage's fifth box holds the matching key columns.
+  __device__ static int n_tmem_steps(uint32_t rank) { return (kPair && rank == 0) ? 4 * kNope - 2 : 4 * kNope; }
+  __device__ static int smem_kk0(uint32_t rank) { return (kPair && rank == 1) ? 2 : 0; }
+  static constexpr int kStageBoxes = kSplitKV ? 3 : 5;
 };
 static_assert(ModeCfg<MODE_MLA>::Q0 + 32 * ModeCfg<MODE_MLA>::kNope <= kTmemCols, "TMEM budget");
 static_assert(ModeCfg<MODE_GLA>::Q0 + 32 * ModeCfg<MODE_GLA>::kNope <= kTmemCols, "TMEM budget");
@@ -124,7 +129,7 @@ struct __align__(16) TcSmem {
   uint64_t vfull[kVStagesT];
   uint64_t vempty[kVStagesT];
   uint64_t s_full, s_free, o_free, q_ready, drain;
-  uint64_t p_full[2], o_done[2], x_full[2], x_free[2], x_ready[2], x_read[2];
+  uint64_t p_full[2], o_done[2], x_full[2], x_free[2];
   uint32_t tmem_base;
   uint32_t abort;
   long long t_begin, t_end, unit_t0;
@@ -192,17 +197,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(smem_u32(&sm.vempty[s]), 1);
     }
     mbar_init(smem_u32(&sm.s_full), 1);
-    mbar_init(smem_u32(&sm.s_free), n_sm_threads);
-    mbar_init(smem_u32(&sm.o_free), n_sm_threads);
-    mbar_init(smem_u32(&sm.q_ready), n_sm_threads);
+    // softmax-side barriers take one arrival per warp (lane 0, after a __syncwarp)
+    mbar_init(smem_u32(&sm.s_free), n_sm_warps);
+    mbar_init(smem_u32(&sm.o_free), n_sm_warps);
+    mbar_init(smem_u32(&sm.q_ready), n_sm_warps);
     mbar_init(smem_u32(&sm.drain), 1);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&sm.p_full[b]), n_sm_threads);
+      mbar_init(smem_u32(&sm.p_full[b]), n_sm_warps);
       mbar_init(smem_u32(&sm.o_done[b]), 1);
       mbar_init(smem_u32(&sm.x_full[b]), 1);      // armed by this CTA, filled by the peer's copy
-      mbar_init(smem_u32(&sm.x_free[b]), 1);      // the peer has read our message b
-      mbar_init(smem_u32(&sm.x_ready[b]), 128);   // all rows of outgoing message b written
-      mbar_init(smem_u32(&sm.x_read[b]), 128);    // all rows of incoming message b read
+      mbar_init(smem_u32(&sm.x_free[b]), 4);      // each of the peer's 4 warps has read its rows of message b
     }
     sm.abort = 0;
     fence_mbar_init();
@@ -249,8 +253,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 0) {
     // ============================================================ TMA producer
     if (lane == 0) {
-      const int nbox = Cfg::n_stage_boxes(rank);
-      const uint32_t bytes = nbox * kBoxBytes;
+      const uint32_t bytes = Cfg::kStageBoxes * kBoxBytes;
       SegCursor cur = cur0;
       Segment sg;
       long long n = 0, nv = 0;   // K (or whole) tiles and V tiles issued
@@ -270,7 +273,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (kMode == MODE_MLA) {
             const int c0 = 256 * static_cast<int>(rank);
             for (int bx = 0; bx < 4; ++bx) tma_load_2d(dst + bx * kBoxBytes, &map_a, fb, c0 + 64 * bx, row);
-            if (rank == 0) tma_load_2d(dst + 4 * kBoxBytes, &map_r, fb, 0, row);
+            if (rank == 0)
+              tma_load_2d(dst + 4 * kBoxBytes, &map_r, fb, 0, row);
+            else
+              tma_load_2d(dst + 4 * kBoxBytes, &map_a, fb, 192, row);  // rank 0's fourth box
           } else if (kMode == MODE_GQLA) {
             const int c0 = 128 * sg.k;
             tma_load_2d(dst, &map_a, fb, c0, row);
@@ -314,7 +320,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   } else if (warp == 1) {
     // ============================================================ UMMA issuer
     if (lane == 0) {
-      const bool rope = Cfg::has_rope(rank);
+      const int n_tm = Cfg::n_tmem_steps(rank), kk0 = Cfg::smem_kk0(rank);
       const uint32_t id_qk = idesc_bf16(128, TN, 0, 0);
       const uint32_t id_pv = idesc_bf16(128, DV, 0, 1);
       const uint64_t qrope_desc = sdesc_sw128(qrope_base, 16, 1024);
@@ -371,18 +377,17 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tc_fence_after();
           const uint64_t kdesc = sdesc_sw128(stage_base + st * kStageBytes, 16, 1024);
 #pragma unroll
-          for (int bx = 0; bx < Cfg::kNope; ++bx) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
+          for (int ks = 0; ks < 4 * Cfg::kNope; ++ks) {
+            const int bx = ks >> 2, kk = ks & 3;
+            if (ks < n_tm)
               umma_ts(tbase + S0, tbase + Q0 + bx * 32 + kk * 8, desc_add(kdesc, bx * kBoxBytes + kk * 32), id_qk,
-                      (bx | kk) ? 1u : 0u);
+                      ks ? 1u : 0u);
           }
-          if (rope) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
+          for (int kk = 0; kk < 4; ++kk)
+            if (kk >= kk0)
               umma_ss(tbase + S0, desc_add(qrope_desc, kk * 32), desc_add(kdesc, Cfg::kRopeBox * kBoxBytes + kk * 32),
                       id_qk, 1u);
-          }
           umma_commit(smem_u32(&sm.s_full));
           if (kSplit) umma_commit(smem_u32(&sm.empty[st]));  // the K slot is free once QK is done
           if (pq_len == kLag && !issue_pv()) {
@@ -425,6 +430,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     auto wait_all = [&](uint32_t bar, uint32_t par, int site) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, par, wc, site)) != 0;
     };
+    auto warp_arrive = [&](uint32_t bar) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+    };
     auto wait_all_cl = [&](uint32_t bar, uint32_t par, int site) -> bool {
       return __all_sync(0xffffffffu, mbar_wait<true>(bar, par, wc, site)) != 0;
     };
@@ -463,8 +472,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tmem_st32(tm_addr(tbase, lb, Q0 + bx * 32), w);
       }
-      if (Cfg::has_rope(rank)) {
-        const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + qrow * 64);
+      {
+        // RoPE part, or (MLA rank 1) latent columns 192..255 of which K-steps 2 and 3 are used
+        const uint4* src = reinterpret_cast<const uint4*>(
+            (kPair && rank == 1) ? p.q_nope + qrow * p.dq + 192 : p.q_rope + qrow * 64);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const uint4 x = row_ok ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
@@ -474,7 +485,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&sm.q_ready));
+      warp_arrive(smem_u32(&sm.q_ready));
     };
 
     float m_run = -INFINITY, l_run = 0.f;
@@ -604,7 +615,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(smem_u32(&sm.p_full[pb]));
+      warp_arrive(smem_u32(&sm.p_full[pb]));
       if (t != sg.tile_hi - 1) return true;
       // ---------------------------------------------------------- segment epilogue
       if (!wait_all(smem_u32(&sm.o_done[pb]), static_cast<uint32_t>((n >> 1) & 1), LKV_WAIT(W_ODONE)))
@@ -654,7 +665,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (r == 0 && rank == 0) p.seg_info[2 * range + sg.slot] = sg.unit_id;
       }
       tc_fence_before();
-      mbar_arrive(smem_u32(&sm.o_free));
+      warp_arrive(smem_u32(&sm.o_free));
       return true;
     };
 
@@ -696,7 +707,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tmem_wait_ld();
         tc_fence_before();
-        mbar_arrive(smem_u32(&sm.s_free));
+        warp_arrive(smem_u32(&sm.s_free));
         const bool last = (tA == sgA.tile_hi - 1);
         bool have_nx = false;
         if (last) {
@@ -740,15 +751,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 make_uint4(ecur[4 * c], ecur[4 * c + 1], ecur[4 * c + 2], ecur[4 * c + 3]);
           reinterpret_cast<float*>(msg + 128 * 128)[r] = tcur;
           fence_proxy_async_smem();
-          mbar_arrive(smem_u32(&sm.x_ready[xb]));
-          bool sent = true;
-          if (r == 0) {
-            sent = mbar_wait(smem_u32(&sm.x_ready[xb]), static_cast<uint32_t>((nA >> 1) & 1), wc, LKV_WAIT(W_XFULL));
-            if (sent) bulk_copy_to_peer(rbuf_remote[xb], smem_u32(msg), kMsgBytes, xfull_remote[xb]);
-          }
-          if (!__shfl_sync(0xffffffffu, sent ? 1 : 0, 0)) {
-            ok = false;
-            break;
+          __syncwarp();
+          if (lane == 0) {
+            // each warp ships its own 32 rows and their tile maxima
+            const uint32_t w0 = static_cast<uint32_t>(r & ~31);
+            bulk_copy_to_peer(rbuf_remote[xb] + w0 * 128, smem_u32(msg) + w0 * 128, 32 * 128, xfull_remote[xb]);
+            bulk_copy_to_peer(rbuf_remote[xb] + 128 * 128 + w0 * 4, smem_u32(msg) + 128 * 128 + w0 * 4, 128,
+                              xfull_remote[xb]);
           }
         }
         gotA = true;
@@ -784,17 +793,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           const float tpeer = reinterpret_cast<const float*>(msg + 128 * 128)[r];
           ++nconsumed;
-          mbar_arrive(smem_u32(&sm.x_read[xb]));
-          bool freed = true;
-          if (r == 0) {
-            // every row of the incoming message has been read: the peer may reuse both buffers
-            freed = mbar_wait(smem_u32(&sm.x_read[xb]), static_cast<uint32_t>((nB >> 1) & 1), wc, LKV_WAIT(W_XFREE));
-            if (freed) mbar_arrive_remote(xfree_remote[xb]);
-          }
-          if (!__shfl_sync(0xffffffffu, freed ? 1 : 0, 0)) {
-            ok = false;
-            break;
-          }
+          // this warp's rows of the incoming message are read: one of the 4 arrivals that let
+          // the peer reuse both copies of buffer xb
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(xfree_remote[xb]);
           uint32_t pw[TN / 2];
           bool rescale;
           float alpha;
