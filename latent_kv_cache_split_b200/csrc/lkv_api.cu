@@ -303,7 +303,7 @@ lkv_status lkv_mla_absorbed_decode(const void* q_nope_abs, const void* q_rope, c
   L.mode = MODE_MLA;
   constexpr int TN = ModeCfg<MODE_MLA>::kTile;
   if (!make_tmap_bf16(&L.map_a, ckv, r_kv, cache_rows, ckv_row_stride * 2, 64, TN) ||
-      !make_tmap_bf16(&L.map_r, kpe, d_rope, cache_rows, kpe_row_stride * 2, 64, TN))
+      !make_tmap_bf16(&L.map_r, kpe, d_rope, cache_rows, kpe_row_stride * 2, 32, TN))  // one RoPE half per CTA
     return LKV_ERR_CUDA;
   L.map_v = L.map_a;
   uint8_t* ws = static_cast<uint8_t*>(workspace);

@@ -43,12 +43,19 @@
 
 namespace lkv {
 
-constexpr int kQropeBytes = 128 * 128;             // 128 rows x 64 bf16, swizzled
-constexpr int kTcThreads = 256;
+// Warps: 0 TMA producer, 1 UMMA issuer, 2-3 MLA message sender, 4-11 softmax.  Softmax warp
+// 4 + q + 4 h owns TMEM lane quadrant q (rows 32q..32q+31) and key-column half h of each tile.
+constexpr int kTcThreads = 384;
 // MLA pair message per tile: 128 rows x 64 fp16 of exp2(partial score - partial tile max)
 // (values in (0, 1], so fp16 keeps 11 significant bits where bf16 would keep 8), then the 128
 // partial tile maxima (fp32).
-constexpr int kMsgBytes = 128 * 128 + 128 * 4;
+// One score message: 128 rows x 64 fp16 factors, then the partial tile maxima of both column
+// halves of each row.
+constexpr int kMsgBytes = 128 * 128 + 2 * 128 * 4;
+// Incoming score messages in flight per CTA of the MLA pair.  A CTA sends message m only after
+// it has read the peer's message m-1, which the peer sent after reading message m-2 (and so
+// m-3) from this CTA, so with 3 slots the slot of message m is always free when it is written.
+constexpr int kMsgSlots = 3;
 constexpr int kTmemCols = 512;
 
 enum DecodeMode { MODE_MLA = 0, MODE_GQLA = 1, MODE_GLA = 2 };
@@ -56,7 +63,7 @@ enum DecodeMode { MODE_MLA = 0, MODE_GQLA = 1, MODE_GLA = 2 };
 // Wait sites (added to LKV_SITE_WAIT_BASE in the error word).
 enum WaitSite {
   W_EMPTY = 1, W_FULL, W_SFREE, W_QREADY, W_PFULL, W_OFREE, W_SFULL, W_ODONE, W_XFREE, W_XFULL,
-  W_DRAIN
+  W_DRAIN, W_XSTAGED, W_XCHG
 };
 
 struct TcParams {
@@ -89,10 +96,15 @@ struct ModeCfg {
   // GQLA keeps K (+ k_rope) and V in separate rings: a K slot is refilled as soon as its QK
   // is done, while V waits for its PV.  Where K = V (MLA, GLA) one ring holds the tile.
   static constexpr bool kSplitKV = (kMode == MODE_GQLA);
-  static constexpr int kStageBytes = (kSplitKV ? 3 : 5) * kBoxBytes;  // K ring (or whole tile)
+  // MLA: each CTA of the pair contracts its 256 latent columns and one 32-column half of the
+  // RoPE key (a 64-byte swizzled box); the other modes take the whole 64-column RoPE key.
+  static constexpr int kRopeBoxBytes = kPair ? kTile * 64 : kBoxBytes;
+  static constexpr int kStageBytes = (kSplitKV ? 2 : 4) * kBoxBytes + kRopeBoxBytes;  // K ring (or whole tile)
   static constexpr int kVStageBytes = 2 * kBoxBytes;                  // V ring (GQLA)
   static constexpr int kDV = (kMode == MODE_GQLA) ? 128 : 256;  // value columns per CTA
-  static constexpr int kStages = (kMode == MODE_GQLA) ? 2 : (kPair ? 3 : 5);
+  static constexpr int kStages = (kMode == MODE_GQLA) ? 2 : (kPair ? 4 : 5);
+  // L2 prefetch distance of the producer in tiles (0: off)
+  static constexpr int kPrefetch = kPair ? kStages + 1 : 0;
   static constexpr int kVStages = kSplitKV ? 3 : 1;
   static constexpr int kNope = (kMode == MODE_GQLA) ? 2 : 4;    // non-RoPE Q boxes (in TMEM)
   static constexpr int kRopeBox = (kMode == MODE_GQLA) ? 2 : 4; // stage box holding k_rope
@@ -102,14 +114,12 @@ struct ModeCfg {
   static constexpr uint32_t S0 = kDV, P0 = kDV + kTile, Q0 = kDV + 2 * kTile;
   static constexpr size_t kRingBytes =
       static_cast<size_t>(kStages) * kStageBytes + (kSplitKV ? static_cast<size_t>(kVStages) * kVStageBytes : 0);
-  static constexpr size_t kSmemBytes = 1024 + kRingBytes + kQropeBytes + (kPair ? 4 * kMsgBytes : 0);
-  // QK K-steps per CTA.  In the MLA pair rank 0 takes latent columns [0, 224) plus the 64
-  // RoPE columns and rank 1 takes latent columns [224, 512): 18 K-steps each.  The part of a
-  // CTA's query that is not in TMEM (RoPE, or latent columns 224..255 for rank 1) sits in
-  // shared memory, and the stage's fifth box holds the matching key columns.
-  __device__ static int n_tmem_steps(uint32_t rank) { return (kPair && rank == 0) ? 4 * kNope - 2 : 4 * kNope; }
-  __device__ static int smem_kk0(uint32_t rank) { return (kPair && rank == 1) ? 2 : 0; }
-  static constexpr int kStageBoxes = kSplitKV ? 3 : 5;
+  // The RoPE part of the query sits in shared memory as an A operand: 128 rows of 64 columns
+  // (128-byte swizzle), or of the CTA's 32-column half in the MLA pair (64-byte swizzle).
+  static constexpr int kQropeBytes = kPair ? 128 * 64 : 128 * 128;
+  static constexpr int kRopeSteps = kPair ? 2 : 4;  // QK K-steps over the RoPE columns
+  // MLA adds kMsgSlots incoming score messages and one outgoing staging copy
+  static constexpr size_t kSmemBytes = 1024 + kRingBytes + kQropeBytes + (kPair ? (kMsgSlots + 1) * kMsgBytes : 0);
 };
 static_assert(ModeCfg<MODE_MLA>::Q0 + 32 * ModeCfg<MODE_MLA>::kNope <= kTmemCols, "TMEM budget");
 static_assert(ModeCfg<MODE_GLA>::Q0 + 32 * ModeCfg<MODE_GLA>::kNope <= kTmemCols, "TMEM budget");
@@ -129,7 +139,11 @@ struct __align__(16) TcSmem {
   uint64_t vfull[kVStagesT];
   uint64_t vempty[kVStagesT];
   uint64_t s_full, s_free, o_free, q_ready, drain;
-  uint64_t p_full[2], o_done[2], x_full[2], x_free[2];
+  uint64_t p_full[2], o_done[2], x_full[kMsgSlots];
+  uint64_t x_staged, x_stage_free;  // MLA: outgoing message staged by the softmax / read by the sender
+  uint64_t x_consumed;              // MLA: incoming message read by the softmax
+  uint64_t xbar[4][2];              // per lane quadrant: both column halves posted a value
+  float xch[2][2][128];             // [buffer][column half][row] values swapped between the halves
   uint32_t tmem_base;
   uint32_t abort;
   long long t_begin, t_end, unit_t0;
@@ -166,15 +180,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const uint32_t vring_base = smem_u32(vring);
   uint8_t* qrope_smem = dsm + Cfg::kRingBytes;
   const uint32_t qrope_base = smem_u32(qrope_smem);
-  uint8_t* sbuf = qrope_smem + kQropeBytes;  // MLA only: 2 outgoing messages, then 2 incoming
-  uint8_t* rbuf = sbuf + 2 * kMsgBytes;
+  uint8_t* rbuf = qrope_smem + Cfg::kQropeBytes;  // MLA only: kMsgSlots incoming messages
+  uint8_t* sbuf = rbuf + kMsgSlots * kMsgBytes;  // MLA only: the outgoing message being staged
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
   const uint32_t rank = kPair ? cluster_ctarank() : 0u;
   const int range = kPair ? (blockIdx.x >> 1) : blockIdx.x;
-  const int n_sm_warps = (p.R + 31) >> 5;  // softmax warps holding valid rows
+  const int n_row_warps = (p.R + 31) >> 5;  // lane quadrants holding valid rows
+  const int n_sm_warps = 2 * n_row_warps;     // softmax warps: two column halves per quadrant
   const int n_sm_threads = n_sm_warps * 32;
 
   SchedArgs sa;
@@ -201,12 +216,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     mbar_init(smem_u32(&sm.s_free), n_sm_warps);
     mbar_init(smem_u32(&sm.o_free), n_sm_warps);
     mbar_init(smem_u32(&sm.q_ready), n_sm_warps);
-    mbar_init(smem_u32(&sm.drain), 1);
+    mbar_init(smem_u32(&sm.drain), 2);  // one commit from each UMMA issuer
+    for (int b = 0; b < kMsgSlots; ++b) mbar_init(smem_u32(&sm.x_full[b]), 1);  // armed here, filled by the peer
+    mbar_init(smem_u32(&sm.x_staged), n_sm_warps);
+    mbar_init(smem_u32(&sm.x_stage_free), 1);
+    mbar_init(smem_u32(&sm.x_consumed), n_sm_warps);
+    for (int q = 0; q < 4; ++q)
+      for (int b = 0; b < 2; ++b) mbar_init(smem_u32(&sm.xbar[q][b]), 2);
     for (int b = 0; b < 2; ++b) {
       mbar_init(smem_u32(&sm.p_full[b]), n_sm_warps);
       mbar_init(smem_u32(&sm.o_done[b]), 1);
-      mbar_init(smem_u32(&sm.x_full[b]), 1);      // armed by this CTA, filled by the peer's copy
-      mbar_init(smem_u32(&sm.x_free[b]), 4);      // each of the peer's 4 warps has read its rows of message b
     }
     sm.abort = 0;
     fence_mbar_init();
@@ -253,13 +272,56 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 0) {
     // ============================================================ TMA producer
     if (lane == 0) {
-      const uint32_t bytes = Cfg::kStageBoxes * kBoxBytes;
+      const uint32_t bytes = Cfg::kStageBytes;
+      // L2 prefetch runs kPrefetch tiles ahead of the loads, so that a load issued when its ring
+      // slot frees finds its rows in L2 instead of waiting for HBM.
+      constexpr int kPrefetch = Cfg::kPrefetch;
+      SegCursor pcur = cur0;
+      Segment psg{};
+      int pt = 0;
+      bool pvalid = false;
+      auto prefetch_next = [&]() {
+        if (pvalid && pt + 1 < psg.tile_hi) {
+          ++pt;
+        } else {
+          pvalid = pcur.next(sa, psg);
+          if (!pvalid) return;
+          pt = psg.tile_lo;
+        }
+        const int prow = psg.cu_b + pt * TN;
+        if (kMode == MODE_MLA) {
+          const int c0 = 256 * static_cast<int>(rank);
+          for (int bx = 0; bx < 4; ++bx) tma_prefetch_l2_2d(&map_a, c0 + 64 * bx, prow);
+          tma_prefetch_l2_2d(&map_r, 32 * static_cast<int>(rank), prow);
+        } else if (kMode == MODE_GQLA) {
+          const int c0 = 128 * psg.k;
+          tma_prefetch_l2_2d(&map_a, c0, prow);
+          tma_prefetch_l2_2d(&map_a, c0 + 64, prow);
+          tma_prefetch_l2_2d(&map_r, 0, prow);
+          tma_prefetch_l2_2d(&map_v, c0, prow);
+          tma_prefetch_l2_2d(&map_v, c0 + 64, prow);
+        } else {
+          const int c0 = 256 * psg.k;
+          for (int bx = 0; bx < 4; ++bx) tma_prefetch_l2_2d(&map_a, c0 + 64 * bx, prow);
+          tma_prefetch_l2_2d(&map_r, 0, prow);
+        }
+      };
+      // the walker skips the tiles that the first loads fetch directly
+      for (int i = 0; kPrefetch > 0 && i < kPrefetch && (i == 0 || pvalid); ++i) {
+        if (pvalid && pt + 1 < psg.tile_hi) {
+          ++pt;
+        } else {
+          pvalid = pcur.next(sa, psg);
+          if (pvalid) pt = psg.tile_lo;
+        }
+      }
       SegCursor cur = cur0;
       Segment sg;
       long long n = 0, nv = 0;   // K (or whole) tiles and V tiles issued
       bool ok = true;
       while (ok && cur.next(sa, sg)) {
         for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
+          if (pvalid) prefetch_next();
           const int st = static_cast<int>(n % KS);
           const uint32_t par = static_cast<uint32_t>(((n / KS) & 1) ^ 1);
           if (!mbar_wait(smem_u32(&sm.empty[st]), par, wc, LKV_WAIT(W_EMPTY))) {
@@ -273,10 +335,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (kMode == MODE_MLA) {
             const int c0 = 256 * static_cast<int>(rank);
             for (int bx = 0; bx < 4; ++bx) tma_load_2d(dst + bx * kBoxBytes, &map_a, fb, c0 + 64 * bx, row);
-            if (rank == 0)
-              tma_load_2d(dst + 4 * kBoxBytes, &map_r, fb, 0, row);
-            else
-              tma_load_2d(dst + 4 * kBoxBytes, &map_a, fb, 192, row);  // rank 0's fourth box
+            tma_load_2d(dst + 4 * kBoxBytes, &map_r, fb, 32 * static_cast<int>(rank), row);  // RoPE half
           } else if (kMode == MODE_GQLA) {
             const int c0 = 128 * sg.k;
             tma_load_2d(dst, &map_a, fb, c0, row);
@@ -317,113 +376,148 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           mbar_wait(smem_u32(&sm.vfull[m % VS]), static_cast<uint32_t>((m / VS) & 1), dc, LKV_WAIT(W_DRAIN));
       }
     }
-  } else if (warp == 1) {
-    // ============================================================ UMMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ============================================================ UMMA issuers
+    // Warp 1 issues the QK products and warp 2 the PV products.  Two issuing threads keep
+    // more MMAs in flight than one, and neither chain stalls behind the other's operands: a
+    // QK waits only for its key tile and a free S, a PV only for its P (and a free O).
     if (lane == 0) {
-      const int n_tm = Cfg::n_tmem_steps(rank), kk0 = Cfg::smem_kk0(rank);
-      const uint32_t id_qk = idesc_bf16(128, TN, 0, 0);
-      const uint32_t id_pv = idesc_bf16(128, DV, 0, 1);
-      const uint64_t qrope_desc = sdesc_sw128(qrope_base, 16, 1024);
       SegCursor cur = cur0;
       Segment sg;
       long long n = 0;   // global tile counter
       int seg = 0;       // segments started
       bool ok = true;
-      // PVs trail their QKs: by one tile, or by two in the MLA pair (its softmax runs one tile
-      // behind the score stream, so P(n-1) is only ready after S(n) has been read).
-      constexpr int kLag = kPair ? 2 : 1;
-      long long pq_n[2] = {0, 0};
-      int pq_seg[2] = {0, 0};
-      bool pq_first[2] = {false, false};
-      int pq_len = 0, pq_head = 0;
-      auto issue_pv = [&]() -> bool {
-        const long long pend_n = pq_n[pq_head];
-        const bool pend_first = pq_first[pq_head];
-        const int pend_seg = pq_seg[pq_head];
-        const int pb = static_cast<int>(pend_n & 1);
-        if (!mbar_wait(smem_u32(&sm.p_full[pb]), static_cast<uint32_t>((pend_n >> 1) & 1), wc,
-                       LKV_WAIT(W_PFULL)))
-          return false;
-        if (pend_first && pend_seg > 0 &&
-            !mbar_wait(smem_u32(&sm.o_free), static_cast<uint32_t>((pend_seg - 1) & 1), wc, LKV_WAIT(W_OFREE)))
-          return false;
-        if (kSplit && !mbar_wait(smem_u32(&sm.vfull[pend_n % VS]), static_cast<uint32_t>((pend_n / VS) & 1), wc,
-                                 LKV_WAIT(W_FULL)))
-          return false;
-        tc_fence_after();
-        const uint32_t vaddr = kSplit ? vring_base + static_cast<uint32_t>(pend_n % VS) * Cfg::kVStageBytes
-                                      : stage_base + static_cast<uint32_t>(pend_n % KS) * kStageBytes;
-        const uint64_t vdesc = sdesc_sw128(vaddr + Cfg::kVBox0 * kBoxBytes, kBoxBytes, 1024);
-        const uint32_t pa = tbase + P0 + Cfg::kPCols * pb;
+      if (warp == 1) {
+        const uint32_t id_qk = idesc_bf16(128, TN, 0, 0);
+        const uint64_t qrope_desc = kPair ? sdesc_sw64(qrope_base, 512) : sdesc_sw128(qrope_base, 16, 1024);
+        while (ok && cur.next(sa, sg)) {
+          for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
+            const int st = static_cast<int>(n % KS);
+            if (!mbar_wait(smem_u32(&sm.full[st]), static_cast<uint32_t>((n / KS) & 1), wc, LKV_WAIT(W_FULL)) ||
+                (n > 0 && !mbar_wait(smem_u32(&sm.s_free), static_cast<uint32_t>((n - 1) & 1), wc, LKV_WAIT(W_SFREE))) ||
+                (t == sg.tile_lo &&
+                 !mbar_wait(smem_u32(&sm.q_ready), static_cast<uint32_t>(seg & 1), wc, LKV_WAIT(W_QREADY)))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t kdesc = sdesc_sw128(stage_base + st * kStageBytes, 16, 1024);
 #pragma unroll
-        for (int kk = 0; kk < TN / 16; ++kk)
-          umma_ts(tbase, pa + kk * 8, desc_add(vdesc, kk * 2048), id_pv, (pend_first && kk == 0) ? 0u : 1u);
-        umma_commit(smem_u32(&sm.o_done[pb]));
-        umma_commit(kSplit ? smem_u32(&sm.vempty[pend_n % VS]) : smem_u32(&sm.empty[pend_n % KS]));
-        pq_head ^= 1;
-        --pq_len;
-        return true;
-      };
-      while (ok && cur.next(sa, sg)) {
-        for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
-          const int st = static_cast<int>(n % KS);
-          if (!mbar_wait(smem_u32(&sm.full[st]), static_cast<uint32_t>((n / KS) & 1), wc, LKV_WAIT(W_FULL)) ||
-              (n > 0 && !mbar_wait(smem_u32(&sm.s_free), static_cast<uint32_t>((n - 1) & 1), wc, LKV_WAIT(W_SFREE))) ||
-              (t == sg.tile_lo &&
-               !mbar_wait(smem_u32(&sm.q_ready), static_cast<uint32_t>(seg & 1), wc, LKV_WAIT(W_QREADY)))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t kdesc = sdesc_sw128(stage_base + st * kStageBytes, 16, 1024);
-#pragma unroll
-          for (int ks = 0; ks < 4 * Cfg::kNope; ++ks) {
-            const int bx = ks >> 2, kk = ks & 3;
-            if (ks < n_tm)
+            for (int ks = 0; ks < 4 * Cfg::kNope; ++ks) {
+              const int bx = ks >> 2, kk = ks & 3;
               umma_ts(tbase + S0, tbase + Q0 + bx * 32 + kk * 8, desc_add(kdesc, bx * kBoxBytes + kk * 32), id_qk,
                       ks ? 1u : 0u);
-          }
+            }
+            const uint32_t rope_addr = stage_base + st * kStageBytes + Cfg::kRopeBox * kBoxBytes;
+            const uint64_t rdesc = kPair ? sdesc_sw64(rope_addr, 512) : sdesc_sw128(rope_addr, 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            if (kk >= kk0)
-              umma_ss(tbase + S0, desc_add(qrope_desc, kk * 32), desc_add(kdesc, Cfg::kRopeBox * kBoxBytes + kk * 32),
-                      id_qk, 1u);
-          umma_commit(smem_u32(&sm.s_full));
-          if (kSplit) umma_commit(smem_u32(&sm.empty[st]));  // the K slot is free once QK is done
-          if (pq_len == kLag && !issue_pv()) {
-            ok = false;
-            break;
+            for (int kk = 0; kk < Cfg::kRopeSteps; ++kk)
+              umma_ss(tbase + S0, desc_add(qrope_desc, kk * 32), desc_add(rdesc, kk * 32), id_qk, 1u);
+            umma_commit(smem_u32(&sm.s_full));
+            if (kSplit) umma_commit(smem_u32(&sm.empty[st]));  // the K slot is free once QK is done
           }
-          const int tail = (pq_head + pq_len) & 1;
-          pq_n[tail] = n;
-          pq_first[tail] = (t == sg.tile_lo);
-          pq_seg[tail] = seg;
-          ++pq_len;
+          ++seg;
         }
-        ++seg;
+      } else {
+        const uint32_t id_pv = idesc_bf16(128, DV, 0, 1);
+        while (ok && cur.next(sa, sg)) {
+          for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
+            const int pb = static_cast<int>(n & 1);
+            const bool first = (t == sg.tile_lo);
+            if (!mbar_wait(smem_u32(&sm.p_full[pb]), static_cast<uint32_t>((n >> 1) & 1), wc, LKV_WAIT(W_PFULL)) ||
+                (first && seg > 0 &&
+                 !mbar_wait(smem_u32(&sm.o_free), static_cast<uint32_t>((seg - 1) & 1), wc, LKV_WAIT(W_OFREE))) ||
+                (kSplit && !mbar_wait(smem_u32(&sm.vfull[n % VS]), static_cast<uint32_t>((n / VS) & 1), wc,
+                                      LKV_WAIT(W_FULL)))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            // P(n) exists only after S(n) was read, so QK(n) is complete and the whole stage
+            // (K and V, where they share it) is free once this PV completes
+            const uint32_t vaddr = kSplit ? vring_base + static_cast<uint32_t>(n % VS) * Cfg::kVStageBytes
+                                          : stage_base + static_cast<uint32_t>(n % KS) * kStageBytes;
+            const uint64_t vdesc = sdesc_sw128(vaddr + Cfg::kVBox0 * kBoxBytes, kBoxBytes, 1024);
+            const uint32_t pa = tbase + P0 + Cfg::kPCols * pb;
+#pragma unroll
+            for (int kk = 0; kk < TN / 16; ++kk)
+              umma_ts(tbase, pa + kk * 8, desc_add(vdesc, kk * 2048), id_pv, (first && kk == 0) ? 0u : 1u);
+            umma_commit(smem_u32(&sm.o_done[pb]));
+            umma_commit(kSplit ? smem_u32(&sm.vempty[n % VS]) : smem_u32(&sm.empty[n % KS]));
+          }
+          ++seg;
+        }
       }
-      while (ok && pq_len > 0) ok = issue_pv();
-      // all tcgen05 work of this thread done before TMEM is released
+      // all tcgen05 work of both issuers done before TMEM is released
       umma_commit(smem_u32(&sm.drain));
       uint32_t zero = 0;
       const WaitCtl dc{&zero, p.err, p.wait_limit_ns};
       mbar_wait(smem_u32(&sm.drain), 0, dc, LKV_WAIT(W_DRAIN));
     }
-  } else if (warp >= 4 && (warp - 4) < n_sm_warps) {
-    // ============================================================ softmax / epilogue
-    const int r = tid - 128;                 // row == TMEM lane
-    const uint32_t lb = static_cast<uint32_t>((warp & 3) * 32);
-    const bool row_ok = r < p.R;
+  } else if (kPair && warp == 3) {
+    // ============================================================ MLA message sender
+    // Copies each staged score message into the peer's slot with st.async (each store completes
+    // its bytes on the peer's x_full), so the softmax warps never wait on the cluster network.
+    const int h = lane;
     const uint32_t peer = rank ^ 1u;
-    uint32_t rbuf_remote[2] = {0u, 0u}, xfull_remote[2] = {0u, 0u}, xfree_remote[2] = {0u, 0u};
-    if (kPair) {
-      for (int b = 0; b < 2; ++b) {
-        rbuf_remote[b] = map_to_peer(smem_u32(rbuf + b * kMsgBytes), peer);
-        xfull_remote[b] = map_to_peer(smem_u32(&sm.x_full[b]), peer);
-        xfree_remote[b] = map_to_peer(smem_u32(&sm.x_free[b]), peer);
+    uint32_t rrem[kMsgSlots], xrem[kMsgSlots];
+#pragma unroll
+    for (int b = 0; b < kMsgSlots; ++b) {
+      rrem[b] = map_to_peer(smem_u32(rbuf + b * kMsgBytes), peer);
+      xrem[b] = map_to_peer(smem_u32(&sm.x_full[b]), peer);
+    }
+    SegCursor cur = cur0;
+    Segment sg;
+    long long m = 0;
+    bool ok = true;
+    while (ok && cur.next(sa, sg)) {
+      for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++m) {
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.x_staged), static_cast<uint32_t>(m & 1), wc,
+                                                LKV_WAIT(W_XSTAGED)))) {
+          ok = false;
+          break;
+        }
+        // Two batches of kChunks 16-byte chunks: chunk lane + 32 i (a warp reads 512 contiguous
+        // bytes per load), then the second half of the message.
+        constexpr int kChunks = kMsgBytes / 16 / 64;
+        static_assert(kChunks * 64 * 16 == kMsgBytes, "message chunking");
+        const uint4* src = reinterpret_cast<const uint4*>(sbuf);
+        uint4 v[kChunks];
+#pragma unroll
+        for (int i = 0; i < kChunks; ++i) v[i] = src[h + 32 * i];
+        // the peer's slot for message m is free once this CTA has read the peer's message m-1.
+        // Releasing the staging copy only after this wait keeps the softmax from reading
+        // message m (which it does after staging m+1) before the wait: x_consumed then never
+        // runs two phases ahead of the parity tested here.
+        if (m >= 1 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.x_consumed), static_cast<uint32_t>((m - 1) & 1),
+                                                          wc, LKV_WAIT(W_XSTAGED)))) {
+          ok = false;
+          break;
+        }
+        const int xb = static_cast<int>(m % kMsgSlots);
+#pragma unroll
+        for (int i = 0; i < kChunks; ++i) st_async_v4(rrem[xb] + 16u * static_cast<uint32_t>(h + 32 * i), v[i], xrem[xb]);
+#pragma unroll
+        for (int i = 0; i < kChunks; ++i) v[i] = src[h + 32 * (kChunks + i)];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.x_stage_free));
+#pragma unroll
+        for (int i = 0; i < kChunks; ++i)
+          st_async_v4(rrem[xb] + 16u * static_cast<uint32_t>(h + 32 * (kChunks + i)), v[i], xrem[xb]);
       }
     }
+  } else if (warp >= 4 && warp < 12 && ((warp - 4) & 3) < n_row_warps) {
+    // ============================================================ softmax / epilogue
+    const int q4 = (warp - 4) & 3;             // TMEM lane quadrant
+    const int hf = (warp - 4) >> 2;            // key-column half of the tile
+    const int r = q4 * 32 + lane;              // row == TMEM lane
+    const uint32_t lb = static_cast<uint32_t>(q4 * 32);
+    const bool row_ok = r < p.R;
+    const int sidx = hf * n_row_warps * 32 + r;  // 0 .. n_sm_threads-1
     const int col_base = kPair ? 256 * static_cast<int>(rank) : 0;
+    constexpr int HC = TN / 2;                 // key columns of this thread per tile
+    constexpr int HW = HC / 2;                 // packed fp16 / bf16 pairs
+    const int c0 = hf * HC;
 
     // every lane of a softmax warp takes the same branch after a wait (tcgen05.ld/st are
     // warp-collective), so a wait that gives up in one lane ends the loop in all of them
@@ -437,6 +531,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     auto wait_all_cl = [&](uint32_t bar, uint32_t par, int site) -> bool {
       return __all_sync(0xffffffffu, mbar_wait<true>(bar, par, wc, site)) != 0;
     };
+    // Swap one value per row with the other column half of this quadrant (double-buffered,
+    // bounded wait: a partner that gave up ends this warp's loop too).
+    int xc = 0;
+    auto pair_xchg = [&](float v, float& other) -> bool {
+      const int b = xc & 1;
+      sm.xch[b][hf][r] = v;
+      warp_arrive(smem_u32(&sm.xbar[q4][b]));
+      const bool okx = wait_all(smem_u32(&sm.xbar[q4][b]), static_cast<uint32_t>((xc >> 1) & 1), LKV_WAIT(W_XCHG));
+      other = sm.xch[b][hf ^ 1][r];
+      ++xc;
+      return okx;
+    };
     // (query token, head) of this row in a unit
     auto row_map = [&](const Segment& sg, int& i, int& h) {
       if (kPair) {
@@ -447,14 +553,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         h = sg.k * p.hpg + (r % p.hpg);
       }
     };
-    // Stage the unit's query: non-RoPE part into TMEM (A operand), RoPE part into the
-    // swizzled shared-memory A operand.
+    // Stage the unit's query: non-RoPE part into TMEM (A operand; each half writes every
+    // other 64-column box), RoPE part (half 0) into the swizzled shared-memory A operand.
     auto load_q = [&](const Segment& sg) {
       int i, h;
       row_map(sg, i, h);
       const size_t qrow = (static_cast<size_t>(sg.b) * p.s_q + i) * p.h_q + h;
 #pragma unroll 1
-      for (int bx = 0; bx < Cfg::kNope; ++bx) {
+      for (int bx = hf; bx < Cfg::kNope; bx += 2) {
         uint32_t w[32];
         if (row_ok) {
           const uint4* src = reinterpret_cast<const uint4*>(p.q_nope + qrow * p.dq + col_base + 64 * bx);
@@ -472,14 +578,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tmem_st32(tm_addr(tbase, lb, Q0 + bx * 32), w);
       }
-      {
-        // RoPE part, or (MLA rank 1) latent columns 192..255 of which K-steps 2 and 3 are used
-        const uint4* src = reinterpret_cast<const uint4*>(
-            (kPair && rank == 1) ? p.q_nope + qrow * p.dq + 192 : p.q_rope + qrow * 64);
+      if (hf == 0) {
+        if (kPair) {
+          // this CTA's 32-column RoPE half, 64-byte swizzle: chunk c of row r at c ^ ((r / 2) % 4)
+          const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + qrow * 64 + 32 * rank);
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 x = row_ok ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-          *reinterpret_cast<uint4*>(qrope_smem + r * 128 + ((c ^ (r & 7)) << 4)) = x;
+          for (int c = 0; c < 4; ++c) {
+            const uint4 x = row_ok ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(qrope_smem + r * 64 + ((c ^ ((r >> 1) & 3)) << 4)) = x;
+          }
+        } else {
+          const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + qrow * 64);
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 x = row_ok ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(qrope_smem + r * 128 + ((c ^ (r & 7)) << 4)) = x;
+          }
         }
         fence_proxy_async_smem();
       }
@@ -488,33 +602,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       warp_arrive(smem_u32(&sm.q_ready));
     };
 
+    // Running max (shared by both halves of a row) and this half's running sum.
     float m_run = -INFINITY, l_run = 0.f;
-    // Grouped modes: softmax of one tile whose scores are in s[] -> P bits in pw[], the running
-    // max / sum updated; `alpha` rescales O when the running max moved.
-    auto softmax_tile = [&](float (&s)[TN], const Segment& sg, int t, int qi, uint32_t (&pw)[TN / 2],
-                            bool& rescale, float& alpha) {
-      if (t == sg.tile_lo) {
-        m_run = -INFINITY;
-        l_run = 0.f;
-      }
-      const int lim = sg.L - p.s_q + qi + 1;  // keys visible to this row
-      const int key0 = t * TN;
-      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (key0 + TN <= lim) {
-#pragma unroll
-        for (int c = 0; c < TN; ++c) {
-          s[c] *= p.sl2;
-          m4[c & 3] = fmaxf(m4[c & 3], s[c]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < TN; ++c) {
-          s[c] = (key0 + c < lim) ? s[c] * p.sl2 : -INFINITY;
-          m4[c & 3] = fmaxf(m4[c & 3], s[c]);
-        }
-      }
-      const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-      // lazy rescale: keep the running max unless the tile max exceeds it by 2^8
+    // Lazy rescale: keep the running max unless the tile max exceeds it by 2^8.
+    auto new_max = [&](float mx, bool& rescale, float& alpha) -> float {
       rescale = false;
       float m_new = m_run;
       if (mx > m_run + 8.f) {
@@ -522,10 +613,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         rescale = (m_run != -INFINITY);
       }
       alpha = rescale ? ex2_approx(m_run - m_new) : 1.f;
+      return m_new;
+    };
+    // Grouped modes: softmax of this half of one tile whose scores are in s[] -> P bits in
+    // pw[], the running max / sum updated; `alpha` rescales O when the running max moved.
+    auto softmax_tile = [&](float (&s)[HC], const Segment& sg, int t, int qi, uint32_t (&pw)[HW], bool& rescale,
+                            float& alpha) -> bool {
+      if (t == sg.tile_lo) {
+        m_run = -INFINITY;
+        l_run = 0.f;
+      }
+      const int lim = sg.L - p.s_q + qi + 1;  // keys visible to this row
+      const int key0 = t * TN + c0;
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (key0 + HC <= lim) {
+#pragma unroll
+        for (int c = 0; c < HC; ++c) {
+          s[c] *= p.sl2;
+          m4[c & 3] = fmaxf(m4[c & 3], s[c]);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < HC; ++c) {
+          s[c] = (key0 + c < lim) ? s[c] * p.sl2 : -INFINITY;
+          m4[c & 3] = fmaxf(m4[c & 3], s[c]);
+        }
+      }
+      const float mh = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      float mo;
+      if (!pair_xchg(mh, mo)) return false;
+      const float m_new = new_max(fmaxf(mh, mo), rescale, alpha);
       const float msub = (m_new == -INFINITY) ? 0.f : m_new;
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < TN / 2; ++c) {
+      for (int c = 0; c < HW; ++c) {
         const uint32_t h = ex2_f16x2(s[2 * c] - msub, s[2 * c + 1] - msub);
         const float e0 = f16_lo(h), e1 = f16_hi(h);
         s4[c & 3] += e0 + e1;
@@ -533,28 +654,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       l_run = l_run * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
       m_run = m_new;
+      return true;
     };
     // MLA pair: P = E_own * E_peer * 2^(t_own + t_peer - M) where E = exp2(partial - t) (fp16) of
-    // each CTA's half of the contraction and t its partial tile max (t_own + t_peer bounds the
-    // tile max of the full score).  Products of two floats commute, so both CTAs get the same P.
-    auto combine_tile = [&](const uint32_t (&eo)[32], const uint32_t (&ep)[32], float t_o, float t_p,
-                            const Segment& sg, int t, uint32_t (&pw)[TN / 2], bool& rescale, float& alpha) {
+    // each CTA's half of the contraction and t its partial max over this column half of the
+    // tile (t_own + t_peer bounds the full scores there).  Products of two floats commute, so
+    // both CTAs get the same P.
+    auto combine_tile = [&](const uint32_t (&eo)[HW], const uint32_t (&ep)[HW], float t_o, float t_p,
+                            const Segment& sg, int t, uint32_t (&pw)[HW], bool& rescale, float& alpha) -> bool {
       if (t == sg.tile_lo) {
         m_run = -INFINITY;
         l_run = 0.f;
       }
-      const float T = t_o + t_p;  // -inf when every key of this tile is masked for the row
-      rescale = false;
-      float m_new = m_run;
-      if (T > m_run + 8.f) {
-        m_new = T;
-        rescale = (m_run != -INFINITY);
-      }
-      alpha = rescale ? ex2_approx(m_run - m_new) : 1.f;
+      const float T = t_o + t_p;  // -inf when every key of this half is masked for the row
+      float To;
+      if (!pair_xchg(T, To)) return false;
+      const float m_new = new_max(fmaxf(T, To), rescale, alpha);
       const float f = (T == -INFINITY) ? 0.f : ex2_approx(T - m_new);
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < 32; ++c) {
+      for (int c = 0; c < HW; ++c) {
         const float e0 = f16_lo(eo[c]) * f16_lo(ep[c]) * f;
         const float e1 = f16_hi(eo[c]) * f16_hi(ep[c]) * f;
         s4[c & 3] += e0 + e1;
@@ -562,10 +681,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       l_run = l_run * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
       m_run = m_new;
+      return true;
     };
-    // Common tail of a tile: publish P(n) (after the PV that last read its buffer), rescale O if
-    // the running max moved, and run the segment epilogue after the unit's last tile here.
-    auto finish_tile = [&](uint32_t (&pw)[TN / 2], bool rescale, float alpha, const Segment& sg, int t,
+    // Common tail of a tile: publish this half of P(n) (after the PV that last read its
+    // buffer), rescale this half of O's columns if the running max moved, and run the segment
+    // epilogue after the unit's last tile here.
+    auto finish_tile = [&](uint32_t (&pw)[HW], bool rescale, float alpha, const Segment& sg, int t,
                            long long n) -> bool {
       int qi, qh;
       row_map(sg, qi, qh);
@@ -580,7 +701,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           return false;
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < DV; c += 32) {
+        for (int c = hf * (DV / 2); c < (hf + 1) * (DV / 2); c += 32) {
           uint32_t o[32];
           tmem_ld32(tm_addr(tbase, lb, c), o);
           tmem_wait_ld();
@@ -590,12 +711,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
       tc_fence_after();
+      {
+        const uint32_t pcol = P0 + Cfg::kPCols * pb + hf * HW;
+        if constexpr (HW == 16) {
+          tmem_st16(tm_addr(tbase, lb, pcol), pw);
+        } else {
 #pragma unroll
-      for (int c = 0; c < TN / 2; c += 32) {
-        uint32_t w[32];
+          for (int c = 0; c < HW; c += 32) {
+            uint32_t w[32];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) w[j] = pw[c + j];
-        tmem_st32(tm_addr(tbase, lb, P0 + Cfg::kPCols * pb + c), w);
+            for (int j = 0; j < 32; ++j) w[j] = pw[c + j];
+            tmem_st32(tm_addr(tbase, lb, pcol + c), w);
+          }
+        }
       }
       if (key0 + TN > sg.keys) {
         // Rows past the unit's last key belong to another request or to unwritten cache:
@@ -606,7 +734,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           return false;  // the copy must land before it is overwritten
         uint8_t* vb = (kSplit ? vring + (n % VS) * Cfg::kVStageBytes : dsm + (n % KS) * kStageBytes) +
                       Cfg::kVBox0 * kBoxBytes;
-        for (int idx = r; idx < per_box * Cfg::kNV; idx += n_sm_threads) {
+        for (int idx = sidx; idx < per_box * Cfg::kNV; idx += n_sm_threads) {
           const int bx = idx / per_box, rem = idx % per_box;
           *reinterpret_cast<uint4*>(vb + bx * kBoxBytes + (first + rem / 8) * 128 + (rem % 8) * 16) =
               make_uint4(0u, 0u, 0u, 0u);
@@ -618,16 +746,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       warp_arrive(smem_u32(&sm.p_full[pb]));
       if (t != sg.tile_hi - 1) return true;
       // ---------------------------------------------------------- segment epilogue
+      float l_other;
+      if (!pair_xchg(l_run, l_other)) return false;
+      const float l_tot = l_run + l_other;
       if (!wait_all(smem_u32(&sm.o_done[pb]), static_cast<uint32_t>((n >> 1) & 1), LKV_WAIT(W_ODONE)))
         return false;
       tc_fence_after();
-      const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
-      const float lse_v = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      const float lse_v = l_tot > 0.f ? (m_run + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
       const size_t orow = (static_cast<size_t>(sg.b) * p.s_q + qi) * p.h_q + qh;
       if (sg.complete) {
         __nv_bfloat16* dst = p.out + orow * p.dv_total + col_base;
 #pragma unroll 1
-        for (int c = 0; c < DV; c += 32) {
+        for (int c = hf * (DV / 2); c < (hf + 1) * (DV / 2); c += 32) {
           uint32_t o[32];
           tmem_ld32(tm_addr(tbase, lb, c), o);
           tmem_wait_ld();
@@ -644,12 +775,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             }
           }
         }
-        if (row_ok && rank == 0) p.lse[orow] = lse_v;
+        if (row_ok && rank == 0 && hf == 0) p.lse[orow] = lse_v;
       } else {
         const size_t prow = static_cast<size_t>(2 * range + sg.slot) * p.rmax + r;
         float* dst = p.part_o + prow * p.dv_total + col_base;
 #pragma unroll 1
-        for (int c = 0; c < DV; c += 32) {
+        for (int c = hf * (DV / 2); c < (hf + 1) * (DV / 2); c += 32) {
           uint32_t o[32];
           tmem_ld32(tm_addr(tbase, lb, c), o);
           tmem_wait_ld();
@@ -661,8 +792,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                   __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
           }
         }
-        if (row_ok && rank == 0) p.part_lse[prow] = lse_v;
-        if (r == 0 && rank == 0) p.seg_info[2 * range + sg.slot] = sg.unit_id;
+        if (row_ok && rank == 0 && hf == 0) p.part_lse[prow] = lse_v;
+        if (r == 0 && rank == 0 && hf == 0) p.seg_info[2 * range + sg.slot] = sg.unit_id;
       }
       tc_fence_before();
       warp_arrive(smem_u32(&sm.o_free));
@@ -675,22 +806,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     int tA = haveA ? sgA.tile_lo : 0;
     long long nA = 0;
     // MLA: tile whose own half has been sent and whose peer half is awaited
-    uint32_t eprev[32];
+    uint32_t eprev[HW];
     float tprev = -INFINITY;
     Segment sgB;
     int tB = 0;
     long long nB = 0;
     bool haveB = false;
-    long long nconsumed = 0;  // incoming messages read (MLA)
+    long long nconsumed = 0, nsent = 0;  // MLA messages read from / sent to the peer
     bool ok = true;
     if (haveA) load_q(sgA);
     while (ok && (haveA || haveB)) {
-      float cs[TN];
+      float cs[HC];
       bool gotA = false;
       Segment sgAc;
       int tAc = 0;
       long long nAc = 0;
-      uint32_t ecur[32];
+      uint32_t ecur[HW];
       float tcur = -INFINITY;
       if (haveA) {
         if (!wait_all(smem_u32(&sm.s_full), static_cast<uint32_t>(nA & 1), LKV_WAIT(W_SFULL))) {
@@ -699,9 +830,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < TN; c += 32) {
+        for (int c = 0; c < HC; c += 32) {
           uint32_t a[32];
-          tmem_ld32(tm_addr(tbase, lb, S0 + c), a);
+          tmem_ld32(tm_addr(tbase, lb, S0 + c0 + c), a);
 #pragma unroll
           for (int j = 0; j < 32; ++j) cs[c + j] = __uint_as_float(a[j]);
         }
@@ -716,20 +847,20 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           if (have_nx) load_q(nx);
         }
         if constexpr (kPair) {
-          // own half: mask, partial tile max, E = exp2(partial - max) in bf16
-          const int xb = static_cast<int>(nA & 1);
-          if (r == 0) mbar_arrive_expect_tx(smem_u32(&sm.x_full[xb]), kMsgBytes);  // the peer's half of nA
-          const int lim = sgA.keys, key0 = tA * TN;
+          // own half: mask, partial max over this column half, E = exp2(partial - max) in fp16
+          const int xb = static_cast<int>(nA % kMsgSlots);
+          if (r == 0 && hf == 0) mbar_arrive_expect_tx(smem_u32(&sm.x_full[xb]), kMsgBytes);  // the peer's half of nA
+          const int lim = sgA.keys, key0 = tA * TN + c0;
           float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-          if (key0 + TN <= lim) {
+          if (key0 + HC <= lim) {
 #pragma unroll
-            for (int c = 0; c < TN; ++c) {
+            for (int c = 0; c < HC; ++c) {
               cs[c] *= p.sl2;
               m4[c & 3] = fmaxf(m4[c & 3], cs[c]);
             }
           } else {
 #pragma unroll
-            for (int c = 0; c < TN; ++c) {
+            for (int c = 0; c < HC; ++c) {
               cs[c] = (key0 + c < lim) ? cs[c] * p.sl2 : -INFINITY;
               m4[c & 3] = fmaxf(m4[c & 3], cs[c]);
             }
@@ -737,28 +868,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tcur = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
           const float tsub = (tcur == -INFINITY) ? 0.f : tcur;
 #pragma unroll
-          for (int c = 0; c < 32; ++c) ecur[c] = ex2_f16x2(cs[2 * c] - tsub, cs[2 * c + 1] - tsub);
-          // our outgoing buffer xb (and the peer's incoming one) are free once message nA-2 was read
-          if (nA >= 2 && !wait_all_cl(smem_u32(&sm.x_free[xb]), static_cast<uint32_t>(((nA - 2) >> 1) & 1),
-                                      LKV_WAIT(W_XFREE))) {
+          for (int c = 0; c < HW; ++c) ecur[c] = ex2_f16x2(cs[2 * c] - tsub, cs[2 * c + 1] - tsub);
+          // stage the message for the sender warps (they read message nA-1 out of it first);
+          // row r is 8 chunks of 16 bytes (this half's 4), XOR-swizzled by r so that the
+          // reader's loads avoid bank conflicts
+          if (nA >= 1 && !wait_all(smem_u32(&sm.x_stage_free), static_cast<uint32_t>((nA - 1) & 1), LKV_WAIT(W_XFREE))) {
             ok = false;
             break;
           }
-          uint8_t* msg = sbuf + xb * kMsgBytes;
 #pragma unroll
-          for (int c = 0; c < 8; ++c)
-            *reinterpret_cast<uint4*>(msg + r * 128 + ((c ^ (r & 7)) << 4)) =
+          for (int c = 0; c < HW / 4; ++c)
+            *reinterpret_cast<uint4*>(sbuf + r * 128 + (((4 * hf + c) ^ (r & 7)) << 4)) =
                 make_uint4(ecur[4 * c], ecur[4 * c + 1], ecur[4 * c + 2], ecur[4 * c + 3]);
-          reinterpret_cast<float*>(msg + 128 * 128)[r] = tcur;
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            // each warp ships its own 32 rows and their tile maxima
-            const uint32_t w0 = static_cast<uint32_t>(r & ~31);
-            bulk_copy_to_peer(rbuf_remote[xb] + w0 * 128, smem_u32(msg) + w0 * 128, 32 * 128, xfull_remote[xb]);
-            bulk_copy_to_peer(rbuf_remote[xb] + 128 * 128 + w0 * 4, smem_u32(msg) + 128 * 128 + w0 * 4, 128,
-                              xfull_remote[xb]);
-          }
+          reinterpret_cast<float*>(sbuf + 128 * 128)[hf * 128 + r] = tcur;
+          warp_arrive(smem_u32(&sm.x_staged));
+          ++nsent;
         }
         gotA = true;
         sgAc = sgA;
@@ -776,32 +900,29 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       if constexpr (kPair) {
         if (haveB) {
-          const int xb = static_cast<int>(nB & 1);
-          if (!wait_all_cl(smem_u32(&sm.x_full[xb]), static_cast<uint32_t>((nB >> 1) & 1), LKV_WAIT(W_XFULL))) {
+          const int xb = static_cast<int>(nB % kMsgSlots);
+          if (!wait_all_cl(smem_u32(&sm.x_full[xb]), static_cast<uint32_t>((nB / kMsgSlots) & 1), LKV_WAIT(W_XFULL))) {
             ok = false;
             break;
           }
           const uint8_t* msg = rbuf + xb * kMsgBytes;
-          uint32_t ep[32];
+          uint32_t ep[HW];
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 x = *reinterpret_cast<const uint4*>(msg + r * 128 + ((c ^ (r & 7)) << 4));
+          for (int c = 0; c < HW / 4; ++c) {
+            const uint4 x = *reinterpret_cast<const uint4*>(msg + r * 128 + (((4 * hf + c) ^ (r & 7)) << 4));
             ep[4 * c] = x.x;
             ep[4 * c + 1] = x.y;
             ep[4 * c + 2] = x.z;
             ep[4 * c + 3] = x.w;
           }
-          const float tpeer = reinterpret_cast<const float*>(msg + 128 * 128)[r];
+          const float tpeer = reinterpret_cast<const float*>(msg + 128 * 128)[hf * 128 + r];
           ++nconsumed;
-          // this warp's rows of the incoming message are read: one of the 4 arrivals that let
-          // the peer reuse both copies of buffer xb
-          __syncwarp();
-          if (lane == 0) mbar_arrive_remote(xfree_remote[xb]);
-          uint32_t pw[TN / 2];
+          warp_arrive(smem_u32(&sm.x_consumed));
+          uint32_t pw[HW];
           bool rescale;
           float alpha;
-          combine_tile(eprev, ep, tprev, tpeer, sgB, tB, pw, rescale, alpha);
-          if (!finish_tile(pw, rescale, alpha, sgB, tB, nB)) {
+          if (!combine_tile(eprev, ep, tprev, tpeer, sgB, tB, pw, rescale, alpha) ||
+              !finish_tile(pw, rescale, alpha, sgB, tB, nB)) {
             ok = false;
             break;
           }
@@ -809,7 +930,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         haveB = gotA;
         if (gotA) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) eprev[c] = ecur[c];
+          for (int c = 0; c < HW; ++c) eprev[c] = ecur[c];
           tprev = tcur;
           sgB = sgAc;
           tB = tAc;
@@ -818,25 +939,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       } else if (gotA) {
         int qi, qh;
         row_map(sgAc, qi, qh);
-        uint32_t pw[TN / 2];
+        uint32_t pw[HW];
         bool rescale;
         float alpha;
-        softmax_tile(cs, sgAc, tAc, qi, pw, rescale, alpha);
-        if (!finish_tile(pw, rescale, alpha, sgAc, tAc, nAc)) {
+        if (!softmax_tile(cs, sgAc, tAc, qi, pw, rescale, alpha) || !finish_tile(pw, rescale, alpha, sgAc, tAc, nAc)) {
           ok = false;
           break;
         }
       }
     }
-    if (kPair && !ok && r == 0) {
-      // After giving up, the peer may still have up to two messages on their way into this
-      // CTA's shared memory (it sends message m once message m-2 was read here).  Let them
-      // land (bounded) before the CTA can exit; every message is armed exactly once.
+    if (kPair && !ok && r == 0 && hf == 0) {
+      // After giving up, the peer may still write messages into this CTA's shared memory: it
+      // sends message m once it has read this CTA's message m-1, so at most up to message
+      // nsent (messages staged here bound those sent).  Let them land (bounded) before the
+      // CTA can exit; every message is armed once.
       uint32_t zero = 0;
       const WaitCtl dc{&zero, p.err, p.wait_limit_ns};
-      for (long long m = nconsumed; m < nconsumed + 2; ++m) {
-        if (m >= nA) mbar_arrive_expect_tx(smem_u32(&sm.x_full[m & 1]), kMsgBytes);
-        mbar_wait<true>(smem_u32(&sm.x_full[m & 1]), static_cast<uint32_t>((m >> 1) & 1), dc, LKV_WAIT(W_DRAIN));
+      for (long long m = nconsumed; m < nsent + 1; ++m) {
+        if (m >= nA) mbar_arrive_expect_tx(smem_u32(&sm.x_full[m % kMsgSlots]), kMsgBytes);
+        mbar_wait<true>(smem_u32(&sm.x_full[m % kMsgSlots]), static_cast<uint32_t>((m / kMsgSlots) & 1), dc,
+                        LKV_WAIT(W_DRAIN));
       }
     }
   }

@@ -1,4 +1,4 @@
-// Host-side construction of 2-D TMA tensor maps (bf16, 128-byte swizzle) through the
+// Host-side construction of 2-D TMA tensor maps (bf16, 128- or 64-byte swizzle) through the
 // driver entry point obtained from the runtime, so the library links only cudart.
 #pragma once
 #include <cstdint>
@@ -26,10 +26,12 @@ inline EncodeTiledFn encode_tiled_fn() {
 }
 
 // Map a row-major bf16 matrix [rows, cols] with a row stride of `row_stride_bytes`
-// as tiles of box_cols (<= 64) x box_rows, 128-byte swizzled, zero fill outside.
+// as tiles of box_cols x box_rows, zero fill outside: 128-byte swizzled for box_cols = 64,
+// 64-byte swizzled for box_cols = 32.
 // Returns false if the driver rejects it (alignment, stride or extent).
 inline bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
                            uint64_t row_stride_bytes, uint32_t box_cols, uint32_t box_rows) {
+  if (box_cols != 64 && box_cols != 32) return false;
   EncodeTiledFn fn = encode_tiled_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {cols, rows};
@@ -37,7 +39,8 @@ inline bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t cols, uint
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
