@@ -32,6 +32,8 @@
  *     a destination row past the cache) never trap: the kernel records a site code in a
  *     device error word, skips the bad access and unwinds.  lkv_check_device() reads it.
  *   - "bf16" means bf16 storage with fp32 accumulation; lse is always fp32, natural log.
+ *   - scale must be finite and > 0 (the pages' softmax scale is 1/sqrt of the score width);
+ *     a positive scale keeps the order of the raw scores, which the kernels rely on.
  *   - Row strides are in elements and must keep every row 16-byte aligned.
  */
 #ifndef LKV_H

@@ -168,7 +168,7 @@ lkv_status common_checks(const void* q, const void* qr, const int32_t* cu, const
   if (s_q != 1 && s_q != 2) return LKV_ERR_UNSUPPORTED;
   if (h_q % groups) return LKV_ERR_INVALID_ARG;
   if (dtype != LKV_BF16 && dtype != LKV_FP32) return LKV_ERR_INVALID_ARG;
-  if (!std::isfinite(scale)) return LKV_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return LKV_ERR_INVALID_ARG;
   if (cache_rows >= (1LL << 31)) return LKV_ERR_UNSUPPORTED;
   if (static_cast<long long>(batch) * s_q * h_q >= (1LL << 31)) return LKV_ERR_UNSUPPORTED;
   return LKV_OK;

@@ -317,7 +317,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       SegCursor cur = cur0;
       Segment sg;
-      long long n = 0, nv = 0;   // K (or whole) tiles and V tiles issued
+      int n = 0, nv = 0;   // K (or whole) tiles and V tiles issued (a CTA's tile count fits an int)
       bool ok = true;
       while (ok && cur.next(sa, sg)) {
         for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
@@ -363,16 +363,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
       // never leave copies in flight into a CTA that is about to exit
-      const long long inflight = n < KS ? n : KS;
+      const int inflight = n < KS ? n : KS;
       uint32_t zero = 0;
       const WaitCtl dc{&zero, p.err, p.wait_limit_ns};  // ignores the abort flag, keeps the limit
-      for (long long m = n - inflight; m < n; ++m)
+      for (int m = n - inflight; m < n; ++m)
         mbar_wait(smem_u32(&sm.full[m % KS]), static_cast<uint32_t>((m / KS) & 1), dc, LKV_WAIT(W_DRAIN));
       if (kSplit) {
         // V copies: issued for every tile whose K was issued, except possibly the last one when
         // its vempty wait gave up; wait only for those actually issued (counted by nv)
-        const long long vin = nv < VS ? nv : VS;
-        for (long long m = nv - vin; m < nv; ++m)
+        const int vin = nv < VS ? nv : VS;
+        for (int m = nv - vin; m < nv; ++m)
           mbar_wait(smem_u32(&sm.vfull[m % VS]), static_cast<uint32_t>((m / VS) & 1), dc, LKV_WAIT(W_DRAIN));
       }
     }
@@ -384,7 +384,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       SegCursor cur = cur0;
       Segment sg;
-      long long n = 0;   // global tile counter
+      int n = 0;         // tile counter of this CTA
       int seg = 0;       // segments started
       bool ok = true;
       if (warp == 1) {
@@ -468,7 +468,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     SegCursor cur = cur0;
     Segment sg;
-    long long m = 0;
+    int m = 0;
     bool ok = true;
     while (ok && cur.next(sa, sg)) {
       for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++m) {
@@ -625,21 +625,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       const int lim = sg.L - p.s_q + qi + 1;  // keys visible to this row
       const int key0 = t * TN + c0;
-      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (key0 + HC <= lim) {
+      // max of the raw scores (the scale is positive), then one FMA per score for the
+      // exponent in log2 units
+      if (key0 + HC > lim) {
 #pragma unroll
-        for (int c = 0; c < HC; ++c) {
-          s[c] *= p.sl2;
-          m4[c & 3] = fmaxf(m4[c & 3], s[c]);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < HC; ++c) {
-          s[c] = (key0 + c < lim) ? s[c] * p.sl2 : -INFINITY;
-          m4[c & 3] = fmaxf(m4[c & 3], s[c]);
-        }
+        for (int c = 0; c < HC; ++c) s[c] = (key0 + c < lim) ? s[c] : -INFINITY;
       }
-      const float mh = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int c = 0; c < HC; ++c) m4[c & 3] = fmaxf(m4[c & 3], s[c]);
+      const float mh = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.sl2;
       float mo;
       if (!pair_xchg(mh, mo)) return false;
       const float m_new = new_max(fmaxf(mh, mo), rescale, alpha);
@@ -647,7 +642,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < HW; ++c) {
-        const uint32_t h = ex2_f16x2(s[2 * c] - msub, s[2 * c + 1] - msub);
+        const uint32_t h = ex2_f16x2(fmaf(s[2 * c], p.sl2, -msub), fmaf(s[2 * c + 1], p.sl2, -msub));
         const float e0 = f16_lo(h), e1 = f16_hi(h);
         s4[c & 3] += e0 + e1;
         pw[c] = pack_bf16x2(e0, e1);
@@ -670,12 +665,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       float To;
       if (!pair_xchg(T, To)) return false;
       const float m_new = new_max(fmaxf(T, To), rescale, alpha);
+      // f = 2^(T - m_new) <= 2^8; products below the fp16 range only drop terms that are
+      // under 2^-24 of the running max
       const float f = (T == -INFINITY) ? 0.f : ex2_approx(T - m_new);
+      const uint32_t f2 = pack_f16x2(f, f);
       float s4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < HW; ++c) {
-        const float e0 = f16_lo(eo[c]) * f16_lo(ep[c]) * f;
-        const float e1 = f16_hi(eo[c]) * f16_hi(ep[c]) * f;
+        const uint32_t pr = mul_f16x2(mul_f16x2(eo[c], ep[c]), f2);
+        const float e0 = f16_lo(pr), e1 = f16_hi(pr);
         s4[c & 3] += e0 + e1;
         pw[c] = pack_bf16x2(e0, e1);
       }
@@ -687,7 +685,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // buffer), rescale this half of O's columns if the running max moved, and run the segment
     // epilogue after the unit's last tile here.
     auto finish_tile = [&](uint32_t (&pw)[HW], bool rescale, float alpha, const Segment& sg, int t,
-                           long long n) -> bool {
+                           int n) -> bool {
       int qi, qh;
       row_map(sg, qi, qh);
       const int key0 = t * TN;
@@ -804,15 +802,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     Segment sgA, nx;
     bool haveA = cur.next(sa, sgA);
     int tA = haveA ? sgA.tile_lo : 0;
-    long long nA = 0;
+    int nA = 0;
     // MLA: tile whose own half has been sent and whose peer half is awaited
     uint32_t eprev[HW];
     float tprev = -INFINITY;
     Segment sgB;
     int tB = 0;
-    long long nB = 0;
+    int nB = 0;
     bool haveB = false;
-    long long nconsumed = 0, nsent = 0;  // MLA messages read from / sent to the peer
+    int nconsumed = 0, nsent = 0;  // MLA messages read from / sent to the peer
     bool ok = true;
     if (haveA) load_q(sgA);
     while (ok && (haveA || haveB)) {
@@ -820,7 +818,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       bool gotA = false;
       Segment sgAc;
       int tAc = 0;
-      long long nAc = 0;
+      int nAc = 0;
       uint32_t ecur[HW];
       float tcur = -INFINITY;
       if (haveA) {
@@ -851,24 +849,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int xb = static_cast<int>(nA % kMsgSlots);
           if (r == 0 && hf == 0) mbar_arrive_expect_tx(smem_u32(&sm.x_full[xb]), kMsgBytes);  // the peer's half of nA
           const int lim = sgA.keys, key0 = tA * TN + c0;
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-          if (key0 + HC <= lim) {
+          if (key0 + HC > lim) {
 #pragma unroll
-            for (int c = 0; c < HC; ++c) {
-              cs[c] *= p.sl2;
-              m4[c & 3] = fmaxf(m4[c & 3], cs[c]);
-            }
-          } else {
-#pragma unroll
-            for (int c = 0; c < HC; ++c) {
-              cs[c] = (key0 + c < lim) ? cs[c] * p.sl2 : -INFINITY;
-              m4[c & 3] = fmaxf(m4[c & 3], cs[c]);
-            }
+            for (int c = 0; c < HC; ++c) cs[c] = (key0 + c < lim) ? cs[c] : -INFINITY;
           }
-          tcur = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int c = 0; c < HC; ++c) m4[c & 3] = fmaxf(m4[c & 3], cs[c]);
+          tcur = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.sl2;  // log2 units
           const float tsub = (tcur == -INFINITY) ? 0.f : tcur;
 #pragma unroll
-          for (int c = 0; c < HW; ++c) ecur[c] = ex2_f16x2(cs[2 * c] - tsub, cs[2 * c + 1] - tsub);
+          for (int c = 0; c < HW; ++c)
+            ecur[c] = ex2_f16x2(fmaf(cs[2 * c], p.sl2, -tsub), fmaf(cs[2 * c + 1], p.sl2, -tsub));
           // stage the message for the sender warps (they read message nA-1 out of it first);
           // row r is 8 chunks of 16 bytes (this half's 4), XOR-swizzled by r so that the
           // reader's loads avoid bank conflicts
@@ -955,7 +947,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       // CTA can exit; every message is armed once.
       uint32_t zero = 0;
       const WaitCtl dc{&zero, p.err, p.wait_limit_ns};
-      for (long long m = nconsumed; m < nsent + 1; ++m) {
+      for (int m = nconsumed; m < nsent + 1; ++m) {
         if (m >= nA) mbar_arrive_expect_tx(smem_u32(&sm.x_full[m % kMsgSlots]), kMsgBytes);
         mbar_wait<true>(smem_u32(&sm.x_full[m % kMsgSlots]), static_cast<uint32_t>((m / kMsgSlots) & 1), dc,
                         LKV_WAIT(W_DRAIN));

@@ -71,6 +71,33 @@ __device__ __forceinline__ bool mbar_test_cluster(uint32_t bar, uint32_t parity)
   return ok != 0;
 }
 
+// The same tests with a suspend-time hint: a thread whose phase is not complete sleeps until
+// the phase completes or `kSuspendNs` pass, instead of spinning on issue slots that the
+// softmax warps sharing its scheduler need.
+constexpr uint32_t kSuspendNs = 10000;
+__device__ __forceinline__ bool mbar_sleep_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "n"(kSuspendNs)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_sleep_test_cluster(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity), "n"(kSuspendNs)
+      : "memory");
+  return ok != 0;
+}
+
 // Wait control shared by every bounded wait of a CTA.  `abort` is a shared-memory flag:
 // once any thread gives up, every later wait in the CTA returns false at once.
 struct WaitCtl {
@@ -85,8 +112,8 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   if (kCluster ? mbar_test_cluster(bar, parity) : mbar_test(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (kCluster ? mbar_test_cluster(bar, parity) : mbar_test(bar, parity)) return true;
-    if ((it & 31u) == 0u) {
+    if (kCluster ? mbar_sleep_test_cluster(bar, parity) : mbar_sleep_test(bar, parity)) return true;
+    if ((it & 7u) == 0u) {
       if (*c.abort) return false;
       if (globaltimer_ns() - t0 > c.limit_ns) {
         record_error(c.err, site);
@@ -352,6 +379,11 @@ __device__ __forceinline__ uint32_t ex2_f16x2(float lo, float hi) {
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint32_t mul_f16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
 }
 __device__ __forceinline__ float f16_lo(uint32_t v) {

@@ -163,6 +163,8 @@ def test_validation_errors_need_no_gpu(lkv):
     assert call(cs=500) == L.ERR_INVALID_ARG          # row stride shorter than r_kv
     assert call(cs=580) == L.ERR_INVALID_ARG          # 1160-byte rows are not 16-byte aligned
     assert call(scale=float("nan")) == L.ERR_INVALID_ARG
+    assert call(scale=0.0) == L.ERR_INVALID_ARG
+    assert call(scale=-0.04) == L.ERR_INVALID_ARG
     assert call(rows=1 << 31) == L.ERR_UNSUPPORTED
     assert call(dt=1, r=2000, cs=2064) == L.ERR_UNSUPPORTED    # fp32 path limit
     # GQLA: h_q not a multiple of g; unsupported head width
