@@ -16,6 +16,8 @@ on a bounded sample of the same workload; under torchrun only rank 0 runs it.
 from __future__ import annotations
 
 import argparse
+import glob
+import hashlib
 import json
 import os
 import statistics
@@ -34,6 +36,31 @@ import synth  # noqa: E402
 
 METRIC = "decode attn tokens/s; KV-cache GB/s & TFLOPS as fraction of B200 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources and the C header: a traffic figure measured with ncu is only
+    reported while the kernels it was measured on are unchanged."""
+    h = hashlib.sha256()
+    files = sorted(glob.glob(os.path.join(ROOT, "latent_kv_cache_split_b200", "csrc", "*")))
+    files.append(os.path.join(ROOT, "include", "lkv.h"))
+    for f in files:
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str):
+    """DRAM bytes (read + write) per decode-kernel launch from an ncu capture recorded in
+    profiles/traffic.json, or None when absent or taken on other kernel sources."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    entry = json.load(open(p)).get(workload)
+    if not entry or entry.get("kernel_hash") != kernel_source_hash():
+        return None
+    return entry.get("dram_bytes_per_launch")
 
 
 def load_peaks():
@@ -310,7 +337,8 @@ def bench_gpu(args, rank, world, local_rank):
             "tflops": tfl,
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak,
                          "unit": "GB/s" if bound == "hbm" else "TFLOP/s", "frac": achieved / peak,
-                         "traffic": None, "peak_source": f"{how} (MEASURED_PEAKS.json burst)",
+                         "traffic": measured_traffic(w.name), "kernel_source_hash": kernel_source_hash(),
+                         "peak_source": f"{how} (MEASURED_PEAKS.json burst)",
                          "roofline_ms": max(t_hbm, t_tc) * 1e3,
                          "frac_of_step_roofline": max(t_hbm, t_tc) * 1e3 / ms,
                          "kernel": "decode_tc_kernel + split combine (one lkv_*_decode call)",
