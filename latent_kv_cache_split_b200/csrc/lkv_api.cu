@@ -76,6 +76,9 @@ int plan_ranges(int kind, int batch, int s_q, int groups, int num_sms) {
   const long long units = static_cast<long long>(batch) * (kind == 0 ? s_q : groups);
   const int pmax = kind == 0 ? num_sms / 2 : num_sms;
   if (pmax <= 0) return -1;
+  // Grouped units run in lockstep (lkv_sched.cuh): G ranges per block of request tiles, as many
+  // blocks as fit on the SMs.
+  if (kind != 0 && groups >= 4) return groups * (num_sms / groups >= 1 ? num_sms / groups : 1);
   // One range per unit when the units alone nearly fill the machine: equal lengths then need
   // no split at all.  Otherwise one range per CTA (pair), cutting long units across SMs.
   if (units <= pmax && 4 * units >= 3LL * pmax) return static_cast<int>(units);
@@ -210,11 +213,17 @@ int lkv_plan_segments(int kind, const int32_t* cu_seqlens_host, int batch, int s
   a.per_query_units = kind == 0 ? 1 : 0;
   a.P = num_ranges;
   a.tile = kind == 0 ? ModeCfg<MODE_MLA>::kTile : (kind == 1 ? ModeCfg<MODE_GQLA>::kTile : ModeCfg<MODE_GLA>::kTile);
+  const bool lockstep = lockstep_groups(a);
+  const SchedArgs ar = request_space(a);
   int n = 0;
   for (int p = 0; p < num_ranges; ++p) {
-    SegCursor c = locate_range_host(a, p);
+    SegCursor c = locate_range_host(ar, lockstep ? p / groups : p);
     Segment sg;
-    while (c.next(a, sg)) {
+    while (c.next(ar, sg)) {
+      if (lockstep) {
+        sg.k = p % groups;
+        sg.unit_id = sg.b * groups + sg.k;
+      }
       if (n < max_out) {
         int32_t* r = out + 8 * n;
         r[0] = p;

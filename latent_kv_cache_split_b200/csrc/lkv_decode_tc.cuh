@@ -192,14 +192,28 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int n_sm_warps = 2 * n_row_warps;     // softmax warps: two column halves per quadrant
   const int n_sm_threads = n_sm_warps * 32;
 
-  SchedArgs sa;
-  sa.cu = p.cu;
-  sa.B = p.B;
-  sa.s_q = p.s_q;
-  sa.tile = TN;
-  sa.units_per_req = kPair ? p.s_q : p.G;
-  sa.per_query_units = kPair ? 1 : 0;
-  sa.P = p.P;
+  SchedArgs sa0;
+  sa0.cu = p.cu;
+  sa0.B = p.B;
+  sa0.s_q = p.s_q;
+  sa0.tile = TN;
+  sa0.units_per_req = kPair ? p.s_q : p.G;
+  sa0.per_query_units = kPair ? 1 : 0;
+  sa0.P = p.P;
+  // grouped units in lockstep (lkv_sched.cuh): the cursor walks request space, and this range
+  // serves group kfix of block range / G
+  const bool lockstep = lockstep_groups(sa0);
+  const SchedArgs sa = request_space(sa0);
+  const int sched_range = lockstep ? range / p.G : range;
+  const int kfix = lockstep ? range % p.G : 0;
+  auto next_seg = [&](SegCursor& c, Segment& sg) -> bool {
+    const bool r = c.next(sa, sg);
+    if (r && lockstep) {
+      sg.k = kfix;
+      sg.unit_id = sg.b * p.G + kfix;
+    }
+    return r;
+  };
 
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
@@ -232,7 +246,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   if (warp == 0) {
     bool malformed = false;
-    SegCursor c = locate_range(sa, range, &malformed);
+    SegCursor c = locate_range(sa, sched_range, &malformed);
     if (lane == 0) {
       // a request shorter than s_q gets no tiles (its outputs are left unwritten): report it
       if (malformed && range == 0 && rank == 0) record_error(p.err, LKV_SITE_BAD_LENGTH);
@@ -284,7 +298,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (pvalid && pt + 1 < psg.tile_hi) {
           ++pt;
         } else {
-          pvalid = pcur.next(sa, psg);
+          pvalid = next_seg(pcur, psg);
           if (!pvalid) return;
           pt = psg.tile_lo;
         }
@@ -311,7 +325,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (pvalid && pt + 1 < psg.tile_hi) {
           ++pt;
         } else {
-          pvalid = pcur.next(sa, psg);
+          pvalid = next_seg(pcur, psg);
           if (pvalid) pt = psg.tile_lo;
         }
       }
@@ -319,7 +333,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       Segment sg;
       int n = 0, nv = 0;   // K (or whole) tiles and V tiles issued (a CTA's tile count fits an int)
       bool ok = true;
-      while (ok && cur.next(sa, sg)) {
+      while (ok && next_seg(cur, sg)) {
         for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
           if (pvalid) prefetch_next();
           const int st = static_cast<int>(n % KS);
@@ -390,7 +404,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (warp == 1) {
         const uint32_t id_qk = idesc_bf16(128, TN, 0, 0);
         const uint64_t qrope_desc = kPair ? sdesc_sw64(qrope_base, 512) : sdesc_sw128(qrope_base, 16, 1024);
-        while (ok && cur.next(sa, sg)) {
+        while (ok && next_seg(cur, sg)) {
           for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
             const int st = static_cast<int>(n % KS);
             if (!mbar_wait(smem_u32(&sm.full[st]), static_cast<uint32_t>((n / KS) & 1), wc, LKV_WAIT(W_FULL)) ||
@@ -420,7 +434,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       } else {
         const uint32_t id_pv = idesc_bf16(128, DV, 0, 1);
-        while (ok && cur.next(sa, sg)) {
+        while (ok && next_seg(cur, sg)) {
           for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
             const int pb = static_cast<int>(n & 1);
             const bool first = (t == sg.tile_lo);
@@ -470,7 +484,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     Segment sg;
     int m = 0;
     bool ok = true;
-    while (ok && cur.next(sa, sg)) {
+    while (ok && next_seg(cur, sg)) {
       for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++m) {
         if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.x_staged), static_cast<uint32_t>(m & 1), wc,
                                                 LKV_WAIT(W_XSTAGED)))) {
@@ -800,7 +814,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
     SegCursor cur = cur0;
     Segment sgA, nx;
-    bool haveA = cur.next(sa, sgA);
+    bool haveA = next_seg(cur, sgA);
     int tA = haveA ? sgA.tile_lo : 0;
     int nA = 0;
     // MLA: tile whose own half has been sent and whose peer half is awaited
@@ -841,7 +855,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         bool have_nx = false;
         if (last) {
           // QK of this tile is done, so the query operands are free: stage the next unit's
-          have_nx = cur.next(sa, nx);
+          have_nx = next_seg(cur, nx);
           if (have_nx) load_q(nx);
         }
         if constexpr (kPair) {

@@ -9,6 +9,13 @@
 // segment that covers its unit entirely writes the final output; the first or last segment
 // of a range may cover only part of a unit and then writes an fp32 partial (slot 0 = first
 // segment of the range, slot 1 = last), merged afterwards by the combine kernel.
+//
+// Lockstep variant for grouped units (G >= 4 groups per request, P a multiple of G): the
+// requests' tiles (one unit per request, every group of a request has the same tiles) are cut
+// into P / G equal blocks, and range p walks block p / G for group p % G.  The G ranges of a
+// block then stream the same requests at the same pace, so the key rows they share (the RoPE
+// key) are fetched from HBM once and served to the other groups from L2.  (With 2 groups the
+// shared key is a tenth of the traffic, and measured no faster in lockstep.)
 #pragma once
 #include <cstdint>
 
@@ -57,6 +64,19 @@ struct Segment {
   int slot;             // partial slot (0 first segment of the range, 1 last); -1 if complete
   int unit_id;          // b * units_per_req + k
 };
+
+// Request-space arguments of the lockstep variant (see above), or `a` itself.
+__host__ __device__ __forceinline__ bool lockstep_groups(const SchedArgs& a) {
+  return !a.per_query_units && a.units_per_req >= 4 && a.P % a.units_per_req == 0;
+}
+__host__ __device__ __forceinline__ SchedArgs request_space(const SchedArgs& a) {
+  SchedArgs r = a;
+  if (lockstep_groups(a)) {
+    r.units_per_req = 1;
+    r.P = a.P / a.units_per_req;
+  }
+  return r;
+}
 
 // Cursor over the segments of one range.  Every role of a CTA runs its own copy from the
 // same start state, so all roles see the same sequence.

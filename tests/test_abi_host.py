@@ -48,9 +48,10 @@ def test_version_and_status_strings(lkv):
     (0, 128, 1, 1, 74),     # varlen MLA: one range per CTA pair
     (0, 128, 2, 1, 74),
     (0, 8, 1, 1, 74),       # long context: split across every pair
-    (1, 64, 2, 8, 148),     # GQLA 512 units
-    (2, 8, 1, 2, 148),      # GLA-2 long context
-    (1, 8, 1, 8, 148),
+    (1, 64, 2, 8, 144),     # GQLA 512 units: 8 groups in lockstep x 18 blocks
+    (2, 8, 1, 2, 148),      # GLA-2 long context: one range per SM (no lockstep for 2 groups)
+    (1, 8, 1, 8, 144),
+    (1, 1, 1, 8, 144),      # one request: every block is a slice of it
 ])
 def test_plan_ranges(lkv, kind, B, s_q, G, want):
     assert lkv.plan_ranges(kind, B, s_q, G, 148) == want
@@ -67,7 +68,7 @@ def test_workspace_sizes(lkv):
     P = 64
     assert mla >= 2 * P * 128 * 512 * 4 + 2 * P * 128 * 4 + 2 * P * 4
     g = lkv.group_decode_workspace_size(1, 64, 2, 128, 8, 128, 148)
-    assert g >= 2 * 148 * 32 * 128 * 4
+    assert g >= 2 * 144 * 32 * 128 * 4
     assert lkv.group_decode_workspace_size(3, 1, 1, 128, 8, 128, 148) == 0
     assert lkv.group_decode_workspace_size(1, 1, 1, 128, 7, 128, 148) == 0
 
@@ -109,7 +110,7 @@ def _check_partition(segs, cu, kind, s_q, G, P):
 
 
 @pytest.mark.parametrize("kind,s_q,G,P", [(0, 1, 1, 74), (0, 2, 1, 74), (1, 2, 8, 148), (2, 1, 2, 148),
-                                         (0, 1, 1, 3), (1, 1, 4, 5)])
+                                         (0, 1, 1, 3), (1, 1, 4, 5), (1, 2, 8, 144), (1, 1, 4, 8)])
 def test_partition_covers_every_tile_once(lkv, kind, s_q, G, P):
     rng = np.random.default_rng(kind * 10 + s_q + P)
     for trial in range(4):
@@ -118,6 +119,24 @@ def test_partition_covers_every_tile_once(lkv, kind, s_q, G, P):
         cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
         segs = lkv.plan_segments(kind, cu, s_q, G, P)
         _check_partition(segs, cu.tolist(), kind, s_q, G, P)
+
+
+def test_lockstep_ranges_share_requests(lkv):
+    """With P a multiple of G, the G ranges of a block walk the same requests and tiles, one
+    group each (the RoPE key rows they share are then read at the same time)."""
+    rng = np.random.default_rng(7)
+    lengths = rng.integers(2, 5000, size=23)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    G, P = 8, 144
+    segs = lkv.plan_segments(1, cu, 2, G, P)
+    _check_partition(segs, cu.tolist(), 1, 2, G, P)
+    by_range = {}
+    for (p, b, k, lo, hi, complete, slot, uid) in segs:
+        assert k == p % G
+        by_range.setdefault(p, []).append((b, lo, hi))
+    for j in range(P // G):
+        walks = [by_range.get(j * G + k, []) for k in range(G)]
+        assert all(w == walks[0] for w in walks)
 
 
 def test_partition_uniform_lengths_never_split(lkv):
