@@ -49,9 +49,8 @@ constexpr int kTcThreads = 384;
 // MLA pair message per tile: 128 rows x 64 fp16 of exp2(partial score - partial tile max)
 // (values in (0, 1], so fp16 keeps 11 significant bits where bf16 would keep 8), then the 128
 // partial tile maxima (fp32).
-// One score message: 128 rows x 64 fp16 factors, then the partial tile maxima of both column
-// halves of each row.
-constexpr int kMsgBytes = 128 * 128 + 2 * 128 * 4;
+// One score message: 128 rows x 64 fp16 factors, then the 128 partial row maxima (fp32).
+constexpr int kMsgBytes = 128 * 128 + 128 * 4;
 // Incoming score messages in flight per CTA of the MLA pair.  A CTA sends message m only after
 // it has read the peer's message m-1, which the peer sent after reading message m-2 (and so
 // m-3) from this CTA, so with 3 slots the slot of message m is always free when it is written.
@@ -141,7 +140,9 @@ struct __align__(16) TcSmem {
   uint64_t s_full, s_free, o_free, q_ready, drain;
   uint64_t p_full[2], o_done[2], x_full[kMsgSlots];
   uint64_t x_staged, x_stage_free;  // MLA: outgoing message staged by the softmax / read by the sender
-  uint64_t x_consumed;              // MLA: incoming message read by the softmax
+  uint64_t x_consumed[2];           // MLA: incoming message of that parity read by the combine warps
+  uint64_t own_read;                // MLA: the combine warps have read the staged message
+  int n_armed;                      // MLA: incoming messages armed so far (for the abort drain)
   uint64_t xbar[4][2];              // per lane quadrant: both column halves posted a value
   float xch[2][2][128];             // [buffer][column half][row] values swapped between the halves
   uint32_t tmem_base;
@@ -227,18 +228,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     mbar_init(smem_u32(&sm.s_full), 1);
     // softmax-side barriers take one arrival per warp (lane 0, after a __syncwarp)
-    mbar_init(smem_u32(&sm.s_free), n_sm_warps);
-    mbar_init(smem_u32(&sm.o_free), n_sm_warps);
-    mbar_init(smem_u32(&sm.q_ready), n_sm_warps);
+    // MLA: 4 score warps (S, Q, staging) and 4 combine warps (P, O); grouped: the softmax warps
+    const int n_a = kPair ? 4 : n_sm_warps, n_b = kPair ? 4 : n_sm_warps;
+    mbar_init(smem_u32(&sm.s_free), n_a);
+    mbar_init(smem_u32(&sm.o_free), n_b);
+    mbar_init(smem_u32(&sm.q_ready), n_a);
     mbar_init(smem_u32(&sm.drain), 2);  // one commit from each UMMA issuer
     for (int b = 0; b < kMsgSlots; ++b) mbar_init(smem_u32(&sm.x_full[b]), 1);  // armed here, filled by the peer
-    mbar_init(smem_u32(&sm.x_staged), n_sm_warps);
+    mbar_init(smem_u32(&sm.x_staged), n_a);
     mbar_init(smem_u32(&sm.x_stage_free), 1);
-    mbar_init(smem_u32(&sm.x_consumed), n_sm_warps);
+    for (int b = 0; b < 2; ++b) mbar_init(smem_u32(&sm.x_consumed[b]), n_b);
+    mbar_init(smem_u32(&sm.own_read), n_b);
+    sm.n_armed = 0;
     for (int q = 0; q < 4; ++q)
       for (int b = 0; b < 2; ++b) mbar_init(smem_u32(&sm.xbar[q][b]), 2);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(smem_u32(&sm.p_full[b]), n_sm_warps);
+      mbar_init(smem_u32(&sm.p_full[b]), n_b);
       mbar_init(smem_u32(&sm.o_done[b]), 1);
     }
     sm.abort = 0;
@@ -491,36 +496,325 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           ok = false;
           break;
         }
-        // Two batches of kChunks 16-byte chunks: chunk lane + 32 i (a warp reads 512 contiguous
-        // bytes per load), then the second half of the message.
-        constexpr int kChunks = kMsgBytes / 16 / 64;
-        static_assert(kChunks * 64 * 16 == kMsgBytes, "message chunking");
+        // Two batches of 16-byte chunks: chunk lane + 32 i (a warp reads 512 contiguous bytes
+        // per load), kC1 of them, then the remaining kC2.
+        constexpr int kPer = kMsgBytes / 16 / 32;
+        static_assert(kPer * 32 * 16 == kMsgBytes, "message chunking");
+        constexpr int kC1 = (kPer + 1) / 2, kC2 = kPer - kC1;
         const uint4* src = reinterpret_cast<const uint4*>(sbuf);
-        uint4 v[kChunks];
+        uint4 v[kC1];
 #pragma unroll
-        for (int i = 0; i < kChunks; ++i) v[i] = src[h + 32 * i];
+        for (int i = 0; i < kC1; ++i) v[i] = src[h + 32 * i];
         // the peer's slot for message m is free once this CTA has read the peer's message m-1.
-        // Releasing the staging copy only after this wait keeps the softmax from reading
-        // message m (which it does after staging m+1) before the wait: x_consumed then never
-        // runs two phases ahead of the parity tested here.
-        if (m >= 1 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.x_consumed), static_cast<uint32_t>((m - 1) & 1),
-                                                          wc, LKV_WAIT(W_XSTAGED)))) {
+        // The staging copy is released only after this wait, and the combine warps read the
+        // peer's message m+1 only after message m+1 was staged: so barrier x_consumed[(m-1) & 1]
+        // never runs a phase ahead of the parity tested here.
+        if (m >= 1 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.x_consumed[(m - 1) & 1]),
+                                                          static_cast<uint32_t>(((m - 1) >> 1) & 1), wc,
+                                                          LKV_WAIT(W_XSTAGED)))) {
           ok = false;
           break;
         }
         const int xb = static_cast<int>(m % kMsgSlots);
 #pragma unroll
-        for (int i = 0; i < kChunks; ++i) st_async_v4(rrem[xb] + 16u * static_cast<uint32_t>(h + 32 * i), v[i], xrem[xb]);
+        for (int i = 0; i < kC1; ++i) st_async_v4(rrem[xb] + 16u * static_cast<uint32_t>(h + 32 * i), v[i], xrem[xb]);
 #pragma unroll
-        for (int i = 0; i < kChunks; ++i) v[i] = src[h + 32 * (kChunks + i)];
+        for (int i = 0; i < kC2; ++i) v[i] = src[h + 32 * (kC1 + i)];
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sm.x_stage_free));
 #pragma unroll
-        for (int i = 0; i < kChunks; ++i)
-          st_async_v4(rrem[xb] + 16u * static_cast<uint32_t>(h + 32 * (kChunks + i)), v[i], xrem[xb]);
+        for (int i = 0; i < kC2; ++i)
+          st_async_v4(rrem[xb] + 16u * static_cast<uint32_t>(h + 32 * (kC1 + i)), v[i], xrem[xb]);
       }
     }
-  } else if (warp >= 4 && warp < 12 && ((warp - 4) & 3) < n_row_warps) {
+  } else if (kPair && warp >= 4 && warp < 12) {
+    // ============================================================ MLA softmax
+    // Warps 4-7 (score warps) turn S into this CTA's factors E and stage them for the peer;
+    // warps 8-11 (combine warps) form P from both CTAs' factors, publish it, rescale O and run
+    // the epilogue.  The two run on different tiles at the same time (the score warps one tile
+    // ahead), each warp owns TMEM lane quadrant q = warp % 4 and all 64 key columns.
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;            // row (head) == TMEM lane
+    const uint32_t lb = static_cast<uint32_t>(q4 * 32);
+    const int col_base = 256 * static_cast<int>(rank);
+    auto wait_all = [&](uint32_t bar, uint32_t par, int site) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, par, wc, site)) != 0;
+    };
+    auto wait_all_cl = [&](uint32_t bar, uint32_t par, int site) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait<true>(bar, par, wc, site)) != 0;
+    };
+    auto warp_arrive = [&](uint32_t bar) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+    };
+    SegCursor cur = cur0;
+    Segment sg, nx;
+    bool ok = true;
+    int n = 0;
+    if (warp < 8) {
+      // ---------------------------------------------------------- score warps
+      auto load_q = [&](const Segment& s) {
+        const size_t qrow = (static_cast<size_t>(s.b) * p.s_q + s.k) * p.h_q + r;
+#pragma unroll 1
+        for (int bx = 0; bx < 4; ++bx) {
+          uint32_t w[32];
+          const uint4* src = reinterpret_cast<const uint4*>(p.q_nope + qrow * p.dq + col_base + 64 * bx);
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            const uint4 x = __ldg(src + v);
+            w[4 * v] = x.x;
+            w[4 * v + 1] = x.y;
+            w[4 * v + 2] = x.z;
+            w[4 * v + 3] = x.w;
+          }
+          tmem_st32(tm_addr(tbase, lb, Q0 + bx * 32), w);
+        }
+        // this CTA's 32-column RoPE half, 64-byte swizzle: chunk c of row r at c ^ ((r / 2) % 4)
+        const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + qrow * 64 + 32 * rank);
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(qrope_smem + r * 64 + ((c ^ ((r >> 1) & 3)) << 4)) = __ldg(src + c);
+        fence_proxy_async_smem();
+        tmem_wait_st();
+        tc_fence_before();
+        warp_arrive(smem_u32(&sm.q_ready));
+      };
+      bool have = next_seg(cur, sg);
+      if (have) load_q(sg);
+      while (ok && have) {
+        for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
+          if (!wait_all(smem_u32(&sm.s_full), static_cast<uint32_t>(n & 1), LKV_WAIT(W_SFULL))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          float cs[TN];
+#pragma unroll
+          for (int c = 0; c < TN; c += 32) {
+            uint32_t a[32];
+            tmem_ld32(tm_addr(tbase, lb, S0 + c), a);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) cs[c + j] = __uint_as_float(a[j]);
+          }
+          tmem_wait_ld();
+          tc_fence_before();
+          warp_arrive(smem_u32(&sm.s_free));
+          if (t == sg.tile_hi - 1 && (have = next_seg(cur, nx))) load_q(nx);  // QK(n) is done: Q is free
+          const int xb = n % kMsgSlots;
+          if (r == 0) {
+            mbar_arrive_expect_tx(smem_u32(&sm.x_full[xb]), kMsgBytes);  // the peer's message n
+            sm.n_armed = n + 1;
+          }
+          const int key0 = t * TN, lim = sg.keys;
+          if (key0 + TN > lim) {
+#pragma unroll
+            for (int c = 0; c < TN; ++c) cs[c] = (key0 + c < lim) ? cs[c] : -INFINITY;
+          }
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+          for (int c = 0; c < TN; ++c) m4[c & 3] = fmaxf(m4[c & 3], cs[c]);
+          const float tcur = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.sl2;  // log2 units
+          const float tsub = (tcur == -INFINITY) ? 0.f : tcur;
+          uint32_t e[TN / 2];
+#pragma unroll
+          for (int c = 0; c < TN / 2; ++c)
+            e[c] = ex2_f16x2(fmaf(cs[2 * c], p.sl2, -tsub), fmaf(cs[2 * c + 1], p.sl2, -tsub));
+          // the staging copy holds message n-1 until the sender and the combine warps read it
+          if (n >= 1 &&
+              (!wait_all(smem_u32(&sm.x_stage_free), static_cast<uint32_t>((n - 1) & 1), LKV_WAIT(W_XFREE)) ||
+               !wait_all(smem_u32(&sm.own_read), static_cast<uint32_t>((n - 1) & 1), LKV_WAIT(W_XFREE)))) {
+            ok = false;
+            break;
+          }
+          // row r: 8 chunks of 16 bytes, XOR-swizzled by r so that readers avoid bank conflicts
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(sbuf + r * 128 + ((c ^ (r & 7)) << 4)) =
+                make_uint4(e[4 * c], e[4 * c + 1], e[4 * c + 2], e[4 * c + 3]);
+          reinterpret_cast<float*>(sbuf + 128 * 128)[r] = tcur;
+          warp_arrive(smem_u32(&sm.x_staged));
+        }
+        if (!ok) break;
+        if (have) sg = nx;
+      }
+    } else {
+      // ---------------------------------------------------------- combine warps
+      float m_run = -INFINITY, l_run = 0.f;
+      int nconsumed = 0;
+      while (ok && next_seg(cur, sg)) {
+        for (int t = sg.tile_lo; t < sg.tile_hi && ok; ++t, ++n) {
+          const bool first = (t == sg.tile_lo), last = (t == sg.tile_hi - 1);
+          if (!wait_all(smem_u32(&sm.x_staged), static_cast<uint32_t>(n & 1), LKV_WAIT(W_XSTAGED))) {
+            ok = false;
+            break;
+          }
+          uint32_t eo[32], ep[32];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 x = *reinterpret_cast<const uint4*>(sbuf + r * 128 + ((c ^ (r & 7)) << 4));
+            eo[4 * c] = x.x;
+            eo[4 * c + 1] = x.y;
+            eo[4 * c + 2] = x.z;
+            eo[4 * c + 3] = x.w;
+          }
+          const float t_o = reinterpret_cast<const float*>(sbuf + 128 * 128)[r];
+          warp_arrive(smem_u32(&sm.own_read));
+          const int xb = n % kMsgSlots;
+          if (!wait_all_cl(smem_u32(&sm.x_full[xb]), static_cast<uint32_t>((n / kMsgSlots) & 1), LKV_WAIT(W_XFULL))) {
+            ok = false;
+            break;
+          }
+          const uint8_t* msg = rbuf + xb * kMsgBytes;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint4 x = *reinterpret_cast<const uint4*>(msg + r * 128 + ((c ^ (r & 7)) << 4));
+            ep[4 * c] = x.x;
+            ep[4 * c + 1] = x.y;
+            ep[4 * c + 2] = x.z;
+            ep[4 * c + 3] = x.w;
+          }
+          const float t_p = reinterpret_cast<const float*>(msg + 128 * 128)[r];
+          ++nconsumed;
+          warp_arrive(smem_u32(&sm.x_consumed[n & 1]));
+          // P = E_own * E_peer * 2^(t_own + t_peer - m): t_own + t_peer bounds the row's scores in
+          // this tile; products of two floats commute, so both CTAs get the same P
+          if (first) {
+            m_run = -INFINITY;
+            l_run = 0.f;
+          }
+          const float T = t_o + t_p;  // -inf when every key of this tile is masked for the row
+          bool rescale = false;
+          float m_new = m_run;
+          if (T > m_run + 8.f) {  // lazy rescale: keep the running max unless it grows by 2^8
+            m_new = T;
+            rescale = (m_run != -INFINITY);
+          }
+          const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.f;
+          // f <= 2^8; products below the fp16 range only drop terms under 2^-24 of the max
+          const float f = (T == -INFINITY) ? 0.f : ex2_approx(T - m_new);
+          const uint32_t f2 = pack_f16x2(f, f);
+          float s4[4] = {0.f, 0.f, 0.f, 0.f};
+          uint32_t pw[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const uint32_t pr = mul_f16x2(mul_f16x2(eo[c], ep[c]), f2);
+            const float e0 = f16_lo(pr), e1 = f16_hi(pr);
+            s4[c & 3] += e0 + e1;
+            pw[c] = pack_bf16x2(e0, e1);
+          }
+          l_run = l_run * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+          m_run = m_new;
+          const int pb = n & 1;
+          // P buffer pb was last read by PV(n-2)
+          if (n >= 2 &&
+              !wait_all(smem_u32(&sm.o_done[pb]), static_cast<uint32_t>(((n - 2) >> 1) & 1), LKV_WAIT(W_ODONE))) {
+            ok = false;
+            break;
+          }
+          if (__any_sync(0xffffffffu, rescale ? 1 : 0) && !first) {
+            // O holds this segment's tiles up to n-1: wait for PV(n-1), then scale in place
+            if (!wait_all(smem_u32(&sm.o_done[pb ^ 1]), static_cast<uint32_t>(((n - 1) >> 1) & 1),
+                          LKV_WAIT(W_ODONE))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll 1
+            for (int c = 0; c < DV; c += 32) {
+              uint32_t o[32];
+              tmem_ld32(tm_addr(tbase, lb, c), o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+              tmem_st32(tm_addr(tbase, lb, c), o);
+            }
+          }
+          tc_fence_after();
+          tmem_st32(tm_addr(tbase, lb, P0 + Cfg::kPCols * pb), pw);
+          const int key0 = t * TN;
+          if (key0 + TN > sg.keys) {
+            // Rows past the unit's last key belong to another request or to unwritten cache:
+            // their P is 0, but 0 * NaN would still poison O, so clear those V rows first.
+            const int firstbad = sg.keys - key0;
+            const int per_box = (TN - firstbad) * 8;  // 16-byte chunks per V box
+            uint8_t* vb = dsm + (n % KS) * kStageBytes;
+            for (int idx = r; idx < per_box * Cfg::kNV; idx += 128) {
+              const int bx = idx / per_box, rem = idx % per_box;
+              *reinterpret_cast<uint4*>(vb + bx * kBoxBytes + (firstbad + rem / 8) * 128 + (rem % 8) * 16) =
+                  make_uint4(0u, 0u, 0u, 0u);
+            }
+            fence_proxy_async_smem();
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          warp_arrive(smem_u32(&sm.p_full[pb]));
+          if (!last) continue;
+          // ---------------------------------------------------------- segment epilogue
+          if (!wait_all(smem_u32(&sm.o_done[pb]), static_cast<uint32_t>((n >> 1) & 1), LKV_WAIT(W_ODONE))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+          const float lse_v = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+          const size_t orow = (static_cast<size_t>(sg.b) * p.s_q + sg.k) * p.h_q + r;
+          if (sg.complete) {
+            __nv_bfloat16* dst = p.out + orow * p.dv_total + col_base;
+#pragma unroll 1
+            for (int c = 0; c < DV; c += 32) {
+              uint32_t o[32];
+              tmem_ld32(tm_addr(tbase, lb, c), o);
+              tmem_wait_ld();
+              uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                uint4 w;
+                w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
+                w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
+                w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
+                w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
+                d4[v] = w;
+              }
+            }
+            if (rank == 0) p.lse[orow] = lse_v;
+          } else {
+            const size_t prow = static_cast<size_t>(2 * range + sg.slot) * p.rmax + r;
+            float* dst = p.part_o + prow * p.dv_total + col_base;
+#pragma unroll 1
+            for (int c = 0; c < DV; c += 32) {
+              uint32_t o[32];
+              tmem_ld32(tm_addr(tbase, lb, c), o);
+              tmem_wait_ld();
+              float4* d4 = reinterpret_cast<float4*>(dst + c);
+#pragma unroll
+              for (int v = 0; v < 8; ++v)
+                d4[v] = make_float4(__uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
+                                    __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
+            }
+            if (rank == 0) p.part_lse[prow] = lse_v;
+            if (r == 0 && rank == 0) p.seg_info[2 * range + sg.slot] = sg.unit_id;
+          }
+          tc_fence_before();
+          warp_arrive(smem_u32(&sm.o_free));
+        }
+      }
+      if (!ok && r == 0) {
+        // After giving up, the peer may still write messages into this CTA's shared memory: it
+        // sends message m once it has read this CTA's message m-1, so at most up to message
+        // n_armed (messages armed here bound those staged).  Let them land (bounded) before the
+        // CTA can exit; every message is armed once.
+        uint32_t zero = 0;
+        const WaitCtl dc{&zero, p.err, p.wait_limit_ns};
+        const int armed = *reinterpret_cast<volatile int*>(&sm.n_armed);
+        for (int m = nconsumed; m <= armed && m < nconsumed + kMsgSlots; ++m) {
+          if (m >= armed) mbar_arrive_expect_tx(smem_u32(&sm.x_full[m % kMsgSlots]), kMsgBytes);
+          mbar_wait<true>(smem_u32(&sm.x_full[m % kMsgSlots]), static_cast<uint32_t>((m / kMsgSlots) & 1), dc,
+                          LKV_WAIT(W_DRAIN));
+        }
+      }
+    }
+  } else if (!kPair && warp >= 4 && warp < 12 && ((warp - 4) & 3) < n_row_warps) {
+   if constexpr (!kPair) {
     // ============================================================ softmax / epilogue
     const int q4 = (warp - 4) & 3;             // TMEM lane quadrant
     const int hf = (warp - 4) >> 2;            // key-column half of the tile
@@ -967,6 +1261,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                         LKV_WAIT(W_DRAIN));
       }
     }
+   }
   }
 
   // ---------------------------------------------------------------- teardown
