@@ -1,33 +1,34 @@
 // Tensor-core (tcgen05 / TMEM) split-KV decode attention for sm_100a.
 //
 // One persistent CTA (MLA: one CTA pair, a thread-block cluster of 2) per work range
-// (lkv_sched.cuh).  Per CTA, 8 warps:
+// (lkv_sched.cuh), 12 warps:
 //   warp 0      TMA producer: streams key/value tiles of the cache (64 keys for MLA / GLA,
-//               128 for GQLA) into a ring of shared-memory stages (2-D boxes of tile rows x
-//               64 bf16, 128-byte swizzle).
-//   warp 1      TMEM owner and UMMA issuer (one thread): S = Q K^T into TMEM, then
-//               O += P V into TMEM.  The non-RoPE part of Q and P are A operands read from
-//               TMEM; the RoPE part of Q is an A operand in shared memory; K and V are B
-//               operands in the stage (V is read MN-major from the very same swizzled tile
-//               that served as K where K = V).
-//   warps 4..7  softmax / epilogue: thread r owns row r (TMEM lane r): stages the unit's
-//               query, reads S, masks, runs the online softmax in the exp2 domain, writes P
-//               (bf16) into TMEM, rescales O when the running max moves, and at the end of a
-//               segment writes out / lse (or fp32 partials).
+//               128 for GQLA) into rings of shared-memory stages (2-D boxes of tile rows x
+//               64 bf16, 128-byte swizzle; the MLA RoPE halves 32 bf16 wide, 64-byte swizzle).
+//   warp 1      TMEM owner and QK issuer (one thread): S = Q K^T into TMEM.  The non-RoPE part
+//               of Q is an A operand in TMEM, the RoPE part one in shared memory; K is the B
+//               operand in the stage.
+//   warp 2      PV issuer (one thread): O += P V into TMEM, P an A operand in TMEM, V read
+//               MN-major from the very same swizzled tile that served as K where K = V.
+//   warp 3      MLA only: sender of the score messages to the peer CTA (st.async).
+//   warps 4-11  softmax / epilogue.  Grouped modes: warp 4 + q + 4h owns TMEM lane quadrant q
+//               and key-column half h of each tile; the two halves of a row agree on the
+//               running max through a bounded shared-memory exchange.  MLA: warps 4-7 (score
+//               warps) turn S into exp2 factors and stage them, warps 8-11 (combine warps) form
+//               P, rescale O and write the output, one tile behind the score warps.
 //
 // TMEM columns: O [0, DV) | S [DV, DV+T) | P0, P1 [DV+T, DV+2T) | Q [DV+2T, ...) for T keys/tile.
 // P is double buffered so the softmax of tile n+1 never waits for the PV of tile n.
 //
 // MLA absorbed path (h_q = 128 heads share the latent, GQLA explainer section 2): the
 // 128 x 512 fp32 output accumulator alone fills a whole TMEM, so a CTA pair splits it:
-// rank 0 owns value columns 0..255 and computes the partial scores over latent columns
-// 0..255 plus the 64 RoPE columns; rank 1 owns value columns 256..511 and the partial
-// scores over latent columns 256..511.  The two partial score tiles are exchanged through
-// distributed shared memory and summed (in the same order on both CTAs, so both derive the
-// same P), and each CTA accumulates its own half of O.  Each CTA streams only the cache
-// columns it needs, so the pair reads every cache byte once.  The softmax runs one tile
-// behind the score stream: tile n's partial scores are sent before tile n-1 is finished,
-// which hides the exchange latency.
+// rank 0 owns value columns 0..255 and contracts latent columns 0..255 plus RoPE columns 0..31,
+// rank 1 owns value columns 256..511 and contracts latent 256..511 plus RoPE 32..63.  Each CTA
+// turns its partial scores into fp16 factors E = exp2(partial - t) (t its partial row max) and
+// sends them to the peer through distributed shared memory; both CTAs form
+// P = E_own * E_peer * 2^(t_own + t_peer - m) (the same P on both sides) and accumulate their
+// own half of O.  Each CTA streams only the cache columns it needs, so the pair reads every
+// cache byte once.
 //
 // GQLA (g groups of expanded K_j, V_j) and GLA (latent groups, K_j = V_j) run one unit per
 // CTA: rows = heads of the group x new tokens (<= 128), padded to the M = 128 UMMA shape.
@@ -822,7 +823,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t lb = static_cast<uint32_t>(q4 * 32);
     const bool row_ok = r < p.R;
     const int sidx = hf * n_row_warps * 32 + r;  // 0 .. n_sm_threads-1
-    const int col_base = kPair ? 256 * static_cast<int>(rank) : 0;
     constexpr int HC = TN / 2;                 // key columns of this thread per tile
     constexpr int HW = HC / 2;                 // packed fp16 / bf16 pairs
     const int c0 = hf * HC;
@@ -853,13 +853,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     };
     // (query token, head) of this row in a unit
     auto row_map = [&](const Segment& sg, int& i, int& h) {
-      if (kPair) {
-        i = sg.k;
-        h = r;
-      } else {
-        i = r / p.hpg;
-        h = sg.k * p.hpg + (r % p.hpg);
-      }
+      i = r / p.hpg;
+      h = sg.k * p.hpg + (r % p.hpg);
     };
     // Stage the unit's query: non-RoPE part into TMEM (A operand; each half writes every
     // other 64-column box), RoPE part (half 0) into the swizzled shared-memory A operand.
@@ -871,7 +866,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int bx = hf; bx < Cfg::kNope; bx += 2) {
         uint32_t w[32];
         if (row_ok) {
-          const uint4* src = reinterpret_cast<const uint4*>(p.q_nope + qrow * p.dq + col_base + 64 * bx);
+          const uint4* src = reinterpret_cast<const uint4*>(p.q_nope + qrow * p.dq + 64 * bx);
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
             const uint4 x = __ldg(src + v);
@@ -887,21 +882,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tmem_st32(tm_addr(tbase, lb, Q0 + bx * 32), w);
       }
       if (hf == 0) {
-        if (kPair) {
-          // this CTA's 32-column RoPE half, 64-byte swizzle: chunk c of row r at c ^ ((r / 2) % 4)
-          const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + qrow * 64 + 32 * rank);
+        const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + qrow * 64);
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint4 x = row_ok ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4*>(qrope_smem + r * 64 + ((c ^ ((r >> 1) & 3)) << 4)) = x;
-          }
-        } else {
-          const uint4* src = reinterpret_cast<const uint4*>(p.q_rope + qrow * 64);
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 x = row_ok ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
-            *reinterpret_cast<uint4*>(qrope_smem + r * 128 + ((c ^ (r & 7)) << 4)) = x;
-          }
+        for (int c = 0; c < 8; ++c) {
+          const uint4 x = row_ok ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(qrope_smem + r * 128 + ((c ^ (r & 7)) << 4)) = x;
         }
         fence_proxy_async_smem();
       }
@@ -952,36 +937,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       for (int c = 0; c < HW; ++c) {
         const uint32_t h = ex2_f16x2(fmaf(s[2 * c], p.sl2, -msub), fmaf(s[2 * c + 1], p.sl2, -msub));
         const float e0 = f16_lo(h), e1 = f16_hi(h);
-        s4[c & 3] += e0 + e1;
-        pw[c] = pack_bf16x2(e0, e1);
-      }
-      l_run = l_run * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
-      m_run = m_new;
-      return true;
-    };
-    // MLA pair: P = E_own * E_peer * 2^(t_own + t_peer - M) where E = exp2(partial - t) (fp16) of
-    // each CTA's half of the contraction and t its partial max over this column half of the
-    // tile (t_own + t_peer bounds the full scores there).  Products of two floats commute, so
-    // both CTAs get the same P.
-    auto combine_tile = [&](const uint32_t (&eo)[HW], const uint32_t (&ep)[HW], float t_o, float t_p,
-                            const Segment& sg, int t, uint32_t (&pw)[HW], bool& rescale, float& alpha) -> bool {
-      if (t == sg.tile_lo) {
-        m_run = -INFINITY;
-        l_run = 0.f;
-      }
-      const float T = t_o + t_p;  // -inf when every key of this half is masked for the row
-      float To;
-      if (!pair_xchg(T, To)) return false;
-      const float m_new = new_max(fmaxf(T, To), rescale, alpha);
-      // f = 2^(T - m_new) <= 2^8; products below the fp16 range only drop terms that are
-      // under 2^-24 of the running max
-      const float f = (T == -INFINITY) ? 0.f : ex2_approx(T - m_new);
-      const uint32_t f2 = pack_f16x2(f, f);
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c = 0; c < HW; ++c) {
-        const uint32_t pr = mul_f16x2(mul_f16x2(eo[c], ep[c]), f2);
-        const float e0 = f16_lo(pr), e1 = f16_hi(pr);
         s4[c & 3] += e0 + e1;
         pw[c] = pack_bf16x2(e0, e1);
       }
@@ -1062,7 +1017,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const float lse_v = l_tot > 0.f ? (m_run + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
       const size_t orow = (static_cast<size_t>(sg.b) * p.s_q + qi) * p.h_q + qh;
       if (sg.complete) {
-        __nv_bfloat16* dst = p.out + orow * p.dv_total + col_base;
+        __nv_bfloat16* dst = p.out + orow * p.dv_total;
 #pragma unroll 1
         for (int c = hf * (DV / 2); c < (hf + 1) * (DV / 2); c += 32) {
           uint32_t o[32];
@@ -1084,7 +1039,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (row_ok && rank == 0 && hf == 0) p.lse[orow] = lse_v;
       } else {
         const size_t prow = static_cast<size_t>(2 * range + sg.slot) * p.rmax + r;
-        float* dst = p.part_o + prow * p.dv_total + col_base;
+        float* dst = p.part_o + prow * p.dv_total;
 #pragma unroll 1
         for (int c = hf * (DV / 2); c < (hf + 1) * (DV / 2); c += 32) {
           uint32_t o[32];
@@ -1111,24 +1066,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bool haveA = next_seg(cur, sgA);
     int tA = haveA ? sgA.tile_lo : 0;
     int nA = 0;
-    // MLA: tile whose own half has been sent and whose peer half is awaited
-    uint32_t eprev[HW];
-    float tprev = -INFINITY;
-    Segment sgB;
-    int tB = 0;
-    int nB = 0;
-    bool haveB = false;
-    int nconsumed = 0, nsent = 0;  // MLA messages read from / sent to the peer
     bool ok = true;
     if (haveA) load_q(sgA);
-    while (ok && (haveA || haveB)) {
+    while (ok && haveA) {
       float cs[HC];
       bool gotA = false;
       Segment sgAc;
       int tAc = 0;
       int nAc = 0;
-      uint32_t ecur[HW];
-      float tcur = -INFINITY;
       if (haveA) {
         if (!wait_all(smem_u32(&sm.s_full), static_cast<uint32_t>(nA & 1), LKV_WAIT(W_SFULL))) {
           ok = false;
@@ -1152,38 +1097,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           have_nx = next_seg(cur, nx);
           if (have_nx) load_q(nx);
         }
-        if constexpr (kPair) {
-          // own half: mask, partial max over this column half, E = exp2(partial - max) in fp16
-          const int xb = static_cast<int>(nA % kMsgSlots);
-          if (r == 0 && hf == 0) mbar_arrive_expect_tx(smem_u32(&sm.x_full[xb]), kMsgBytes);  // the peer's half of nA
-          const int lim = sgA.keys, key0 = tA * TN + c0;
-          if (key0 + HC > lim) {
-#pragma unroll
-            for (int c = 0; c < HC; ++c) cs[c] = (key0 + c < lim) ? cs[c] : -INFINITY;
-          }
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-          for (int c = 0; c < HC; ++c) m4[c & 3] = fmaxf(m4[c & 3], cs[c]);
-          tcur = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.sl2;  // log2 units
-          const float tsub = (tcur == -INFINITY) ? 0.f : tcur;
-#pragma unroll
-          for (int c = 0; c < HW; ++c)
-            ecur[c] = ex2_f16x2(fmaf(cs[2 * c], p.sl2, -tsub), fmaf(cs[2 * c + 1], p.sl2, -tsub));
-          // stage the message for the sender warps (they read message nA-1 out of it first);
-          // row r is 8 chunks of 16 bytes (this half's 4), XOR-swizzled by r so that the
-          // reader's loads avoid bank conflicts
-          if (nA >= 1 && !wait_all(smem_u32(&sm.x_stage_free), static_cast<uint32_t>((nA - 1) & 1), LKV_WAIT(W_XFREE))) {
-            ok = false;
-            break;
-          }
-#pragma unroll
-          for (int c = 0; c < HW / 4; ++c)
-            *reinterpret_cast<uint4*>(sbuf + r * 128 + (((4 * hf + c) ^ (r & 7)) << 4)) =
-                make_uint4(ecur[4 * c], ecur[4 * c + 1], ecur[4 * c + 2], ecur[4 * c + 3]);
-          reinterpret_cast<float*>(sbuf + 128 * 128)[hf * 128 + r] = tcur;
-          warp_arrive(smem_u32(&sm.x_staged));
-          ++nsent;
-        }
         gotA = true;
         sgAc = sgA;
         tAc = tA;
@@ -1198,45 +1111,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       }
-      if constexpr (kPair) {
-        if (haveB) {
-          const int xb = static_cast<int>(nB % kMsgSlots);
-          if (!wait_all_cl(smem_u32(&sm.x_full[xb]), static_cast<uint32_t>((nB / kMsgSlots) & 1), LKV_WAIT(W_XFULL))) {
-            ok = false;
-            break;
-          }
-          const uint8_t* msg = rbuf + xb * kMsgBytes;
-          uint32_t ep[HW];
-#pragma unroll
-          for (int c = 0; c < HW / 4; ++c) {
-            const uint4 x = *reinterpret_cast<const uint4*>(msg + r * 128 + (((4 * hf + c) ^ (r & 7)) << 4));
-            ep[4 * c] = x.x;
-            ep[4 * c + 1] = x.y;
-            ep[4 * c + 2] = x.z;
-            ep[4 * c + 3] = x.w;
-          }
-          const float tpeer = reinterpret_cast<const float*>(msg + 128 * 128)[hf * 128 + r];
-          ++nconsumed;
-          warp_arrive(smem_u32(&sm.x_consumed));
-          uint32_t pw[HW];
-          bool rescale;
-          float alpha;
-          if (!combine_tile(eprev, ep, tprev, tpeer, sgB, tB, pw, rescale, alpha) ||
-              !finish_tile(pw, rescale, alpha, sgB, tB, nB)) {
-            ok = false;
-            break;
-          }
-        }
-        haveB = gotA;
-        if (gotA) {
-#pragma unroll
-          for (int c = 0; c < HW; ++c) eprev[c] = ecur[c];
-          tprev = tcur;
-          sgB = sgAc;
-          tB = tAc;
-          nB = nAc;
-        }
-      } else if (gotA) {
+      if (gotA) {
         int qi, qh;
         row_map(sgAc, qi, qh);
         uint32_t pw[HW];
@@ -1246,19 +1121,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           ok = false;
           break;
         }
-      }
-    }
-    if (kPair && !ok && r == 0 && hf == 0) {
-      // After giving up, the peer may still write messages into this CTA's shared memory: it
-      // sends message m once it has read this CTA's message m-1, so at most up to message
-      // nsent (messages staged here bound those sent).  Let them land (bounded) before the
-      // CTA can exit; every message is armed once.
-      uint32_t zero = 0;
-      const WaitCtl dc{&zero, p.err, p.wait_limit_ns};
-      for (int m = nconsumed; m < nsent + 1; ++m) {
-        if (m >= nA) mbar_arrive_expect_tx(smem_u32(&sm.x_full[m % kMsgSlots]), kMsgBytes);
-        mbar_wait<true>(smem_u32(&sm.x_full[m % kMsgSlots]), static_cast<uint32_t>((m / kMsgSlots) & 1), dc,
-                        LKV_WAIT(W_DRAIN));
       }
     }
    }
