@@ -606,10 +606,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_arrive_expect_tx(smem_u32(&sm.x_full[xb]), kMsgBytes);  // the peer's message n
             sm.n_armed = n + 1;
           }
-          const int key0 = t * TN, lim = sg.keys;
-          if (key0 + TN > lim) {
+          const int rem = sg.keys - t * TN;  // valid keys in this tile
+          if (rem < TN) {
 #pragma unroll
-            for (int c = 0; c < TN; ++c) cs[c] = (key0 + c < lim) ? cs[c] : -INFINITY;
+            for (int c = 0; c < TN; ++c) cs[c] = (c < rem) ? cs[c] : -INFINITY;
           }
           float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
@@ -916,13 +916,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         m_run = -INFINITY;
         l_run = 0.f;
       }
-      const int lim = sg.L - p.s_q + qi + 1;  // keys visible to this row
-      const int key0 = t * TN + c0;
+      // keys of this half of the tile visible to this row
+      const int rem = (sg.L - p.s_q + qi + 1) - (t * TN + c0);
       // max of the raw scores (the scale is positive), then one FMA per score for the
       // exponent in log2 units
-      if (key0 + HC > lim) {
+      if (rem < HC) {
 #pragma unroll
-        for (int c = 0; c < HC; ++c) s[c] = (key0 + c < lim) ? s[c] : -INFINITY;
+        for (int c = 0; c < HC; ++c) s[c] = (c < rem) ? s[c] : -INFINITY;
       }
       float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
