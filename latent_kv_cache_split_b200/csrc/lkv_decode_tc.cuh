@@ -156,6 +156,60 @@ __device__ __forceinline__ uint32_t tm_addr(uint32_t base, uint32_t lane_base, u
   return base + (lane_base << 16) + col;
 }
 
+// Rarely executed per-row blocks of the softmax warps, kept out of line so that the per-tile loops
+// stay short in the instruction cache.  `trow` is the TMEM address of this thread's row at column
+// c0; every lane of the warp calls them together (tcgen05.ld / st are warp-collective).
+// O[row, c0 .. c0+ncols) *= alpha.
+__device__ __noinline__ void tmem_scale_row(uint32_t trow, int ncols, float alpha) {
+#pragma unroll 1
+  for (int c = 0; c < ncols; c += 32) {
+    uint32_t o[32];
+    tmem_ld32(trow + c, o);
+    tmem_wait_ld();
+#pragma unroll
+    for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+    tmem_st32(trow + c, o);
+  }
+  tmem_wait_st();
+}
+// dst[0 .. ncols) = bf16(O[row, c0 ..] * inv_l) (stores skipped for a padding row).
+__device__ __noinline__ void tmem_row_to_bf16(uint32_t trow, int ncols, float inv_l, __nv_bfloat16* dst, bool store) {
+#pragma unroll 1
+  for (int c = 0; c < ncols; c += 32) {
+    uint32_t o[32];
+    tmem_ld32(trow + c, o);
+    tmem_wait_ld();
+    if (store) {
+      uint4* d4 = reinterpret_cast<uint4*>(dst + c);
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        uint4 w;
+        w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
+        w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
+        w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
+        w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
+        d4[v] = w;
+      }
+    }
+  }
+}
+// dst[0 .. ncols) = O[row, c0 ..] * inv_l in fp32 (a split partial).
+__device__ __noinline__ void tmem_row_to_f32(uint32_t trow, int ncols, float inv_l, float* dst, bool store) {
+#pragma unroll 1
+  for (int c = 0; c < ncols; c += 32) {
+    uint32_t o[32];
+    tmem_ld32(trow + c, o);
+    tmem_wait_ld();
+    if (store) {
+      float4* d4 = reinterpret_cast<float4*>(dst + c);
+#pragma unroll
+      for (int v = 0; v < 8; ++v)
+        d4[v] = make_float4(__uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
+                            __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
+    }
+  }
+}
+
 template <int kMode>
 __global__ void __launch_bounds__(kTcThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap map_a,  // MLA ckv | GQLA k | GLA clat
@@ -720,15 +774,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
               break;
             }
             tc_fence_after();
-#pragma unroll 1
-            for (int c = 0; c < DV; c += 32) {
-              uint32_t o[32];
-              tmem_ld32(tm_addr(tbase, lb, c), o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-              tmem_st32(tm_addr(tbase, lb, c), o);
-            }
+            tmem_scale_row(tm_addr(tbase, lb, 0), DV, alpha);
           }
           tc_fence_after();
           tmem_st32(tm_addr(tbase, lb, P0 + Cfg::kPCols * pb), pw);
@@ -760,38 +806,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const float lse_v = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
           const size_t orow = (static_cast<size_t>(sg.b) * p.s_q + sg.k) * p.h_q + r;
           if (sg.complete) {
-            __nv_bfloat16* dst = p.out + orow * p.dv_total + col_base;
-#pragma unroll 1
-            for (int c = 0; c < DV; c += 32) {
-              uint32_t o[32];
-              tmem_ld32(tm_addr(tbase, lb, c), o);
-              tmem_wait_ld();
-              uint4* d4 = reinterpret_cast<uint4*>(dst + c);
-#pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                uint4 w;
-                w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
-                w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
-                w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
-                w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
-                d4[v] = w;
-              }
-            }
+            tmem_row_to_bf16(tm_addr(tbase, lb, 0), DV, inv_l, p.out + orow * p.dv_total + col_base, true);
             if (rank == 0) p.lse[orow] = lse_v;
           } else {
             const size_t prow = static_cast<size_t>(2 * range + sg.slot) * p.rmax + r;
-            float* dst = p.part_o + prow * p.dv_total + col_base;
-#pragma unroll 1
-            for (int c = 0; c < DV; c += 32) {
-              uint32_t o[32];
-              tmem_ld32(tm_addr(tbase, lb, c), o);
-              tmem_wait_ld();
-              float4* d4 = reinterpret_cast<float4*>(dst + c);
-#pragma unroll
-              for (int v = 0; v < 8; ++v)
-                d4[v] = make_float4(__uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
-                                    __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
-            }
+            tmem_row_to_f32(tm_addr(tbase, lb, 0), DV, inv_l, p.part_o + prow * p.dv_total + col_base, true);
             if (rank == 0) p.part_lse[prow] = lse_v;
             if (r == 0 && rank == 0) p.seg_info[2 * range + sg.slot] = sg.unit_id;
           }
@@ -961,15 +980,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (!wait_all(smem_u32(&sm.o_done[pb ^ 1]), static_cast<uint32_t>(((n - 1) >> 1) & 1), LKV_WAIT(W_ODONE)))
           return false;
         tc_fence_after();
-#pragma unroll 1
-        for (int c = hf * (DV / 2); c < (hf + 1) * (DV / 2); c += 32) {
-          uint32_t o[32];
-          tmem_ld32(tm_addr(tbase, lb, c), o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-          tmem_st32(tm_addr(tbase, lb, c), o);
-        }
+        tmem_scale_row(tm_addr(tbase, lb, hf * (DV / 2)), DV / 2, alpha);
       }
       tc_fence_after();
       {
@@ -1017,42 +1028,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const float lse_v = l_tot > 0.f ? (m_run + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
       const size_t orow = (static_cast<size_t>(sg.b) * p.s_q + qi) * p.h_q + qh;
       if (sg.complete) {
-        __nv_bfloat16* dst = p.out + orow * p.dv_total;
-#pragma unroll 1
-        for (int c = hf * (DV / 2); c < (hf + 1) * (DV / 2); c += 32) {
-          uint32_t o[32];
-          tmem_ld32(tm_addr(tbase, lb, c), o);
-          tmem_wait_ld();
-          if (row_ok) {
-            uint4* d4 = reinterpret_cast<uint4*>(dst + c);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l, __uint_as_float(o[8 * v + 1]) * inv_l);
-              w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l, __uint_as_float(o[8 * v + 3]) * inv_l);
-              w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l, __uint_as_float(o[8 * v + 5]) * inv_l);
-              w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l, __uint_as_float(o[8 * v + 7]) * inv_l);
-              d4[v] = w;
-            }
-          }
-        }
+        tmem_row_to_bf16(tm_addr(tbase, lb, hf * (DV / 2)), DV / 2, inv_l, p.out + orow * p.dv_total + hf * (DV / 2),
+                         row_ok);
         if (row_ok && rank == 0 && hf == 0) p.lse[orow] = lse_v;
       } else {
         const size_t prow = static_cast<size_t>(2 * range + sg.slot) * p.rmax + r;
-        float* dst = p.part_o + prow * p.dv_total;
-#pragma unroll 1
-        for (int c = hf * (DV / 2); c < (hf + 1) * (DV / 2); c += 32) {
-          uint32_t o[32];
-          tmem_ld32(tm_addr(tbase, lb, c), o);
-          tmem_wait_ld();
-          if (row_ok) {
-            float4* d4 = reinterpret_cast<float4*>(dst + c);
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              d4[v] = make_float4(__uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
-                                  __uint_as_float(o[4 * v + 2]) * inv_l, __uint_as_float(o[4 * v + 3]) * inv_l);
-          }
-        }
+        tmem_row_to_f32(tm_addr(tbase, lb, hf * (DV / 2)), DV / 2, inv_l, p.part_o + prow * p.dv_total + hf * (DV / 2),
+                        row_ok);
         if (row_ok && rank == 0 && hf == 0) p.part_lse[prow] = lse_v;
         if (r == 0 && rank == 0 && hf == 0) p.seg_info[2 * range + sg.slot] = sg.unit_id;
       }
