@@ -36,6 +36,9 @@ import synth  # noqa: E402
 
 METRIC = "decode attn tokens/s; KV-cache GB/s & TFLOPS as fraction of B200 roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Datasheet figures (HGX B200, dense bf16), reported beside the measured-peak fraction: the fraction
+# of the roofline time max(bytes / HBM, FLOPs / tensor) that the decode call achieves.
+NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 
 def kernel_source_hash() -> str:
@@ -339,6 +342,9 @@ def bench_gpu(args, rank, world, local_rank):
                          "unit": "GB/s" if bound == "hbm" else "TFLOP/s", "frac": achieved / peak,
                          "traffic": measured_traffic(w.name), "kernel_source_hash": kernel_source_hash(),
                          "peak_source": f"{how} (MEASURED_PEAKS.json burst)",
+                         "nominal": {"hbm_gbs": NOMINAL_PEAKS["hbm_gbs"], "bf16_tflops": NOMINAL_PEAKS["bf16_tflops"],
+                                     "frac": max(alg_bytes / (NOMINAL_PEAKS["hbm_gbs"] * 1e9),
+                                                 flops / (NOMINAL_PEAKS["bf16_tflops"] * 1e12)) / dec_s},
                          "roofline_ms": max(t_hbm, t_tc) * 1e3,
                          "frac_of_step_roofline": max(t_hbm, t_tc) * 1e3 / ms,
                          "kernel": "decode_tc_kernel + split combine (one lkv_*_decode call)",
