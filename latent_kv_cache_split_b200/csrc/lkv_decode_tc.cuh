@@ -52,6 +52,9 @@ constexpr int kTcThreads = 384;
 // partial tile maxima (fp32).
 // One score message: 128 rows x 64 fp16 factors, then the 128 partial row maxima (fp32).
 constexpr int kMsgBytes = 128 * 128 + 128 * 4;
+// Slot stride in shared memory: 1024-byte aligned, because the combine warps overwrite the
+// peer's factors in a slot with P (same 128-byte-swizzled rows), the A operand of that tile's PV.
+constexpr int kMsgStride = 17 * 1024;
 // Incoming score messages in flight per CTA of the MLA pair.  A CTA sends message m only after
 // it has read the peer's message m-1, which the peer sent after reading message m-2 (and so
 // m-3) from this CTA, so with 3 slots the slot of message m is always free when it is written.
@@ -119,7 +122,7 @@ struct ModeCfg {
   static constexpr int kQropeBytes = kPair ? 128 * 64 : 128 * 128;
   static constexpr int kRopeSteps = kPair ? 2 : 4;  // QK K-steps over the RoPE columns
   // MLA adds kMsgSlots incoming score messages and one outgoing staging copy
-  static constexpr size_t kSmemBytes = 1024 + kRingBytes + kQropeBytes + (kPair ? (kMsgSlots + 1) * kMsgBytes : 0);
+  static constexpr size_t kSmemBytes = 1024 + kRingBytes + kQropeBytes + (kPair ? (kMsgSlots + 1) * kMsgStride : 0);
 };
 static_assert(ModeCfg<MODE_MLA>::Q0 + 32 * ModeCfg<MODE_MLA>::kNope <= kTmemCols, "TMEM budget");
 static_assert(ModeCfg<MODE_GLA>::Q0 + 32 * ModeCfg<MODE_GLA>::kNope <= kTmemCols, "TMEM budget");
@@ -138,7 +141,9 @@ struct __align__(16) TcSmem {
   uint64_t empty[kStagesT];
   uint64_t vfull[kVStagesT];
   uint64_t vempty[kVStagesT];
-  uint64_t s_full, s_free, o_free, q_ready, drain;
+  uint64_t s_full[2], s_free[2];  // per S buffer (MLA double-buffers S; grouped modes use [0])
+  uint64_t o_free, q_ready, drain;
+  uint64_t pvd[kMsgSlots];         // MLA: PV of a tile done, by message slot (for the sender)
   uint64_t p_full[2], o_done[2], x_full[kMsgSlots];
   uint64_t x_staged, x_stage_free;  // MLA: outgoing message staged by the softmax / read by the sender
   uint64_t x_consumed[2];           // MLA: incoming message of that parity read by the combine warps
@@ -237,7 +242,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint8_t* qrope_smem = dsm + Cfg::kRingBytes;
   const uint32_t qrope_base = smem_u32(qrope_smem);
   uint8_t* rbuf = qrope_smem + Cfg::kQropeBytes;  // MLA only: kMsgSlots incoming messages
-  uint8_t* sbuf = rbuf + kMsgSlots * kMsgBytes;  // MLA only: the outgoing message being staged
+  uint8_t* sbuf = rbuf + kMsgSlots * kMsgStride;  // MLA only: the outgoing message being staged
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -281,11 +286,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(smem_u32(&sm.vfull[s]), 1);
       mbar_init(smem_u32(&sm.vempty[s]), 1);
     }
-    mbar_init(smem_u32(&sm.s_full), 1);
+    for (int b = 0; b < 2; ++b) mbar_init(smem_u32(&sm.s_full[b]), 1);
     // softmax-side barriers take one arrival per warp (lane 0, after a __syncwarp)
     // MLA: 4 score warps (S, Q, staging) and 4 combine warps (P, O); grouped: the softmax warps
     const int n_a = kPair ? 4 : n_sm_warps, n_b = kPair ? 4 : n_sm_warps;
-    mbar_init(smem_u32(&sm.s_free), n_a);
+    for (int b = 0; b < 2; ++b) mbar_init(smem_u32(&sm.s_free[b]), n_a);
+    for (int b = 0; b < kMsgSlots; ++b) mbar_init(smem_u32(&sm.pvd[b]), 1);
     mbar_init(smem_u32(&sm.o_free), n_b);
     mbar_init(smem_u32(&sm.q_ready), n_a);
     mbar_init(smem_u32(&sm.drain), 2);  // one commit from each UMMA issuer
@@ -467,8 +473,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         while (ok && next_seg(cur, sg)) {
           for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
             const int st = static_cast<int>(n % KS);
+            // MLA double-buffers S (buffer n % 2, last read for tile n-2); grouped modes have one
+            const int sb = kPair ? (n & 1) : 0;
+            const int prev = kPair ? n - 2 : n - 1;
+            const uint32_t prev_par = static_cast<uint32_t>((kPair ? (prev >> 1) : prev) & 1);
             if (!mbar_wait(smem_u32(&sm.full[st]), static_cast<uint32_t>((n / KS) & 1), wc, LKV_WAIT(W_FULL)) ||
-                (n > 0 && !mbar_wait(smem_u32(&sm.s_free), static_cast<uint32_t>((n - 1) & 1), wc, LKV_WAIT(W_SFREE))) ||
+                (prev >= 0 && !mbar_wait(smem_u32(&sm.s_free[sb]), prev_par, wc, LKV_WAIT(W_SFREE))) ||
                 (t == sg.tile_lo &&
                  !mbar_wait(smem_u32(&sm.q_ready), static_cast<uint32_t>(seg & 1), wc, LKV_WAIT(W_QREADY)))) {
               ok = false;
@@ -479,15 +489,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
             for (int ks = 0; ks < 4 * Cfg::kNope; ++ks) {
               const int bx = ks >> 2, kk = ks & 3;
-              umma_ts(tbase + S0, tbase + Q0 + bx * 32 + kk * 8, desc_add(kdesc, bx * kBoxBytes + kk * 32), id_qk,
-                      ks ? 1u : 0u);
+              umma_ts(tbase + S0 + TN * sb, tbase + Q0 + bx * 32 + kk * 8, desc_add(kdesc, bx * kBoxBytes + kk * 32),
+                      id_qk, ks ? 1u : 0u);
             }
             const uint32_t rope_addr = stage_base + st * kStageBytes + Cfg::kRopeBox * kBoxBytes;
             const uint64_t rdesc = kPair ? sdesc_sw64(rope_addr, 512) : sdesc_sw128(rope_addr, 16, 1024);
 #pragma unroll
             for (int kk = 0; kk < Cfg::kRopeSteps; ++kk)
-              umma_ss(tbase + S0, desc_add(qrope_desc, kk * 32), desc_add(rdesc, kk * 32), id_qk, 1u);
-            umma_commit(smem_u32(&sm.s_full));
+              umma_ss(tbase + S0 + TN * sb, desc_add(qrope_desc, kk * 32), desc_add(rdesc, kk * 32), id_qk, 1u);
+            umma_commit(smem_u32(&sm.s_full[sb]));
             if (kSplit) umma_commit(smem_u32(&sm.empty[st]));  // the K slot is free once QK is done
           }
           ++seg;
@@ -512,12 +522,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             const uint32_t vaddr = kSplit ? vring_base + static_cast<uint32_t>(n % VS) * Cfg::kVStageBytes
                                           : stage_base + static_cast<uint32_t>(n % KS) * kStageBytes;
             const uint64_t vdesc = sdesc_sw128(vaddr + Cfg::kVBox0 * kBoxBytes, kBoxBytes, 1024);
-            const uint32_t pa = tbase + P0 + Cfg::kPCols * pb;
+            if constexpr (kPair) {
+              // P(n) was written over the peer's factors in message slot n % 3 (K-major, 128-byte swizzle)
+              const uint64_t pdesc = sdesc_sw128(smem_u32(rbuf + (n % kMsgSlots) * kMsgStride), 16, 1024);
 #pragma unroll
-            for (int kk = 0; kk < TN / 16; ++kk)
-              umma_ts(tbase, pa + kk * 8, desc_add(vdesc, kk * 2048), id_pv, (first && kk == 0) ? 0u : 1u);
+              for (int kk = 0; kk < TN / 16; ++kk)
+                umma_ss(tbase, desc_add(pdesc, kk * 32), desc_add(vdesc, kk * 2048), id_pv, (first && kk == 0) ? 0u : 1u);
+            } else {
+              const uint32_t pa = tbase + P0 + Cfg::kPCols * pb;
+#pragma unroll
+              for (int kk = 0; kk < TN / 16; ++kk)
+                umma_ts(tbase, pa + kk * 8, desc_add(vdesc, kk * 2048), id_pv, (first && kk == 0) ? 0u : 1u);
+            }
             umma_commit(smem_u32(&sm.o_done[pb]));
             umma_commit(kSplit ? smem_u32(&sm.vempty[n % VS]) : smem_u32(&sm.empty[n % KS]));
+            if (kPair) umma_commit(smem_u32(&sm.pvd[n % kMsgSlots]));  // slot n % 3 readable again
           }
           ++seg;
         }
@@ -537,7 +556,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     uint32_t rrem[kMsgSlots], xrem[kMsgSlots];
 #pragma unroll
     for (int b = 0; b < kMsgSlots; ++b) {
-      rrem[b] = map_to_peer(smem_u32(rbuf + b * kMsgBytes), peer);
+      rrem[b] = map_to_peer(smem_u32(rbuf + b * kMsgStride), peer);
       xrem[b] = map_to_peer(smem_u32(&sm.x_full[b]), peer);
     }
     SegCursor cur = cur0;
@@ -571,6 +590,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         const int xb = static_cast<int>(m % kMsgSlots);
+        // The peer sends message m+1 into slot (m+1) % 3 after reading this message m; that slot
+        // holds this CTA's P(m-2) until PV(m-2) is done.  Message m therefore goes only after
+        // PV(m-2) (barrier pvd[(m-2) % 3]; its next phase needs PV(m+1), so no phase is skipped).
+        if (m >= 2 && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.pvd[(m - 2) % kMsgSlots]),
+                                                          static_cast<uint32_t>(((m - 2) / kMsgSlots) & 1), wc,
+                                                          LKV_WAIT(W_ODONE)))) {
+          ok = false;
+          break;
+        }
 #pragma unroll
         for (int i = 0; i < kC1; ++i) st_async_v4(rrem[xb] + 16u * static_cast<uint32_t>(h + 32 * i), v[i], xrem[xb]);
 #pragma unroll
@@ -638,7 +666,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (have) load_q(sg);
       while (ok && have) {
         for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
-          if (!wait_all(smem_u32(&sm.s_full), static_cast<uint32_t>(n & 1), LKV_WAIT(W_SFULL))) {
+          const int sb = n & 1;
+          if (!wait_all(smem_u32(&sm.s_full[sb]), static_cast<uint32_t>((n >> 1) & 1), LKV_WAIT(W_SFULL))) {
             ok = false;
             break;
           }
@@ -647,13 +676,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
           for (int c = 0; c < TN; c += 32) {
             uint32_t a[32];
-            tmem_ld32(tm_addr(tbase, lb, S0 + c), a);
+            tmem_ld32(tm_addr(tbase, lb, S0 + TN * sb + c), a);
 #pragma unroll
             for (int j = 0; j < 32; ++j) cs[c + j] = __uint_as_float(a[j]);
           }
           tmem_wait_ld();
           tc_fence_before();
-          warp_arrive(smem_u32(&sm.s_free));
+          warp_arrive(smem_u32(&sm.s_free[sb]));
           if (t == sg.tile_hi - 1 && (have = next_seg(cur, nx))) load_q(nx);  // QK(n) is done: Q is free
           const int xb = n % kMsgSlots;
           if (r == 0) {
@@ -719,7 +748,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ok = false;
             break;
           }
-          const uint8_t* msg = rbuf + xb * kMsgBytes;
+          uint8_t* msg = rbuf + xb * kMsgStride;
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const uint4 x = *reinterpret_cast<const uint4*>(msg + r * 128 + ((c ^ (r & 7)) << 4));
@@ -760,12 +789,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           l_run = l_run * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
           m_run = m_new;
           const int pb = n & 1;
-          // P buffer pb was last read by PV(n-2)
-          if (n >= 2 &&
-              !wait_all(smem_u32(&sm.o_done[pb]), static_cast<uint32_t>(((n - 2) >> 1) & 1), LKV_WAIT(W_ODONE))) {
-            ok = false;
-            break;
-          }
+          // P(n) replaces the peer's factors in slot xb: the same 128-byte swizzled rows are the
+          // K-major A operand of PV(n) (the sender keeps the peer off this slot until PV(n) is done)
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(msg + r * 128 + ((c ^ (r & 7)) << 4)) =
+                make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+          fence_proxy_async_smem();
           if (__any_sync(0xffffffffu, rescale ? 1 : 0) && !first) {
             // O holds this segment's tiles up to n-1: wait for PV(n-1), then scale in place
             if (!wait_all(smem_u32(&sm.o_done[pb ^ 1]), static_cast<uint32_t>(((n - 1) >> 1) & 1),
@@ -776,8 +806,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_after();
             tmem_scale_row(tm_addr(tbase, lb, 0), DV, alpha);
           }
-          tc_fence_after();
-          tmem_st32(tm_addr(tbase, lb, P0 + Cfg::kPCols * pb), pw);
           const int key0 = t * TN;
           if (key0 + TN > sg.keys) {
             // Rows past the unit's last key belong to another request or to unwritten cache:
@@ -1057,7 +1085,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       int tAc = 0;
       int nAc = 0;
       if (haveA) {
-        if (!wait_all(smem_u32(&sm.s_full), static_cast<uint32_t>(nA & 1), LKV_WAIT(W_SFULL))) {
+        if (!wait_all(smem_u32(&sm.s_full[0]), static_cast<uint32_t>(nA & 1), LKV_WAIT(W_SFULL))) {
           ok = false;
           break;
         }
@@ -1071,7 +1099,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tmem_wait_ld();
         tc_fence_before();
-        warp_arrive(smem_u32(&sm.s_free));
+        warp_arrive(smem_u32(&sm.s_free[0]));
         const bool last = (tA == sgA.tile_hi - 1);
         bool have_nx = false;
         if (last) {
