@@ -16,7 +16,6 @@ on a bounded sample of the same workload; under torchrun only rank 0 runs it.
 from __future__ import annotations
 
 import argparse
-import glob
 import hashlib
 import json
 import os
@@ -41,12 +40,16 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 
+# The sources the decode kernels and their launch are built from (the projections' translation unit
+# and the header's declarations do not change what a decode launch reads or writes).
+DECODE_SOURCES = ("lkv_api.cu", "lkv_aux.cuh", "lkv_decode_tc.cuh", "lkv_ptx.cuh", "lkv_sched.cuh", "lkv_tma_host.h")
+
+
 def kernel_source_hash() -> str:
-    """Hash of the CUDA sources and the C header: a traffic figure measured with ncu is only
+    """Hash of the decode kernels' CUDA sources: a traffic figure measured with ncu is only
     reported while the kernels it was measured on are unchanged."""
     h = hashlib.sha256()
-    files = sorted(glob.glob(os.path.join(ROOT, "latent_kv_cache_split_b200", "csrc", "*")))
-    files.append(os.path.join(ROOT, "include", "lkv.h"))
+    files = [os.path.join(ROOT, "latent_kv_cache_split_b200", "csrc", f) for f in DECODE_SOURCES]
     for f in files:
         h.update(os.path.basename(f).encode())
         with open(f, "rb") as fh:

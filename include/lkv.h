@@ -219,6 +219,32 @@ lkv_status lkv_check_device(int32_t* code_out, int clear);
  */
 lkv_status lkv_selftest_wait_timeout(uint64_t limit_ns, lkv_stream_t stream);
 
+/*
+ * Projections either side of the decode path (GQLA explainer, section 2 "Methodology": the
+ * absorbed path folds W_UK into the query and applies W_UV after attention; the GQA path expands
+ * the latent into per-group keys and values).  j(h) = h / (h_q / groups).  bf16 operands, fp32
+ * accumulation, bf16 results (dtype must be LKV_BF16, else LKV_ERR_UNSUPPORTED); all arrays are
+ * contiguous device arrays unless a row stride is given.  These are plain GEMMs run by cuBLAS,
+ * which the library opens (dlopen "libcublas.so.12") at the first projection call: LKV_ERR_UNSUPPORTED
+ * if it cannot be loaded.  The first call on a device creates that device's cuBLAS handle, which
+ * allocates cuBLAS's own workspace; later calls allocate nothing.  Asynchronous on `stream`.
+ *
+ * lkv_absorb_query:    q [n_tok, h_q, d_h], w_uk [groups, r, d_h] -> q_abs [n_tok, h_q, r],
+ *                      q_abs[t, h, :] = w_uk[j(h)] q[t, h, :]
+ * lkv_unabsorb_output: o_lat [n_tok, h_q, r], w_uv [groups, r, d_v] -> out [n_tok, h_q, d_v],
+ *                      out[t, h, :] = w_uv[j(h)]^T o_lat[t, h, :]
+ * lkv_expand_latent:   c [n_rows, r] (row stride c_row_stride elements >= r), w [groups, r, d]
+ *                      -> x [n_rows, groups, d],  x[t, j, :] = c[t, :] w[j]
+ * Errors: LKV_ERR_INVALID_ARG for NULL pointers, non-positive sizes, h_q % groups != 0 or
+ * leading dimensions beyond int range (checked before any launch); LKV_ERR_CUDA if cuBLAS fails.
+ */
+lkv_status lkv_absorb_query(const void* q, const void* w_uk, void* q_abs, int n_tok, int h_q, int groups,
+                            int d_h, int r, int dtype, lkv_stream_t stream);
+lkv_status lkv_unabsorb_output(const void* o_lat, const void* w_uv, void* out, int n_tok, int h_q,
+                               int groups, int r, int d_v, int dtype, lkv_stream_t stream);
+lkv_status lkv_expand_latent(const void* c, int64_t c_row_stride, const void* w, void* x, int64_t n_rows,
+                             int groups, int r, int d, int dtype, lkv_stream_t stream);
+
 /* Site codes stored in the device error word. */
 #define LKV_SITE_SELFTEST 1
 #define LKV_SITE_BAD_LENGTH 2     /* a request with L_b < s_q (append or decode)      */

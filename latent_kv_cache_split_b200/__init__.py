@@ -8,7 +8,8 @@ fallback: if liblkv.so is missing the import fails.
 Functions (same names as the C entry points without the ``lkv_`` prefix):
     mla_absorbed_decode, gqla_group_decode, gla_group_decode, latent_cache_append,
     merge_partials, check_device, selftest_wait_timeout, plan_ranges,
-    mla_decode_workspace_size, group_decode_workspace_size
+    mla_decode_workspace_size, group_decode_workspace_size,
+    absorb_query, unabsorb_output, expand_latent (the projections either side of the path)
 """
 from __future__ import annotations
 
@@ -59,12 +60,16 @@ _merge = _sig("lkv_merge_partials", _i32, _vp, _vp, _i32, _i64, _i32, _i32, _vp,
 _check = _sig("lkv_check_device", _i32, ctypes.POINTER(ctypes.c_int32), _i32)
 _selftest = _sig("lkv_selftest_wait_timeout", _i32, ctypes.c_uint64, _vp)
 _segments = _sig("lkv_plan_segments", _i32, _i32, _vp, _i32, _i32, _i32, _i32, _vp, _i32)
+_absorb = _sig("lkv_absorb_query", _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp)
+_unabsorb = _sig("lkv_unabsorb_output", _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp)
+_expand = _sig("lkv_expand_latent", _i32, _vp, _i64, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _vp)
 
 EXPORTED = ["lkv_version", "lkv_status_string", "lkv_plan_ranges", "lkv_mla_decode_workspace_size",
             "lkv_group_decode_workspace_size", "lkv_mla_absorbed_decode", "lkv_gqla_group_decode",
             "lkv_gla_group_decode", "lkv_latent_cache_append", "lkv_merge_partials",
             "lkv_check_device", "lkv_selftest_wait_timeout", "lkv_plan_segments",
-            "lkv_gqla_group_decode_noalloc"]
+            "lkv_gqla_group_decode_noalloc", "lkv_absorb_query", "lkv_unabsorb_output",
+            "lkv_expand_latent"]
 
 
 class LkvError(RuntimeError):
@@ -279,3 +284,50 @@ def check_device(clear: bool = True) -> int:
 
 def selftest_wait_timeout(limit_ns: int, stream=None):
     _ck(_selftest(int(limit_ns), _stream(stream)), "lkv_selftest_wait_timeout")
+
+
+def absorb_query(q, w_uk, out=None, stream=None):
+    """q_abs[..., h, :] = w_uk[j(h)] @ q[..., h, :].  q [..., h_q, d_h], w_uk [G, r, d_h] (bf16,
+    contiguous) -> [..., h_q, r] bf16."""
+    G, r, d_h = w_uk.shape
+    h_q = q.shape[-2]
+    if q.shape[-1] != d_h:
+        raise ValueError("q and w_uk disagree on d_h")
+    n_tok = q.numel() // (h_q * d_h)
+    if out is None:
+        out = torch.empty(q.shape[:-1] + (r,), dtype=q.dtype, device=q.device)
+    _contig(q, w_uk, out)
+    _ck(_absorb(_ptr(q), _ptr(w_uk), _ptr(out), n_tok, h_q, G, d_h, r, _dtype_code(q), _stream(stream)),
+        "lkv_absorb_query")
+    return out
+
+
+def unabsorb_output(o_lat, w_uv, out=None, stream=None):
+    """out[..., h, :] = w_uv[j(h)]^T @ o_lat[..., h, :].  o_lat [..., h_q, r], w_uv [G, r, d_v]
+    (bf16, contiguous) -> [..., h_q, d_v] bf16."""
+    G, r, d_v = w_uv.shape
+    h_q = o_lat.shape[-2]
+    if o_lat.shape[-1] != r:
+        raise ValueError("o_lat and w_uv disagree on r")
+    n_tok = o_lat.numel() // (h_q * r)
+    if out is None:
+        out = torch.empty(o_lat.shape[:-1] + (d_v,), dtype=o_lat.dtype, device=o_lat.device)
+    _contig(o_lat, w_uv, out)
+    _ck(_unabsorb(_ptr(o_lat), _ptr(w_uv), _ptr(out), n_tok, h_q, G, r, d_v, _dtype_code(o_lat), _stream(stream)),
+        "lkv_unabsorb_output")
+    return out
+
+
+def expand_latent(c, w, out=None, stream=None):
+    """x[t, j, :] = c[t, :] @ w[j].  c [T, r] (unit inner stride; may be a column slice of the
+    cache), w [G, r, d] contiguous (bf16) -> x [T, G, d] bf16."""
+    G, r, d = w.shape
+    T = c.shape[0]
+    if c.shape[1] != r:
+        raise ValueError("c and w disagree on r")
+    if out is None:
+        out = torch.empty((T, G, d), dtype=c.dtype, device=c.device)
+    _contig(w, out)
+    _ck(_expand(_ptr(c), _row_stride(c), _ptr(w), _ptr(out), T, G, r, d, _dtype_code(c), _stream(stream)),
+        "lkv_expand_latent")
+    return out

@@ -2,8 +2,10 @@
 
     python latent_kv_cache_split_b200/build.py [--verbose]
 
-The library is a single translation unit (csrc/lkv_api.cu includes the kernel headers)
-linked against the static CUDA runtime, so the .so only needs the NVIDIA driver at run time.
+The library is two translation units: csrc/lkv_api.cu (the decode path; it includes the kernel
+headers) and csrc/lkv_proj.cu (the projections, which open cuBLAS at run time).  Both link the
+static CUDA runtime, so the .so only needs the NVIDIA driver at run time (and cuBLAS for the
+projections).
 """
 from __future__ import annotations
 
@@ -16,7 +18,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "liblkv.so")
-SOURCES = ["lkv_api.cu"]
+SOURCES = ["lkv_api.cu", "lkv_proj.cu"]
 HEADERS = ["lkv_ptx.cuh", "lkv_sched.cuh", "lkv_decode_tc.cuh", "lkv_aux.cuh", "lkv_tma_host.h"]
 
 NVCC_FLAGS = [

@@ -201,3 +201,19 @@ def test_validation_errors_need_no_gpu(lkv):
     assert L._merge(P16, P16, 0, 4, 8, 0, P16, P16, None) == L.ERR_INVALID_ARG
     assert L._merge(P16, P16, 2, 4, 6, 0, P16, P16, None) == L.ERR_INVALID_ARG
     assert L._selftest(0, None) == L.ERR_INVALID_ARG
+
+
+def test_projection_argument_errors_need_no_gpu(lkv):
+    """The projection entry points reject bad arguments before any CUDA or cuBLAS call."""
+    P = _fake(1 << 20)
+    st = ctypes.c_void_p(0)
+    assert lkv._absorb(None, P, P, 4, 8, 4, 8, 16, 0, st) == lkv.ERR_INVALID_ARG
+    assert lkv._absorb(P, P, P, 4, 6, 4, 8, 16, 0, st) == lkv.ERR_INVALID_ARG      # 6 heads, 4 groups
+    assert lkv._absorb(P, P, P, 0, 8, 4, 8, 16, 0, st) == lkv.ERR_INVALID_ARG
+    assert lkv._absorb(P, P, P, 4, 8, 4, 8, 16, 1, st) == lkv.ERR_UNSUPPORTED      # fp32
+    assert lkv._unabsorb(P, P, None, 4, 8, 4, 16, 8, 0, st) == lkv.ERR_INVALID_ARG
+    assert lkv._unabsorb(P, P, P, 4, 8, 3, 16, 8, 0, st) == lkv.ERR_INVALID_ARG
+    assert lkv._unabsorb(P, P, P, 4, 8, 4, 16, 8, 1, st) == lkv.ERR_UNSUPPORTED
+    assert lkv._expand(P, 8, P, P, 4, 2, 16, 8, 0, st) == lkv.ERR_INVALID_ARG      # row stride < r
+    assert lkv._expand(P, 16, P, P, 0, 2, 16, 8, 0, st) == lkv.ERR_INVALID_ARG
+    assert lkv._expand(P, 16, P, P, 4, 2, 16, 8, 1, st) == lkv.ERR_UNSUPPORTED

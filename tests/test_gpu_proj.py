@@ -1,0 +1,144 @@
+"""GPU tests for the projections either side of the decode path (GQLA explainer, section 2
+"Methodology": W_UK folded into the query and W_UV applied after attention on the absorbed path,
+the latent expanded into per-group keys and values on the GQA path), against the fp64 oracle on
+the same bf16 inputs, and the same-weights agreement of the two decode forms with every step on
+the GPU."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+# bf16 results of fp32-accumulated products of bf16 inputs: the output rounding alone gives a
+# relative error of up to 2^-9 per element
+GATE = dict(rel_l2=5e-3, max_rel=1e-2)
+
+
+@pytest.fixture(scope="module")
+def L(gpu):
+    import latent_kv_cache_split_b200 as lib
+    lib.check_device(clear=True)
+    return lib
+
+
+def _bf(a, dev):
+    return torch.from_numpy(np.asarray(a, dtype=np.float32)).bfloat16().to(dev)
+
+
+def _f64(t):
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def _check(got, ref):
+    got = _f64(got)
+    rel = np.linalg.norm(got - ref) / np.linalg.norm(ref)
+    max_rel = np.abs(got - ref).max() / np.abs(ref).max()
+    assert rel <= GATE["rel_l2"] and max_rel <= GATE["max_rel"], (rel, max_rel)
+
+
+@pytest.mark.parametrize("n_tok,h_q,G,d_h,r", [(64, 128, 1, 128, 512), (128, 128, 8, 128, 512), (5, 32, 4, 64, 96)])
+def test_absorb_query(L, gpu, n_tok, h_q, G, d_h, r):
+    rng = np.random.default_rng(n_tok + G)
+    q = _bf(rng.standard_normal((n_tok, h_q, d_h)), gpu)
+    w = _bf(rng.standard_normal((G, r, d_h)) / math.sqrt(d_h), gpu)
+    _check(L.absorb_query(q, w), oracle.absorb_query(_f64(q), _f64(w), G))
+
+
+@pytest.mark.parametrize("n_tok,h_q,G,r,d_v", [(64, 128, 1, 512, 128), (128, 128, 8, 512, 128), (7, 16, 2, 64, 32)])
+def test_unabsorb_output(L, gpu, n_tok, h_q, G, r, d_v):
+    rng = np.random.default_rng(n_tok + 3 * G)
+    o = _bf(rng.standard_normal((n_tok, h_q, r)), gpu)
+    w = _bf(rng.standard_normal((G, r, d_v)) / math.sqrt(r), gpu)
+    _check(L.unabsorb_output(o, w), oracle.unabsorb_output(_f64(o), _f64(w), G))
+
+
+@pytest.mark.parametrize("T,G,r,d", [(300, 8, 512, 128), (1, 2, 256, 64), (4099, 8, 512, 128)])
+def test_expand_latent_from_interleaved_cache(L, gpu, T, G, r, d):
+    """The latent is a column slice of the interleaved [T, r + 64] cache (row stride r + 64)."""
+    rng = np.random.default_rng(T + G)
+    cache = _bf(rng.standard_normal((T, r + 64)), gpu)
+    w = _bf(rng.standard_normal((G, r, d)) / math.sqrt(r), gpu)
+    c = cache[:, :r]
+    _check(L.expand_latent(c, w), oracle.expand_latent(_f64(c), _f64(w)))
+
+
+def test_projection_argument_errors(L, gpu):
+    q = torch.zeros((4, 6, 8), dtype=torch.bfloat16, device=gpu)
+    w = torch.zeros((4, 16, 8), dtype=torch.bfloat16, device=gpu)
+    with pytest.raises(L.LkvError) as e:
+        L.absorb_query(q, w)  # 6 heads do not split into 4 groups
+    assert e.value.status == L.ERR_INVALID_ARG
+    q8 = torch.zeros((4, 8, 8), dtype=torch.float32, device=gpu)
+    with pytest.raises(L.LkvError) as e:
+        L.absorb_query(q8, w.float())  # fp32 operands: only bf16 is implemented
+    assert e.value.status == L.ERR_UNSUPPORTED
+
+
+def test_same_weights_agreement_all_on_gpu(L, gpu):
+    """GQLA explainer, section 2: absorbed path (q -> W_UK q on the GPU, MLA decode over the latent,
+    W_UV^T o_lat on the GPU) against the GQA path (K_j = C W_UK[j], V_j = C W_UV[j] expanded on the
+    GPU, GQLA decode).  Exact in real arithmetic; bf16 rounding of the intermediate tensors bounds
+    the difference (gate rel-L2 <= 2e-2, as for the oracle-projected diagnostic)."""
+    rng = np.random.default_rng(78)
+    B, H, G, dh, r, dr, Lk = 3, 128, 8, 128, 512, 64, 700
+    cu = synth.prefix_offsets([Lk, Lk - 40, 129])
+    T = int(cu[-1])
+    cache = _bf(np.concatenate([rng.standard_normal((T, r)) / math.sqrt(r), rng.standard_normal((T, dr)) / 8], 1), gpu)
+    C, kr = cache[:, :r], cache[:, r:]
+    w_uk = _bf(rng.standard_normal((G, r, dh)) / math.sqrt(r) * 2, gpu)
+    w_uv = _bf(rng.standard_normal((G, r, dh)) / math.sqrt(r), gpu)
+    q = _bf(rng.standard_normal((B, 1, H, dh)) / math.sqrt(dh) * 4, gpu)
+    qr = _bf(rng.standard_normal((B, 1, H, dr)) / 8, gpu)
+    scale = 1 / math.sqrt(dh + dr)
+    cu_d = torch.from_numpy(cu.astype(np.int32)).to(gpu)
+    q_abs = L.absorb_query(q, w_uk)
+    o_lat, lse_a = L.mla_absorbed_decode(q_abs, qr, C, kr, cu_d, scale)
+    out_a = L.unabsorb_output(o_lat, w_uv)
+    K = L.expand_latent(C, w_uk)
+    V = L.expand_latent(C, w_uv)
+    out_g, lse_g = L.gqla_group_decode(q, qr, K, V, kr.contiguous(), cu_d, scale)
+    a, g = _f64(out_a), _f64(out_g)
+    rel = np.linalg.norm(a - g) / np.linalg.norm(g)
+    assert rel < 2e-2, rel
+    assert np.abs(lse_a.cpu().numpy() - lse_g.cpu().numpy()).max() < 2e-2
+    # and each side matches the fp64 oracle on its own GPU-produced bf16 operands
+    ref_a, _ = oracle.mla_absorbed_decode(_f64(q_abs), _f64(qr), _f64(C), _f64(kr), cu, scale)
+    rel_a = np.linalg.norm(_f64(o_lat) - ref_a) / np.linalg.norm(ref_a)
+    assert rel_a < 5e-3, rel_a
+
+
+def test_projection_throughput(L, gpu):
+    """Measurement (printed with -s): the projections of one decode step of the MLA B=64 workload
+    (absorb for 64 tokens x 128 heads, unabsorb) and the GQLA expansion of 4096 new cache rows,
+    as TFLOP/s of the plain GEMMs (bf16, fp32 accumulation)."""
+    rng = np.random.default_rng(5)
+    cases = []
+    q = _bf(rng.standard_normal((64, 128, 128)), gpu)
+    wk = _bf(rng.standard_normal((8, 512, 128)) / 11, gpu)
+    wk1 = wk[:1].contiguous()
+    cases.append(("absorb 64 tok x 128 heads, g=1", lambda: L.absorb_query(q, wk1), 2 * 64 * 128 * 128 * 512))
+    cases.append(("absorb 64 tok x 128 heads, g=8", lambda: L.absorb_query(q, wk), 2 * 64 * 128 * 128 * 512))
+    o = _bf(rng.standard_normal((64, 128, 512)), gpu)
+    wv = _bf(rng.standard_normal((8, 512, 128)) / 22, gpu)
+    wv1 = wv[:1].contiguous()
+    cases.append(("unabsorb 64 tok x 128 heads, g=1", lambda: L.unabsorb_output(o, wv1), 2 * 64 * 128 * 512 * 128))
+    cases.append(("unabsorb 64 tok x 128 heads, g=8", lambda: L.unabsorb_output(o, wv), 2 * 64 * 128 * 512 * 128))
+    c = _bf(rng.standard_normal((4096, 512)), gpu)
+    cases.append(("expand 4096 rows to g=8 x 128", lambda: L.expand_latent(c, wk), 2 * 4096 * 512 * 8 * 128))
+    for name, fn, flops in cases:
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(20):
+            fn()
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / 20
+        print(f"{name}: {ms * 1e3:.1f} us, {flops / ms / 1e9:.1f} TFLOP/s")
