@@ -7,10 +7,10 @@ pages (see attend.py for the citations) and pinned by brute force, closed forms
 and identities in tests/test_oracle_*.py.
 """
 from .attend import (grouped_decode, mla_absorbed_decode, gqla_group_decode, gla_group_decode,
-                     merge_partials, append_rows, append_destinations, visible_keys,
+                     gta_group_decode, merge_partials, append_rows, append_destinations, visible_keys,
                      absorb_query, unabsorb_output, expand_latent)
 from . import accounting
 
 __all__ = ["grouped_decode", "mla_absorbed_decode", "gqla_group_decode", "gla_group_decode",
-           "merge_partials", "append_rows", "append_destinations", "visible_keys",
+           "gta_group_decode", "merge_partials", "append_rows", "append_destinations", "visible_keys",
            "absorb_query", "unabsorb_output", "expand_latent", "accounting"]

@@ -6,6 +6,9 @@ query/output/lse element once; work on padding or split partials is not counted.
 * Cache bytes per token: the absorbed path stores the latent plus the shared
   RoPE key, r_kv + d_R elements; the GQA path stores 2*g*d_h + d_R -- GQLA
   explainer, section 2 ("MQA absorbed path" / "GQA path", cache lines).
+* GTA stores one tied key/value state per group plus the shared RoPE key,
+  g*d_h + d_R per token; the article on GTA/GLA puts the saving against GQA at
+  about half of the KV cache ("Grouped Latent Attention" article, section "GTA").
 * FLOPs: per visible (query row, key) pair, 2*(d_k + d_R) for q.k and 2*d_v
   for p.v, over h_q heads.
 * Arithmetic intensity = FLOPs / cache bytes per token; the page gives about
@@ -22,7 +25,7 @@ __all__ = ["cache_row_elems", "cache_bytes_per_token", "flops_per_token",
 
 def cache_row_elems(kind, groups, d_k, d_v, d_rope):
     """Elements stored per cached token: latent(s) + RoPE key, or expanded K and V + RoPE key."""
-    if kind in ("mla", "gla"):
+    if kind in ("mla", "gla", "gta"):
         return groups * d_k + d_rope
     if kind == "gqla":
         return groups * (d_k + d_v) + d_rope

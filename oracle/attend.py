@@ -29,6 +29,11 @@ Sources:
 * GLA: query heads are split into groups and each group shares its own latent
   -- "Grouped Latent Attention" article (Tri Dao et al. news page), section
   "GLA".  Instance: G = n_lat, K_j = V_j = latent group j, one shared RoPE key.
+* GTA (grouped-tied attention): the heads of a group share one tied key/value
+  state, so the group's cached state is read as its key and as its value --
+  same article, section "GTA".  Instance: G = g, K_j = V_j = tied state j (width
+  d_h), with the one shared RoPE key of the other forms (a reading: the article
+  does not say where RoPE goes).
 * MHA: G = h_q.
 
 Readings where the pages are silent (listed again in the design notes):
@@ -42,7 +47,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = ["grouped_decode", "mla_absorbed_decode", "gqla_group_decode", "gla_group_decode",
-           "merge_partials", "append_rows", "append_destinations", "visible_keys",
+           "gta_group_decode", "merge_partials", "append_rows", "append_destinations", "visible_keys",
            "absorb_query", "unabsorb_output", "expand_latent"]
 
 
@@ -128,6 +133,14 @@ def gla_group_decode(q, q_rope, clat, kpe, n_lat, cu_seqlens, scale, requests=No
     T = clat.shape[0]
     lat = clat.reshape(T, n_lat, -1)
     return grouped_decode(q, q_rope, lat, lat, kpe, cu_seqlens, scale, requests=requests)
+
+
+def gta_group_decode(q, q_rope, kv, kpe, g, cu_seqlens, scale, requests=None):
+    """GTA: g tied groups kv [T, g*d_h]; group j's heads read tied state j as both key and value,
+    plus the shared k_rope kpe [T, d_R].  Output out [B, s_q, h_q, d_h]."""
+    T = kv.shape[0]
+    tied = kv.reshape(T, g, -1)
+    return grouped_decode(q, q_rope, tied, tied, kpe, cu_seqlens, scale, requests=requests)
 
 
 def merge_partials(o_parts, lse_parts):

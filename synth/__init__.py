@@ -31,6 +31,7 @@ class Workload:
     kind    "mla"  -- all h_q heads share one latent (G = 1, K = V = latent).
             "gqla" -- G = g expanded key/value groups, separate K_j and V_j.
             "gla"  -- G = n_lat latent groups, K_j = V_j = latent group j.
+            "gta"  -- G = g tied groups, K_j = V_j = tied state j (same layout as "gla").
     d_k     width of the non-RoPE part of each key (r_kv, d_h or r_g).
     d_v     width of each value row (equals d_k for "mla" and "gla").
     seqlen  uniform per-request cache length, or None for log-uniform lengths
@@ -94,6 +95,12 @@ WORKLOADS = {
                          131072, 4, _std(576)),
     "long_gqla_g8": Workload("long_gqla_g8", "gqla", "bf16", 8, 1, 128, 8, 128, 128, 64,
                              131072, 4, _std(192)),
+    # GTA: the GQLA shapes (g=8, d_h=128, d_R=64, s_q=2, L=8192) with K and V tied per group.
+    "gta_g8_sq2_l8192": Workload("gta_g8_sq2_l8192", "gta", "bf16", 64, 2, 128, 8, 128, 128, 64,
+                                 8192, 5, _std(192)),
+    # GQA-2: two K/V groups of 64 heads each (the group size the VHA fold gives), s_q=2, L=8192.
+    "gqa2_sq2_l8192": Workload("gqa2_sq2_l8192", "gqla", "bf16", 64, 2, 128, 2, 128, 128, 64,
+                               8192, 6, _std(192)),
 }
 
 
@@ -149,7 +156,7 @@ def make_inputs(w: Workload, extra_rows: int = 0, lengths=None) -> dict:
       lengths     int64 numpy [B]
       cu_seqlens  int32 torch [B+1]
       q, q_rope   [B, s_q, h_q, d_k], [B, s_q, h_q, d_R]
-      mla / gla:  cache [T + extra_rows, G*d_k + d_R] with the latent in the
+      mla / gla / gta:  cache [T + extra_rows, G*d_k + d_R] with the latent (tied state) in the
                   first G*d_k columns and k_rope in the last d_R (one row per token)
       gqla:       k, v [T + extra_rows, g, d_h]; kpe [T + extra_rows, d_R]
     Rows past T (extra_rows) are zero; tests poison them to check masking.
@@ -172,7 +179,7 @@ def make_inputs(w: Workload, extra_rows: int = 0, lengths=None) -> dict:
     res = {"lengths": lengths, "cu_seqlens": torch.from_numpy(cu.astype(np.int32)),
            "q": q, "q_rope": q_rope, "workload": w}
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-    if w.kind in ("mla", "gla"):
+    if w.kind in ("mla", "gla", "gta"):
         width = G * w.d_k
         cache = torch.zeros((rows, width + w.d_rope), dtype=tdt)
         cache[:total, :width] = _normal(rng, (total, width), std, w.dtype)
@@ -194,11 +201,11 @@ def make_inputs(w: Workload, extra_rows: int = 0, lengths=None) -> dict:
 def new_token_rows(w: Workload, seed_offset: int = 1000) -> dict:
     """Rows for the s_q new tokens of every request (the cache-append input).
 
-    mla/gla: [B*s_q, G*d_k + d_R];  gqla: k/v [B*s_q, g, d_h] and kpe [B*s_q, d_R].
+    mla/gla/gta: [B*s_q, G*d_k + d_R];  gqla: k/v [B*s_q, g, d_h] and kpe [B*s_q, d_R].
     """
     rng = np.random.default_rng(w.seed + seed_offset)
     n = w.batch * w.s_q
-    if w.kind in ("mla", "gla"):
+    if w.kind in ("mla", "gla", "gta"):
         return {"rows": _normal(rng, (n, w.groups * w.d_k + w.d_rope), w.input_std, w.dtype)}
     return {"k": _normal(rng, (n, w.groups, w.d_k), w.input_std, w.dtype),
             "v": _normal(rng, (n, w.groups, w.d_v), w.input_std, w.dtype),

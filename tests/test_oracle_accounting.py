@@ -40,6 +40,16 @@ def test_gqa_intensity(key):
     _close(ai, e)
 
 
+def test_gta_cache_fraction():
+    """Tied groups store g*d_h + d_R per token against GQA's 2*g*d_h + d_R."""
+    e = GOLD["gta_cache_fraction_vs_gqa"]
+    s = e["setting"]
+    gta = acc.cache_bytes_per_token("gta", s["g"], s["d_h"], s["d_h"], s["d_rope"])
+    gqa = acc.cache_bytes_per_token("gqla", s["g"], s["d_h"], s["d_h"], s["d_rope"])
+    assert gta == 2 * (s["g"] * s["d_h"] + s["d_rope"])
+    _close(1 - gta / gqa, e)
+
+
 def test_heads_per_group():
     e = GOLD["gqla_heads_per_group"]
     _close(e["setting"]["h_q"] // e["setting"]["g"], e)

@@ -91,6 +91,25 @@ def test_mla_and_gla_instances_match_brute_force():
     np.testing.assert_allclose(lse, bl, atol=1e-12)
 
 
+def test_gta_instance_matches_brute_force():
+    """GTA, g = 2 tied groups of width 3: heads 0, 1 read columns 0..2 as key and value,
+    heads 2, 3 read columns 3..5; the RoPE key is shared."""
+    rng = np.random.default_rng(11)
+    B, S, H, g, d, dr = 2, 2, 4, 2, 3, 2
+    lengths = [3, 6]
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    T = int(cu[-1])
+    q = rng.standard_normal((B, S, H, d))
+    qr = rng.standard_normal((B, S, H, dr))
+    kv = rng.standard_normal((T, g * d))
+    kr = rng.standard_normal((T, dr))
+    out, lse = oracle.gta_group_decode(q, qr, kv, kr, g, cu, 0.6)
+    tied = np.stack([kv[:, :d], kv[:, d:]], axis=1)
+    bo, bl = _brute(q, qr, tied, tied, kr, cu, 0.6)
+    np.testing.assert_allclose(out, bo, atol=1e-12)
+    np.testing.assert_allclose(lse, bl, atol=1e-12)
+
+
 def test_brute_force_itself_on_hand_example():
     """One key pair worked by hand: s = scale*(q.k + qr.kr) for two keys, then a 2-way softmax."""
     q = np.array([[[[1.0, 2.0]]]])          # B=1,S=1,H=1,dk=2
