@@ -102,7 +102,7 @@ def job_throughput(tokens_per_rank: int, ms_this_rank: float, world: int, device
 def workload_accounting(w, lengths):
     """Algorithmic bytes (cache rows once, q, out, lse) and FLOPs (visible query-key pairs)."""
     lengths = np.asarray(lengths, dtype=np.int64)
-    if w.kind in ("mla", "gla"):
+    if w.kind in ("mla", "gla", "gta"):
         row = w.groups * w.d_k + w.d_rope
     else:
         row = w.groups * (w.d_k + w.d_v) + w.d_rope
@@ -185,7 +185,7 @@ def bench_gpu(args, rank, world, local_rank):
     q = d["q"].to(dev)
     qr = d["q_rope"].to(dev)
     B, S = w.batch, w.s_q
-    if w.kind in ("mla", "gla"):
+    if w.kind in ("mla", "gla", "gta"):
         cache = d["cache"].to(dev)
         width = w.groups * w.d_k
         lat, kpe = cache[:, :width], cache[:, width:]
@@ -199,14 +199,14 @@ def bench_gpu(args, rank, world, local_rank):
     if w.kind == "mla":
         ws = torch.empty(lkv.mla_decode_workspace_size(B, S, w.h_q, w.d_k, nsm), dtype=torch.uint8, device=dev)
     else:
-        kind = lkv.KIND_GQLA if w.kind == "gqla" else lkv.KIND_GLA
+        kind = {"gqla": lkv.KIND_GQLA, "gla": lkv.KIND_GLA, "gta": lkv.KIND_GTA}[w.kind]
         ws = torch.empty(lkv.group_decode_workspace_size(kind, B, S, w.h_q, w.groups, w.d_v, nsm),
                          dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     launches_per_step = 3 if w.kind != "gqla" else 5   # append(s) + decode + combine
 
     def append():
-        if w.kind in ("mla", "gla"):
+        if w.kind in ("mla", "gla", "gta"):
             lkv.latent_cache_append(new_rows, cache, cu, S)
         else:
             lkv.latent_cache_append(new_k, k, cu, S)
@@ -218,6 +218,8 @@ def bench_gpu(args, rank, world, local_rank):
             lkv.mla_absorbed_decode(qq, qqr, lat, kpe, cu, w.scale, out=o, lse=l, workspace=ws)
         elif w.kind == "gqla":
             lkv.gqla_group_decode(qq, qqr, k, v, kpe, cu, w.scale, out=o, lse=l, workspace=ws)
+        elif w.kind == "gta":
+            lkv.gta_group_decode(qq, qqr, lat, kpe, w.groups, cu, w.scale, out=o, lse=l, workspace=ws)
         else:
             lkv.gla_group_decode(qq, qqr, lat, kpe, w.groups, cu, w.scale, out=o, lse=l, workspace=ws)
 
@@ -273,7 +275,7 @@ def bench_gpu(args, rank, world, local_rank):
     lse_h = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
     q_d = torch.empty_like(q)
     qr_d = torch.empty_like(qr)
-    if w.kind in ("mla", "gla"):
+    if w.kind in ("mla", "gla", "gta"):
         rows_h = new["rows"].pin_memory()
         step_in = [(rows_h, new_rows)]
     else:
@@ -383,6 +385,11 @@ def cpu_baseline(w, budget_s: float):
             oracle.mla_absorbed_decode(d["q"], d["q_rope"], c[:, :w.d_k], c[:, w.d_k:], cu, w.scale, requests=[b])
         elif w.kind == "gqla":
             oracle.gqla_group_decode(d["q"], d["q_rope"], d["k"], d["v"], d["kpe"], cu, w.scale, requests=[b])
+        elif w.kind == "gta":
+            width = w.groups * w.d_k
+            c = d["cache"]
+            oracle.gta_group_decode(d["q"], d["q_rope"], c[:, :width], c[:, width:], w.groups, cu, w.scale,
+                                    requests=[b])
         else:
             width = w.groups * w.d_k
             c = d["cache"]

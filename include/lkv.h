@@ -70,7 +70,8 @@ const char* lkv_status_string(int status);
  * (request, unit) pairs are laid end to end and cut into `ranges` equal runs, one per
  * persistent CTA (MLA: per CTA pair).  A unit is one query token of a request for MLA,
  * one group of a request for GQLA / GLA.  Returns the number of ranges, or -1 on bad input.
- *   kind: 0 = MLA absorbed, 1 = GQLA, 2 = GLA.  num_sms: SMs available on the device.
+ *   kind: 0 = MLA absorbed, 1 = GQLA, 2 = GLA, 3 = GTA (partitioned like GQLA).
+ *   num_sms: SMs available on the device.
  */
 int lkv_plan_ranges(int kind, int batch, int s_q, int groups, int num_sms);
 
@@ -78,7 +79,7 @@ int lkv_plan_ranges(int kind, int batch, int s_q, int groups, int num_sms);
  * Host-only view of the same partition (no CUDA call): for host-side cu_seqlens_host [batch+1]
  * and `num_ranges` ranges, writes one record of 8 int32 per segment, in processing order:
  *   (range, request, unit, tile_lo, tile_hi, complete, slot, unit_id)
- * tiles are 64 keys (MLA, GLA) or 128 keys (GQLA); slot is -1 for a segment that covers its whole unit, else the partial
+ * tiles are 64 keys (MLA, GLA) or 128 keys (GQLA, GTA); slot is -1 for a segment that covers its whole unit, else the partial
  * slot (0 = first segment of its range, 1 = last).  Returns the number of segments (records
  * past max_out are counted but not written), or -1 on bad input.
  */
@@ -147,6 +148,26 @@ lkv_status lkv_gla_group_decode(const void* q, const void* q_rope, const void* c
                                 int64_t clat_row_stride, const void* kpe, int64_t kpe_row_stride,
                                 int64_t cache_rows, const int32_t* cu_seqlens, int batch, int s_q,
                                 int h_q, int n_lat, int r_g, int d_rope, float scale, int dtype,
+                                void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                lkv_stream_t stream);
+
+/*
+ * GTA (grouped-tied attention) decode: the heads of group j read one tied state per cached token
+ * as both their key (with the shared RoPE key appended) and their value.  Source: the Grouped
+ * Latent Attention article (news page), section "GTA": K and V parameters are tied inside a
+ * group, so the cache holds g*d_h + d_rope elements per token, about half of GQA's.
+ *   q      [batch, s_q, h_q, d_h], q_rope [batch, s_q, h_q, d_rope] contiguous
+ *   kv     [cache_rows, g, d_h] row stride kv_row_stride (elements, >= g*d_h); kpe
+ *          [cache_rows, d_rope] row stride kpe_row_stride (kv and kpe may interleave in one
+ *          [cache_rows, g*d_h + d_rope] array)
+ *   out    [batch, s_q, h_q, d_h]; lse [batch, s_q, h_q]
+ * Runs the grouped kernel of lkv_gqla_group_decode with its value stream reading the key rows:
+ * same limits, same workspace (lkv_group_decode_workspace_size with kind 1 or 3).
+ */
+lkv_status lkv_gta_group_decode(const void* q, const void* q_rope, const void* kv,
+                                int64_t kv_row_stride, const void* kpe, int64_t kpe_row_stride,
+                                int64_t cache_rows, const int32_t* cu_seqlens, int batch, int s_q,
+                                int h_q, int g, int d_h, int d_rope, float scale, int dtype,
                                 void* out, float* lse, void* workspace, size_t workspace_bytes,
                                 lkv_stream_t stream);
 

@@ -29,7 +29,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE = range(6)
 BF16, FP32 = 0, 1
-KIND_MLA, KIND_GQLA, KIND_GLA = 0, 1, 2
+KIND_MLA, KIND_GQLA, KIND_GLA, KIND_GTA = 0, 1, 2, 3
 
 _vp, _i64, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 
@@ -52,6 +52,8 @@ _gqla = _sig("lkv_gqla_group_decode", _i32, _vp, _vp, _vp, _i64, _vp, _i64, _vp,
              _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp)
 _gla = _sig("lkv_gla_group_decode", _i32, _vp, _vp, _vp, _i64, _vp, _i64, _i64, _vp,
             _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp)
+_gta = _sig("lkv_gta_group_decode", _i32, _vp, _vp, _vp, _i64, _vp, _i64, _i64, _vp,
+            _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp)
 _gqla_noalloc = _sig("lkv_gqla_group_decode_noalloc", _i32, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _i64,
                      _i64, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp)
 _append = _sig("lkv_latent_cache_append", _i32, _vp, _i64, _vp, _i64, _i64, _i64, _vp,
@@ -69,7 +71,7 @@ EXPORTED = ["lkv_version", "lkv_status_string", "lkv_plan_ranges", "lkv_mla_deco
             "lkv_gla_group_decode", "lkv_latent_cache_append", "lkv_merge_partials",
             "lkv_check_device", "lkv_selftest_wait_timeout", "lkv_plan_segments",
             "lkv_gqla_group_decode_noalloc", "lkv_absorb_query", "lkv_unabsorb_output",
-            "lkv_expand_latent"]
+            "lkv_expand_latent", "lkv_gta_group_decode"]
 
 
 class LkvError(RuntimeError):
@@ -222,6 +224,29 @@ def gqla_group_decode_noalloc(q, q_rope, k, v, kpe, cu_seqlens, scale, out=None,
                       _row_stride(kpe), k.shape[0], _ptr(cu_seqlens), B, s_q, h_q, g, d_h, d_r,
                       float(scale), _dtype_code(q), _ptr(out), _ptr(lse), _stream(stream)),
         "lkv_gqla_group_decode_noalloc")
+    return out, lse
+
+
+def gta_group_decode(q, q_rope, kv, kpe, g, cu_seqlens, scale, out=None, lse=None,
+                     workspace=None, stream=None):
+    """GTA decode over tied groups.  q [B,s_q,h_q,d_h], kv [rows, g*d_h] (tied key/value state
+    of each group, contiguous within a row), kpe [rows,d_R]."""
+    B, s_q, h_q, d_h = q.shape
+    d_r = q_rope.shape[-1]
+    dev = q.device
+    if kv.shape[-1] != g * d_h:
+        raise ValueError("kv rows must hold g * d_h elements")
+    if out is None:
+        out = torch.empty((B, s_q, h_q, d_h), dtype=q.dtype, device=dev)
+    if lse is None:
+        lse = torch.empty((B, s_q, h_q), dtype=torch.float32, device=dev)
+    if workspace is None and q.dtype == torch.bfloat16:
+        workspace = _alloc_ws(group_decode_workspace_size(KIND_GTA, B, s_q, h_q, g, d_h, _num_sms(dev)), dev)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _contig(q, q_rope, out, lse)
+    _ck(_gta(_ptr(q), _ptr(q_rope), _ptr(kv), _row_stride(kv), _ptr(kpe), _row_stride(kpe), kv.shape[0],
+             _ptr(cu_seqlens), B, s_q, h_q, g, d_h, d_r, float(scale), _dtype_code(q), _ptr(out), _ptr(lse),
+             _ptr(workspace), ws_bytes, _stream(stream)), "lkv_gta_group_decode")
     return out, lse
 
 

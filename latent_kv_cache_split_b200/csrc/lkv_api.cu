@@ -196,12 +196,14 @@ const char* lkv_status_string(int s) {
 }
 
 int lkv_plan_ranges(int kind, int batch, int s_q, int groups, int num_sms) {
+  if (kind == 3) kind = 1;  // GTA runs the GQLA kernel
   if (kind < 0 || kind > 2) return -1;
   return plan_ranges(kind, batch, s_q, kind == 0 ? 1 : groups, num_sms);
 }
 
 int lkv_plan_segments(int kind, const int32_t* cu_seqlens_host, int batch, int s_q, int groups,
                       int num_ranges, int32_t* out, int max_out) {
+  if (kind == 3) kind = 1;
   if (kind < 0 || kind > 2 || !cu_seqlens_host || batch <= 0 || s_q <= 0 || num_ranges <= 0 ||
       (kind != 0 && groups <= 0) || max_out < 0 || (max_out > 0 && !out))
     return -1;
@@ -249,6 +251,7 @@ size_t lkv_mla_decode_workspace_size(int batch, int s_q, int h_q, int r_kv, int 
 
 size_t lkv_group_decode_workspace_size(int kind, int batch, int s_q, int h_q, int groups, int d_v,
                                        int num_sms) {
+  if (kind == 3) kind = 1;
   if (kind != 1 && kind != 2) return 0;
   const int P = plan_ranges(kind, batch, s_q, groups, num_sms);
   if (P <= 0 || h_q <= 0 || groups <= 0 || h_q % groups || d_v <= 0) return 0;
@@ -434,6 +437,19 @@ lkv_status lkv_gqla_group_decode(const void* q, const void* q_rope, const void* 
   L.units_per_req = g;
   L.per_query_units = 0;
   return run_tc(L, *d, s);
+}
+
+lkv_status lkv_gta_group_decode(const void* q, const void* q_rope, const void* kv,
+                                int64_t kv_row_stride, const void* kpe, int64_t kpe_row_stride,
+                                int64_t cache_rows, const int32_t* cu_seqlens, int batch, int s_q,
+                                int h_q, int g, int d_h, int d_rope, float scale, int dtype,
+                                void* out, float* lse, void* workspace, size_t workspace_bytes,
+                                lkv_stream_t stream) {
+  // Tied groups: the value stream reads the key rows.  The grouped kernel never writes K or V, and
+  // the second read of a tile follows the first within a few tiles, so it is served from L2.
+  return lkv_gqla_group_decode(q, q_rope, kv, kv_row_stride, kv, kv_row_stride, kpe, kpe_row_stride,
+                               cache_rows, cu_seqlens, batch, s_q, h_q, g, d_h, d_rope, scale, dtype,
+                               out, lse, workspace, workspace_bytes, stream);
 }
 
 lkv_status lkv_gla_group_decode(const void* q, const void* q_rope, const void* clat,

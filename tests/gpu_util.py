@@ -34,6 +34,9 @@ def run_lib(L, d):
         return L.gqla_group_decode(d["q"], d["q_rope"], d["k"], d["v"], d["kpe"],
                                    d["cu_seqlens"], w.scale)
     c = d["cache"]
+    if w.kind == "gta":
+        return L.gta_group_decode(d["q"], d["q_rope"], c[:, :w.groups * w.d_k], c[:, w.groups * w.d_k:],
+                                  w.groups, d["cu_seqlens"], w.scale)
     return L.gla_group_decode(d["q"], d["q_rope"], c[:, :w.groups * w.d_k], c[:, w.groups * w.d_k:],
                               w.groups, d["cu_seqlens"], w.scale)
 
@@ -51,6 +54,9 @@ def run_oracle(d, requests=None):
                                         requests=requests)
     c = d["cache"]
     width = w.groups * w.d_k
+    if w.kind == "gta":
+        return oracle.gta_group_decode(d["q"], d["q_rope"], c[:, :width].contiguous(), c[:, width:], w.groups,
+                                       cu, w.scale, requests=requests)
     return oracle.gla_group_decode(d["q"], d["q_rope"], c[:, :width].contiguous(), c[:, width:], w.groups,
                                    cu, w.scale, requests=requests)
 

@@ -52,6 +52,8 @@ def test_version_and_status_strings(lkv):
     (2, 8, 1, 2, 148),      # GLA-2 long context: one range per SM (no lockstep for 2 groups)
     (1, 8, 1, 8, 144),
     (1, 1, 1, 8, 144),      # one request: every block is a slice of it
+    (3, 64, 2, 8, 144),     # GTA runs the GQLA kernel and partition
+    (1, 64, 2, 2, 128),     # GQA-2: 128 equal units nearly fill 148 SMs: one range per unit
 ])
 def test_plan_ranges(lkv, kind, B, s_q, G, want):
     assert lkv.plan_ranges(kind, B, s_q, G, 148) == want
@@ -69,7 +71,8 @@ def test_workspace_sizes(lkv):
     assert mla >= 2 * P * 128 * 512 * 4 + 2 * P * 128 * 4 + 2 * P * 4
     g = lkv.group_decode_workspace_size(1, 64, 2, 128, 8, 128, 148)
     assert g >= 2 * 144 * 32 * 128 * 4
-    assert lkv.group_decode_workspace_size(3, 1, 1, 128, 8, 128, 148) == 0
+    assert lkv.group_decode_workspace_size(3, 64, 2, 128, 8, 128, 148) == g   # GTA: the GQLA layout
+    assert lkv.group_decode_workspace_size(4, 1, 1, 128, 8, 128, 148) == 0
     assert lkv.group_decode_workspace_size(1, 1, 1, 128, 7, 128, 148) == 0
 
 
@@ -196,6 +199,13 @@ def test_validation_errors_need_no_gpu(lkv):
     g = L._gla(P16, P16, P16, 512, P16, 64, 1000, cu, 2, 1, 128, 2, 128, 64, 0.05, 0, P16, P16,
                P16, 1 << 30, None)
     assert g == L.ERR_UNSUPPORTED
+    # GTA: tied rows shorter than g*d_h; h_q not a multiple of g; unsupported head width
+    assert L._gta(P16, P16, P16, 1000, P16, 1088, 1000, cu, 2, 2, 128, 8, 128, 64, 0.07, 0,
+                  P16, P16, P16, 1 << 30, None) == L.ERR_INVALID_ARG
+    assert L._gta(P16, P16, P16, 1088, P16, 1088, 1000, cu, 2, 2, 128, 3, 128, 64, 0.07, 0,
+                  P16, P16, P16, 1 << 30, None) == L.ERR_INVALID_ARG
+    assert L._gta(P16, P16, P16, 1088, P16, 1088, 1000, cu, 2, 2, 128, 8, 96, 64, 0.07, 0,
+                  P16, P16, P16, 1 << 30, None) == L.ERR_UNSUPPORTED
     # append: misaligned row size
     assert L._append(P16, 24, P16, 24, 10, 24, cu, 1, 1, None) == L.ERR_INVALID_ARG
     assert L._merge(P16, P16, 0, 4, 8, 0, P16, P16, None) == L.ERR_INVALID_ARG

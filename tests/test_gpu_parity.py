@@ -81,6 +81,33 @@ def test_gla_small(L, gpu, s_q, lengths):
     _run(L, gpu, w, lengths=lengths)
 
 
+@pytest.mark.parametrize("s_q,lengths", [(2, [130, 7]), (1, [1, 200, 64]), (2, [8192, 2, 129])])
+def test_gta_small(L, gpu, s_q, lengths):
+    """Tied groups (K_j = V_j) through the grouped kernel: ragged tails, one-key requests, splits."""
+    w = synth.workload("gta_g8_sq2_l8192", batch=len(lengths), s_q=s_q, seqlen=None)
+    _run(L, gpu, w, lengths=lengths)
+
+
+def test_gta_b64_l8192_sampled(L, gpu):
+    _run(L, gpu, synth.workload("gta_g8_sq2_l8192"), requests=[0, 29, 63])
+
+
+def test_gta_unscaled_stress(L, gpu):
+    w = synth.workload("gta_g8_sq2_l8192", batch=3, seqlen=700, input_std=1.0)
+    _run(L, gpu, w)
+
+
+@pytest.mark.parametrize("s_q,lengths", [(2, [130, 7]), (1, [1, 300, 64]), (2, [4097, 2])])
+def test_gqa2_small(L, gpu, s_q, lengths):
+    """Two K/V groups of 64 heads: 128 score rows per unit at s_q = 2 (the full M of one UMMA)."""
+    w = synth.workload("gqa2_sq2_l8192", batch=len(lengths), s_q=s_q, seqlen=None)
+    _run(L, gpu, w, lengths=lengths)
+
+
+def test_gqa2_b64_l8192_sampled(L, gpu):
+    _run(L, gpu, synth.workload("gqa2_sq2_l8192"), requests=[0, 40])
+
+
 @pytest.mark.parametrize("name,requests", [("long_gla2", [0, 5]), ("long_mla", [3]),
                                            ("long_gqla_g8", [6])])
 def test_long_context_sampled(L, gpu, name, requests):
