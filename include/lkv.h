@@ -216,6 +216,43 @@ lkv_status lkv_latent_cache_append(const void* new_rows, int64_t new_row_stride_
                                    lkv_stream_t stream);
 
 /*
+ * FP8 (e4m3) latent cache rows (the pages run FP8 inference -- Grouped Latent Attention article,
+ * section on the GLA-vs-MLA decoding test -- but fix no format; this is the library's reading).
+ * One row per token of lkv_fp8_cache_row_bytes(r, d_rope) = r + 16 + 2*d_rope bytes:
+ *   bytes [0, r)          e4m3 codes of the latent row (OCP E4M3: bias 7, largest finite 448)
+ *   bytes [r, r + 4)      fp32 scale s = max|latent row| / 448 (0 for an all-zero row)
+ *   bytes [r + 4, r + 16) zero
+ *   bytes [r + 16, ...)   the bf16 RoPE key, copied unchanged
+ * The dequantised latent is e4m3(code) * s.  Codes are taken in fp32: y = x / s (IEEE division),
+ * clamped to [-448, 448], rounded to the nearest e4m3 value with ties to the even code.
+ * lkv_fp8_cache_row_bytes returns 0 unless r is a multiple of 16 in [16, 1024] and d_rope a
+ * non-negative multiple of 8 (host-only, no CUDA call).
+ */
+size_t lkv_fp8_cache_row_bytes(int r, int d_rope);
+
+/*
+ * Quantise n_rows bf16 rows into FP8 cache rows, row i to row i.
+ *   src    [n_rows, >= r + d_rope] bf16: latent in columns [0, r), RoPE key in [r, r + d_rope);
+ *          row stride src_row_stride elements (its byte size a multiple of 16); 16-byte aligned
+ *   cache  [n_rows] rows of cache_row_stride_bytes (a multiple of 16, >= the row size), aligned
+ * Source values must be finite.  Asynchronous on `stream`.
+ */
+lkv_status lkv_quantize_latent_fp8(const void* src, int64_t src_row_stride, void* cache,
+                                   int64_t cache_row_stride_bytes, int64_t n_rows, int r, int d_rope,
+                                   lkv_stream_t stream);
+
+/*
+ * Cache append into an FP8 cache: quantise the s_q new bf16 rows of every request (row b*s_q + i
+ * of new_rows, laid out as for lkv_quantize_latent_fp8) into cache row cu_seqlens[b] + L_b - s_q + i
+ * (the destinations of lkv_latent_cache_append).  A request with L_b < s_q or a destination past
+ * cache_rows is skipped and recorded in the device error word.
+ */
+lkv_status lkv_latent_cache_append_fp8(const void* new_rows, int64_t new_row_stride, void* cache,
+                                       int64_t cache_row_stride_bytes, int64_t cache_rows, int r,
+                                       int d_rope, const int32_t* cu_seqlens, int batch, int s_q,
+                                       lkv_stream_t stream);
+
+/*
  * Merge attention results computed over disjoint key sets (split-KV combine):
  *   lse[r] = ln sum_p exp(lse_parts[p, r]);  out[r, :] = sum_p exp(lse_parts[p, r] - lse[r]) * o_parts[p, r, :]
  *   o_parts [n_parts, rows, d_v] fp32, lse_parts [n_parts, rows] fp32 (a part with lse = -inf

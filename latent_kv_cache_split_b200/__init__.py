@@ -9,7 +9,9 @@ Functions (same names as the C entry points without the ``lkv_`` prefix):
     mla_absorbed_decode, gqla_group_decode, gla_group_decode, latent_cache_append,
     merge_partials, check_device, selftest_wait_timeout, plan_ranges,
     mla_decode_workspace_size, group_decode_workspace_size,
-    absorb_query, unabsorb_output, expand_latent (the projections either side of the path)
+    absorb_query, unabsorb_output, expand_latent (the projections either side of the path),
+    gta_group_decode, fp8_cache_row_bytes, quantize_latent_fp8, latent_cache_append_fp8
+    (and fp8_cache_fields: views of the fields of FP8 cache rows)
 """
 from __future__ import annotations
 
@@ -30,6 +32,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE = range(6)
 BF16, FP32 = 0, 1
 KIND_MLA, KIND_GQLA, KIND_GLA, KIND_GTA = 0, 1, 2, 3
+SITE_SELFTEST, SITE_BAD_LENGTH, SITE_BAD_ROW, SITE_WAIT_BASE = 1, 2, 3, 100   # device error word
 
 _vp, _i64, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 
@@ -54,6 +57,10 @@ _gla = _sig("lkv_gla_group_decode", _i32, _vp, _vp, _vp, _i64, _vp, _i64, _i64, 
             _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp)
 _gta = _sig("lkv_gta_group_decode", _i32, _vp, _vp, _vp, _i64, _vp, _i64, _i64, _vp,
             _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp)
+_fp8_row_bytes = _sig("lkv_fp8_cache_row_bytes", _sz, _i32, _i32)
+_quant_fp8 = _sig("lkv_quantize_latent_fp8", _i32, _vp, _i64, _vp, _i64, _i64, _i32, _i32, _vp)
+_append_fp8 = _sig("lkv_latent_cache_append_fp8", _i32, _vp, _i64, _vp, _i64, _i64, _i32, _i32, _vp,
+                   _i32, _i32, _vp)
 _gqla_noalloc = _sig("lkv_gqla_group_decode_noalloc", _i32, _vp, _vp, _vp, _i64, _vp, _i64, _vp, _i64,
                      _i64, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp)
 _append = _sig("lkv_latent_cache_append", _i32, _vp, _i64, _vp, _i64, _i64, _i64, _vp,
@@ -71,7 +78,8 @@ EXPORTED = ["lkv_version", "lkv_status_string", "lkv_plan_ranges", "lkv_mla_deco
             "lkv_gla_group_decode", "lkv_latent_cache_append", "lkv_merge_partials",
             "lkv_check_device", "lkv_selftest_wait_timeout", "lkv_plan_segments",
             "lkv_gqla_group_decode_noalloc", "lkv_absorb_query", "lkv_unabsorb_output",
-            "lkv_expand_latent", "lkv_gta_group_decode"]
+            "lkv_expand_latent", "lkv_gta_group_decode", "lkv_fp8_cache_row_bytes",
+            "lkv_quantize_latent_fp8", "lkv_latent_cache_append_fp8"]
 
 
 class LkvError(RuntimeError):
@@ -281,6 +289,53 @@ def latent_cache_append(new_rows, cache, cu_seqlens, s_q, stream=None):
     _ck(_append(_ptr(new_rows), new_rows.stride(0) * new_rows.element_size(), _ptr(cache),
                 cache.stride(0) * cache.element_size(), cache.shape[0], row_bytes,
                 _ptr(cu_seqlens), B, s_q, _stream(stream)), "lkv_latent_cache_append")
+    return cache
+
+
+def fp8_cache_row_bytes(r: int, d_rope: int) -> int:
+    """Bytes of one FP8 cache row (e4m3 latent, fp32 scale + pad, bf16 RoPE key); 0 if unsupported."""
+    return _fp8_row_bytes(r, d_rope)
+
+
+def fp8_cache_fields(cache, r: int, d_rope: int):
+    """Views of the fields of FP8 cache rows cache [rows, >= row_bytes] uint8 (row stride and
+    start 16-byte aligned): (codes uint8 [rows, r], scales fp32 [rows], k_rope bf16 [rows, d_rope])."""
+    rb = fp8_cache_row_bytes(r, d_rope)
+    if (rb == 0 or cache.dtype != torch.uint8 or cache.dim() != 2 or cache.shape[1] < rb
+            or cache.stride(1) != 1 or cache.stride(0) % 16 or cache.storage_offset() % 16):
+        raise ValueError("cache must be [rows, >= row_bytes] uint8 rows on 16-byte boundaries")
+    rows, rs, off = cache.shape[0], cache.stride(0), cache.storage_offset()
+    st = cache.untyped_storage()
+    scales = torch.empty(0, dtype=torch.float32, device=cache.device).set_(st, (off + r) // 4, (rows,), (rs // 4,))
+    kpe = torch.empty(0, dtype=torch.bfloat16, device=cache.device).set_(st, (off + r + 16) // 2, (rows, d_rope),
+                                                                           (rs // 2, 1))
+    return cache[:, :r], scales, kpe
+
+
+def quantize_latent_fp8(rows, r: int, cache=None, stream=None):
+    """Quantise bf16 rows [n, >= r + d_rope] (latent then RoPE key) into FP8 cache rows, row i to
+    row i.  Returns the cache [n, row_bytes] uint8 (allocated if not given)."""
+    n, width = rows.shape
+    d_rope = width - r
+    rb = fp8_cache_row_bytes(r, d_rope)
+    if rb == 0:
+        raise ValueError("unsupported r / d_rope for the FP8 cache")
+    if cache is None:
+        cache = torch.empty((n, rb), dtype=torch.uint8, device=rows.device)
+    _ck(_quant_fp8(_ptr(rows), _row_stride(rows), _ptr(cache), cache.stride(0), n, r, d_rope,
+                   _stream(stream)), "lkv_quantize_latent_fp8")
+    return cache
+
+
+def latent_cache_append_fp8(new_rows, cache, cu_seqlens, s_q, r: int, stream=None):
+    """Quantise row b*s_q+i of the bf16 new_rows [B*s_q, r + d_rope] into FP8 cache row
+    cu[b] + L_b - s_q + i of cache [rows, row_bytes] uint8."""
+    n, width = new_rows.shape
+    B = cu_seqlens.numel() - 1
+    if n != B * s_q:
+        raise ValueError("new_rows must hold batch * s_q rows")
+    _ck(_append_fp8(_ptr(new_rows), _row_stride(new_rows), _ptr(cache), cache.stride(0), cache.shape[0], r,
+                    width - r, _ptr(cu_seqlens), B, s_q, _stream(stream)), "lkv_latent_cache_append_fp8")
     return cache
 
 

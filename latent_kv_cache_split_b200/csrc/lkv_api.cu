@@ -179,6 +179,15 @@ lkv_status common_checks(const void* q, const void* qr, const int32_t* cu, const
 
 }  // namespace
 
+// Device address of the error word of the current device, for the kernels of the other translation
+// units (which cannot name the __device__ variable); sets the device up on first use.
+lkv_status lkv_internal_error_word(int** err) {
+  DeviceState* d;
+  const lkv_status st = device_state(&d);
+  if (st == LKV_OK) *err = d->err;
+  return st;
+}
+
 extern "C" {
 
 int lkv_version(void) { return 100; }

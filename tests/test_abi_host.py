@@ -227,3 +227,23 @@ def test_projection_argument_errors_need_no_gpu(lkv):
     assert lkv._expand(P, 8, P, P, 4, 2, 16, 8, 0, st) == lkv.ERR_INVALID_ARG      # row stride < r
     assert lkv._expand(P, 16, P, P, 0, 2, 16, 8, 0, st) == lkv.ERR_INVALID_ARG
     assert lkv._expand(P, 16, P, P, 4, 2, 16, 8, 1, st) == lkv.ERR_UNSUPPORTED
+
+
+def test_fp8_cache_rows_host_side(lkv):
+    """FP8 row size and argument checks: no CUDA call is made for any of these."""
+    assert lkv.fp8_cache_row_bytes(512, 64) == 656
+    assert lkv.fp8_cache_row_bytes(16, 0) == 32
+    assert lkv.fp8_cache_row_bytes(1024, 8) == 1056
+    for r, dr in [(0, 64), (500, 64), (1040, 64), (512, 60), (512, -8)]:
+        assert lkv.fp8_cache_row_bytes(r, dr) == 0
+    P = _fake(1 << 20)
+    st = ctypes.c_void_p(0)
+    assert lkv._quant_fp8(None, 576, P, 656, 4, 512, 64, st) == lkv.ERR_INVALID_ARG
+    assert lkv._quant_fp8(_fake((1 << 20) + 8), 576, P, 656, 4, 512, 64, st) == lkv.ERR_INVALID_ARG  # misaligned
+    assert lkv._quant_fp8(P, 570, P, 656, 4, 512, 64, st) == lkv.ERR_INVALID_ARG    # rows shorter than r + d_rope
+    assert lkv._quant_fp8(P, 580, P, 656, 4, 512, 64, st) == lkv.ERR_INVALID_ARG    # 1160-byte source rows
+    assert lkv._quant_fp8(P, 576, P, 640, 4, 512, 64, st) == lkv.ERR_INVALID_ARG    # cache rows too short
+    assert lkv._quant_fp8(P, 576, P, 656, 0, 512, 64, st) == lkv.ERR_INVALID_ARG
+    assert lkv._quant_fp8(P, 576, P, 656, 4, 500, 64, st) == lkv.ERR_INVALID_ARG
+    assert lkv._append_fp8(P, 576, P, 656, 10, 512, 64, None, 2, 1, st) == lkv.ERR_INVALID_ARG
+    assert lkv._append_fp8(P, 576, P, 656, 10, 512, 64, P, 0, 1, st) == lkv.ERR_INVALID_ARG
