@@ -216,6 +216,19 @@ lkv_status lkv_latent_cache_append(const void* new_rows, int64_t new_row_stride_
                                    lkv_stream_t stream);
 
 /*
+ * Output projection y = o W_O (bf16 operands, fp32 accumulation; cuBLAS, as the other projections).
+ *   o    [n_tok, k] bf16 row-major: the heads' attention outputs side by side (k = heads * d_v)
+ *   w_o  [k, d_model] bf16 row-major
+ *   y    [n_tok, d_model], bf16 (out_dtype LKV_BF16) or fp32 (LKV_FP32)
+ * With the heads split along the group axis across GPUs (GQLA explainer, section 2, GQA path), each
+ * GPU passes its heads' columns of o and the matching row block of W_O and gets a partial y; the sum
+ * over GPUs is the full projection.  LKV_ERR_INVALID_ARG for NULL pointers, non-positive sizes or
+ * another out_dtype; LKV_ERR_UNSUPPORTED if cuBLAS cannot be opened.
+ */
+lkv_status lkv_output_projection(const void* o, const void* w_o, void* y, int n_tok, int k, int d_model,
+                                 int out_dtype, lkv_stream_t stream);
+
+/*
  * FP8 (e4m3) latent cache rows (the pages run FP8 inference -- Grouped Latent Attention article,
  * section on the GLA-vs-MLA decoding test -- but fix no format; this is the library's reading).
  * One row per token of lkv_fp8_cache_row_bytes(r, d_rope) = r + 16 + 2*d_rope bytes:

@@ -72,6 +72,7 @@ _segments = _sig("lkv_plan_segments", _i32, _i32, _vp, _i32, _i32, _i32, _i32, _
 _absorb = _sig("lkv_absorb_query", _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp)
 _unabsorb = _sig("lkv_unabsorb_output", _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp)
 _expand = _sig("lkv_expand_latent", _i32, _vp, _i64, _vp, _vp, _i64, _i32, _i32, _i32, _i32, _vp)
+_oproj = _sig("lkv_output_projection", _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _vp)
 
 EXPORTED = ["lkv_version", "lkv_status_string", "lkv_plan_ranges", "lkv_mla_decode_workspace_size",
             "lkv_group_decode_workspace_size", "lkv_mla_absorbed_decode", "lkv_gqla_group_decode",
@@ -79,7 +80,7 @@ EXPORTED = ["lkv_version", "lkv_status_string", "lkv_plan_ranges", "lkv_mla_deco
             "lkv_check_device", "lkv_selftest_wait_timeout", "lkv_plan_segments",
             "lkv_gqla_group_decode_noalloc", "lkv_absorb_query", "lkv_unabsorb_output",
             "lkv_expand_latent", "lkv_gta_group_decode", "lkv_fp8_cache_row_bytes",
-            "lkv_quantize_latent_fp8", "lkv_latent_cache_append_fp8"]
+            "lkv_quantize_latent_fp8", "lkv_latent_cache_append_fp8", "lkv_output_projection"]
 
 
 class LkvError(RuntimeError):
@@ -410,4 +411,22 @@ def expand_latent(c, w, out=None, stream=None):
     _contig(w, out)
     _ck(_expand(_ptr(c), _row_stride(c), _ptr(w), _ptr(out), T, G, r, d, _dtype_code(c), _stream(stream)),
         "lkv_expand_latent")
+    return out
+
+
+def output_projection(o, w_o, out_dtype=torch.float32, out=None, stream=None):
+    """y = o @ w_o.  o [n_tok, k] (or [n_tok, heads, d_v], flattened) bf16 contiguous, w_o [k, d_model]
+    bf16 contiguous -> y [n_tok, d_model] in out_dtype (fp32 by default: a partial sum to reduce)."""
+    n = o.shape[0]
+    o2 = o.reshape(n, -1)
+    k, d_model = w_o.shape
+    if o2.shape[1] != k:
+        raise ValueError("o and w_o disagree on k")
+    if o2.dtype != torch.bfloat16 or w_o.dtype != torch.bfloat16:
+        raise TypeError("output_projection takes bf16 operands")
+    if out is None:
+        out = torch.empty((n, d_model), dtype=out_dtype, device=o.device)
+    _contig(o2, w_o, out)
+    _ck(_oproj(_ptr(o2), _ptr(w_o), _ptr(out), n, k, d_model, _dtype_code(out), _stream(stream)),
+        "lkv_output_projection")
     return out

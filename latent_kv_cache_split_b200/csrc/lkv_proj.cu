@@ -2,7 +2,10 @@
 //   absorbed path:  q_abs[t, h, :] = W_UK[j(h)] q[t, h, :]       (the query in latent space)
 //                   out[t, h, :]   = W_UV[j(h)]^T o_lat[t, h, :]  (the output back in head space)
 //   GQA path:       X[t, j, :]     = c_KV[t, :] W[j]              (expanded K_j or V_j of the cache)
-// with j(h) = h / (h_q / G).  These are plain batched GEMMs (bf16 operands, fp32 accumulation, bf16
+// with j(h) = h / (h_q / G), and the output projection that follows attention,
+//                   y[t, :]        = o[t, :] W_O                  (o = the heads' outputs side by side)
+// which, with the heads split across GPUs along the group axis, gives each GPU a partial y to be summed
+// (GQLA explainer, section 2, GQA path: tensor parallelism along the group axis).  These are plain GEMMs (bf16 operands, fp32 accumulation, bf16
 // result), run by cuBLAS.  cuBLAS is opened at the first projection call (dlopen), so the decode path
 // and the rest of the library never depend on it; each device gets one cuBLAS handle, created at its
 // first projection call (cuBLAS allocates its own workspace then).
@@ -66,13 +69,14 @@ lkv_status handle_for(cudaStream_t stream, cublasHandle_t* out) {
   return LKV_OK;
 }
 
-// One strided-batched bf16 GEMM in cuBLAS's column-major terms: C = op(A) op(B), fp32 accumulate.
+// One strided-batched GEMM of bf16 operands in cuBLAS's column-major terms: C = op(A) op(B), fp32
+// accumulate, C in bf16 (or fp32 when c_fp32).
 lkv_status gemm(cublasHandle_t h, cublasOperation_t ta, int m, int n, int k, const void* A, int lda, long long sA,
-                const void* B, int ldb, long long sB, void* C, int ldc, long long sC, int batch) {
+                const void* B, int ldb, long long sB, void* C, int ldc, long long sC, int batch, bool c_fp32 = false) {
   const float one = 1.f, zero = 0.f;
   const cublasStatus_t s = cublas_api().gemm(h, ta, CUBLAS_OP_N, m, n, k, &one, A, CUDA_R_16BF, lda, sA, B, CUDA_R_16BF,
-                                             ldb, sB, &zero, C, CUDA_R_16BF, ldc, sC, batch, CUBLAS_COMPUTE_32F,
-                                             CUBLAS_GEMM_DEFAULT);
+                                             ldb, sB, &zero, C, c_fp32 ? CUDA_R_32F : CUDA_R_16BF, ldc, sC, batch,
+                                             CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
   return s == CUBLAS_STATUS_SUCCESS ? LKV_OK : LKV_ERR_CUDA;
 }
 
@@ -142,6 +146,17 @@ lkv_status lkv_expand_latent(const void* c, int64_t c_row_stride, const void* w,
   // per group j: (X_j)^T [d x T] = W_j^T [d x r] * c^T [r x T]
   return gemm(h, CUBLAS_OP_N, d, static_cast<int>(n_rows), r, w, d, static_cast<long long>(r) * d, c,
               static_cast<int>(c_row_stride), 0, x, groups * d, d, groups);
+}
+
+lkv_status lkv_output_projection(const void* o, const void* w_o, void* y, int n_tok, int k, int d_model,
+                                 int out_dtype, lkv_stream_t stream) {
+  if (!o || !w_o || !y || n_tok <= 0 || k <= 0 || d_model <= 0) return LKV_ERR_INVALID_ARG;
+  if (out_dtype != LKV_BF16 && out_dtype != LKV_FP32) return LKV_ERR_INVALID_ARG;
+  cublasHandle_t h;
+  const lkv_status st = handle_for(static_cast<cudaStream_t>(stream), &h);
+  if (st != LKV_OK) return st;
+  // y^T [d_model x n] = W_O^T [d_model x k] * o^T [k x n]
+  return gemm(h, CUBLAS_OP_N, d_model, n_tok, k, w_o, d_model, 0, o, k, 0, y, d_model, 0, 1, out_dtype == LKV_FP32);
 }
 
 }  // extern "C"

@@ -8,10 +8,10 @@ and identities in tests/test_oracle_*.py.
 """
 from .attend import (grouped_decode, mla_absorbed_decode, gqla_group_decode, gla_group_decode,
                      gta_group_decode, merge_partials, append_rows, append_destinations, visible_keys,
-                     absorb_query, unabsorb_output, expand_latent)
+                     absorb_query, unabsorb_output, expand_latent, output_projection)
 from . import accounting
 from . import fp8
 
 __all__ = ["grouped_decode", "mla_absorbed_decode", "gqla_group_decode", "gla_group_decode",
            "gta_group_decode", "merge_partials", "append_rows", "append_destinations", "visible_keys",
-           "absorb_query", "unabsorb_output", "expand_latent", "accounting", "fp8"]
+           "absorb_query", "unabsorb_output", "expand_latent", "output_projection", "accounting", "fp8"]

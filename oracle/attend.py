@@ -48,7 +48,7 @@ import numpy as np
 
 __all__ = ["grouped_decode", "mla_absorbed_decode", "gqla_group_decode", "gla_group_decode",
            "gta_group_decode", "merge_partials", "append_rows", "append_destinations", "visible_keys",
-           "absorb_query", "unabsorb_output", "expand_latent"]
+           "absorb_query", "unabsorb_output", "expand_latent", "output_projection"]
 
 
 def _f64(x) -> np.ndarray:
@@ -219,3 +219,11 @@ def expand_latent(c, w):
     c = _f64(c)
     w = _f64(w)
     return np.einsum("tr,grd->tgd", c, w)
+
+
+def output_projection(o, w_o):
+    """Output projection after attention: y[t, :] = sum over heads h and columns c of
+    o[t, h, c] * W_O[h*d_v + c, :]  (o [n, h, d_v] or [n, h*d_v], W_O [h*d_v, d_model])."""
+    o = _f64(o)
+    w = _f64(w_o)
+    return o.reshape(o.shape[0], -1) @ w

@@ -247,3 +247,11 @@ def test_fp8_cache_rows_host_side(lkv):
     assert lkv._quant_fp8(P, 576, P, 656, 4, 500, 64, st) == lkv.ERR_INVALID_ARG
     assert lkv._append_fp8(P, 576, P, 656, 10, 512, 64, None, 2, 1, st) == lkv.ERR_INVALID_ARG
     assert lkv._append_fp8(P, 576, P, 656, 10, 512, 64, P, 0, 1, st) == lkv.ERR_INVALID_ARG
+
+
+def test_output_projection_argument_errors_need_no_gpu(lkv):
+    P = _fake(1 << 20)
+    st = ctypes.c_void_p(0)
+    assert lkv._oproj(None, P, P, 4, 16, 8, 1, st) == lkv.ERR_INVALID_ARG
+    assert lkv._oproj(P, P, P, 0, 16, 8, 1, st) == lkv.ERR_INVALID_ARG
+    assert lkv._oproj(P, P, P, 4, 16, 8, 7, st) == lkv.ERR_INVALID_ARG

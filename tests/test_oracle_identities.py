@@ -123,3 +123,19 @@ def test_gla_is_block_diagonal_mla():
     for h in range(H):
         j = h // (H // 2)
         np.testing.assert_allclose(out_g[:, :, h], out_m[:, :, h, j * rg:(j + 1) * rg], atol=1e-13)
+
+
+def test_output_projection_identity_and_head_blocks():
+    """y = o W_O: with W_O = I the heads come back side by side, and splitting the heads into blocks
+    (the group-axis split) and summing the blocks' products gives the full projection."""
+    rng = np.random.default_rng(41)
+    o = rng.standard_normal((3, 4, 5))
+    y = oracle.output_projection(o, np.eye(20))
+    np.testing.assert_array_equal(y, o.reshape(3, 20))
+    w = rng.standard_normal((20, 7))
+    full = oracle.output_projection(o, w)
+    parts = sum(oracle.output_projection(o[:, h0:h0 + 2], w[h0 * 5:(h0 + 2) * 5]) for h0 in (0, 2))
+    np.testing.assert_allclose(parts, full, atol=1e-12)
+    # brute force on one entry
+    t, c = 2, 6
+    assert abs(full[t, c] - sum(o[t, h, e] * w[h * 5 + e, c] for h in range(4) for e in range(5))) < 1e-12
