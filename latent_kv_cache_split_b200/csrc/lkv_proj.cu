@@ -51,15 +51,21 @@ const CublasApi& cublas_api() {
 
 constexpr int kMaxDevices = 64;
 
-// The cuBLAS handle of the current device, bound to `stream`.
+// Serialises the projection calls of all host threads: a device's one handle is re-bound to the
+// caller's stream at every call, so the binding and the GEMMs it enqueues must not interleave with
+// another thread's.  Only the enqueueing is serialised, not the GPU work.
+std::mutex& proj_mutex() {
+  static std::mutex mu;
+  return mu;
+}
+
+// The cuBLAS handle of the current device, bound to `stream`.  Call with proj_mutex() held.
 lkv_status handle_for(cudaStream_t stream, cublasHandle_t* out) {
   const CublasApi& api = cublas_api();
   if (!api.ok) return LKV_ERR_UNSUPPORTED;
   static cublasHandle_t handles[kMaxDevices] = {};
-  static std::mutex mu;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LKV_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(mu);
   if (!handles[dev] && api.create(&handles[dev]) != CUBLAS_STATUS_SUCCESS) {
     handles[dev] = nullptr;
     return LKV_ERR_CUDA;
@@ -92,6 +98,7 @@ lkv_status lkv_absorb_query(const void* q, const void* w_uk, void* q_abs, int n_
       h_q % groups != 0 || !fits_int(static_cast<long long>(h_q) * r) || !fits_int(static_cast<long long>(h_q) * d_h))
     return LKV_ERR_INVALID_ARG;
   if (dtype != LKV_BF16) return LKV_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(proj_mutex());
   cublasHandle_t h;
   lkv_status st = handle_for(static_cast<cudaStream_t>(stream), &h);
   if (st != LKV_OK) return st;
@@ -116,6 +123,7 @@ lkv_status lkv_unabsorb_output(const void* o_lat, const void* w_uv, void* out, i
       h_q % groups != 0 || !fits_int(static_cast<long long>(h_q) * r) || !fits_int(static_cast<long long>(h_q) * d_v))
     return LKV_ERR_INVALID_ARG;
   if (dtype != LKV_BF16) return LKV_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(proj_mutex());
   cublasHandle_t h;
   lkv_status st = handle_for(static_cast<cudaStream_t>(stream), &h);
   if (st != LKV_OK) return st;
@@ -140,6 +148,7 @@ lkv_status lkv_expand_latent(const void* c, int64_t c_row_stride, const void* w,
       !fits_int(n_rows) || !fits_int(c_row_stride) || !fits_int(static_cast<long long>(groups) * d))
     return LKV_ERR_INVALID_ARG;
   if (dtype != LKV_BF16) return LKV_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(proj_mutex());
   cublasHandle_t h;
   const lkv_status st = handle_for(static_cast<cudaStream_t>(stream), &h);
   if (st != LKV_OK) return st;
@@ -152,6 +161,7 @@ lkv_status lkv_output_projection(const void* o, const void* w_o, void* y, int n_
                                  int out_dtype, lkv_stream_t stream) {
   if (!o || !w_o || !y || n_tok <= 0 || k <= 0 || d_model <= 0) return LKV_ERR_INVALID_ARG;
   if (out_dtype != LKV_BF16 && out_dtype != LKV_FP32) return LKV_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(proj_mutex());
   cublasHandle_t h;
   const lkv_status st = handle_for(static_cast<cudaStream_t>(stream), &h);
   if (st != LKV_OK) return st;
