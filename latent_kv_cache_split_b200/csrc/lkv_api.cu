@@ -39,8 +39,10 @@ unsigned long long wait_limit_ns() {
 }
 
 constexpr size_t tc_smem_bytes(int mode) {
-  return mode == MODE_MLA ? ModeCfg<MODE_MLA>::kSmemBytes
-                          : (mode == MODE_GQLA ? ModeCfg<MODE_GQLA>::kSmemBytes : ModeCfg<MODE_GLA>::kSmemBytes);
+  return mode == MODE_MLA    ? ModeCfg<MODE_MLA>::kSmemBytes
+         : mode == MODE_GQLA ? ModeCfg<MODE_GQLA>::kSmemBytes
+         : mode == MODE_GTA  ? ModeCfg<MODE_GTA>::kSmemBytes
+                             : ModeCfg<MODE_GLA>::kSmemBytes;
 }
 
 // Per-device one-time set-up: SM count, error-word address, kernel attributes.
@@ -59,7 +61,9 @@ lkv_status device_state(DeviceState** out) {
         cudaFuncSetAttribute(decode_tc_kernel<MODE_GQLA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(tc_smem_bytes(MODE_GQLA))) != cudaSuccess ||
         cudaFuncSetAttribute(decode_tc_kernel<MODE_GLA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(tc_smem_bytes(MODE_GLA))) != cudaSuccess)
+                             static_cast<int>(tc_smem_bytes(MODE_GLA))) != cudaSuccess ||
+        cudaFuncSetAttribute(decode_tc_kernel<MODE_GTA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(tc_smem_bytes(MODE_GTA))) != cudaSuccess)
       return LKV_ERR_CUDA;
     d.ready = true;
   }
@@ -130,6 +134,8 @@ lkv_status run_tc(TcLaunch& L, const DeviceState& d, cudaStream_t stream) {
     e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<MODE_MLA>, L.map_a, L.map_r, L.map_v, L.p);
   } else if (L.mode == MODE_GQLA) {
     e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<MODE_GQLA>, L.map_a, L.map_r, L.map_v, L.p);
+  } else if (L.mode == MODE_GTA) {
+    e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<MODE_GTA>, L.map_a, L.map_r, L.map_v, L.p);
   } else {
     e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<MODE_GLA>, L.map_a, L.map_r, L.map_v, L.p);
   }
@@ -454,11 +460,62 @@ lkv_status lkv_gta_group_decode(const void* q, const void* q_rope, const void* k
                                 int h_q, int g, int d_h, int d_rope, float scale, int dtype,
                                 void* out, float* lse, void* workspace, size_t workspace_bytes,
                                 lkv_stream_t stream) {
-  // Tied groups: the value stream reads the key rows.  The grouped kernel never writes K or V, and
-  // the second read of a tile follows the first within a few tiles, so it is served from L2.
-  return lkv_gqla_group_decode(q, q_rope, kv, kv_row_stride, kv, kv_row_stride, kpe, kpe_row_stride,
-                               cache_rows, cu_seqlens, batch, s_q, h_q, g, d_h, d_rope, scale, dtype,
-                               out, lse, workspace, workspace_bytes, stream);
+  // fp32 storage: the CUDA-core kernel of the GQA path with its value pointer on the tied rows
+  if (dtype == LKV_FP32)
+    return lkv_gqla_group_decode(q, q_rope, kv, kv_row_stride, kv, kv_row_stride, kpe, kpe_row_stride,
+                                 cache_rows, cu_seqlens, batch, s_q, h_q, g, d_h, d_rope, scale, dtype,
+                                 out, lse, workspace, workspace_bytes, stream);
+  lkv_status st = common_checks(q, q_rope, cu_seqlens, out, lse, batch, s_q, h_q, g, d_rope,
+                                cache_rows, dtype, scale);
+  if (st != LKV_OK) return st;
+  if (!kv || !kpe || d_h <= 0) return LKV_ERR_INVALID_ARG;
+  if (kv_row_stride < static_cast<int64_t>(g) * d_h || kpe_row_stride < d_rope) return LKV_ERR_INVALID_ARG;
+  const int hpg = h_q / g;
+  if (d_h != 128 || d_rope != 64 || hpg > 64 || s_q * hpg > 128) return LKV_ERR_UNSUPPORTED;
+  if (!al16(q) || !al16(q_rope) || !al16(kv) || !al16(kpe) || !al16(out) || (kv_row_stride * 2) % 16 ||
+      (kpe_row_stride * 2) % 16)
+    return LKV_ERR_INVALID_ARG;
+  DeviceState* d;
+  if ((st = device_state(&d)) != LKV_OK) return st;
+  const int P = plan_ranges(1, batch, s_q, g, d->num_sms);
+  const int R = s_q * hpg;
+  const WsLayout w = ws_layout(P, R, d_h);
+  if (!workspace || !al16(workspace) || workspace_bytes < w.total) return LKV_ERR_WORKSPACE;
+  // One ring of whole tiles: the tied state is read once into shared memory and serves as the
+  // key (with the RoPE key) and as the value.
+  TcLaunch L;
+  L.mode = MODE_GTA;
+  constexpr int TN = ModeCfg<MODE_GTA>::kTile;
+  if (!make_tmap_bf16(&L.map_a, kv, static_cast<uint64_t>(g) * d_h, cache_rows, kv_row_stride * 2, 64, TN) ||
+      !make_tmap_bf16(&L.map_r, kpe, d_rope, cache_rows, kpe_row_stride * 2, 64, TN))
+    return LKV_ERR_CUDA;
+  L.map_v = L.map_a;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  TcParams& p = L.p;
+  p.q_nope = static_cast<const __nv_bfloat16*>(q);
+  p.q_rope = static_cast<const __nv_bfloat16*>(q_rope);
+  p.dq = d_h;
+  p.cu = cu_seqlens;
+  p.B = batch;
+  p.s_q = s_q;
+  p.h_q = h_q;
+  p.G = g;
+  p.hpg = hpg;
+  p.R = R;
+  p.sl2 = scale * 1.4426950408889634f;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.dv_total = d_h;
+  p.seg_info = reinterpret_cast<int*>(ws + w.seg);
+  p.part_lse = reinterpret_cast<float*>(ws + w.lse);
+  p.part_o = reinterpret_cast<float*>(ws + w.o);
+  p.rmax = R;
+  p.P = P;
+  p.err = d->err;
+  p.wait_limit_ns = wait_limit_ns();
+  L.units_per_req = g;
+  L.per_query_units = 0;
+  return run_tc(L, *d, reinterpret_cast<cudaStream_t>(stream));
 }
 
 lkv_status lkv_gla_group_decode(const void* q, const void* q_rope, const void* clat,

@@ -61,7 +61,8 @@ constexpr int kMsgStride = 17 * 1024;
 constexpr int kMsgSlots = 3;
 constexpr int kTmemCols = 512;
 
-enum DecodeMode { MODE_MLA = 0, MODE_GQLA = 1, MODE_GLA = 2 };
+// MODE_GTA: grouped-tied attention, the GQLA shapes with K_j = V_j (one tied state per group).
+enum DecodeMode { MODE_MLA = 0, MODE_GQLA = 1, MODE_GLA = 2, MODE_GTA = 3 };
 
 // Wait sites (added to LKV_SITE_WAIT_BASE in the error word).
 enum WaitSite {
@@ -91,26 +92,30 @@ struct TcParams {
 template <int kMode>
 struct ModeCfg {
   static constexpr bool kPair = (kMode == MODE_MLA);
+  static constexpr bool kHead128 = (kMode == MODE_GQLA || kMode == MODE_GTA);  // d_h = 128 groups
   // Keys per tile.  GQLA runs 128-key tiles so that every QK UMMA is N = 128 (one issuing
   // thread then keeps the tensor pipe at full rate); MLA and GLA keep 64-key tiles because a
   // 128-column S tile would not fit next to their 256-column O accumulator and resident Q.
-  static constexpr int kTile = (kMode == MODE_GQLA) ? 128 : 64;
+  static constexpr int kTile = kHead128 ? 128 : 64;
   static constexpr int kBoxBytes = kTile * 128;                 // one TMA box: kTile rows x 64 bf16
   // GQLA keeps K (+ k_rope) and V in separate rings: a K slot is refilled as soon as its QK
-  // is done, while V waits for its PV.  Where K = V (MLA, GLA) one ring holds the tile.
+  // is done, while V waits for its PV.  Where K = V (MLA, GLA, GTA) one ring holds the tile.
   static constexpr bool kSplitKV = (kMode == MODE_GQLA);
+  static constexpr int kKBoxes = kHead128 ? 2 : 4;  // 64-column boxes of the non-RoPE key per stage
   // MLA: each CTA of the pair contracts its 256 latent columns and one 32-column half of the
   // RoPE key (a 64-byte swizzled box); the other modes take the whole 64-column RoPE key.
   static constexpr int kRopeBoxBytes = kPair ? kTile * 64 : kBoxBytes;
-  static constexpr int kStageBytes = (kSplitKV ? 2 : 4) * kBoxBytes + kRopeBoxBytes;  // K ring (or whole tile)
+  static constexpr int kStageBytes = kKBoxes * kBoxBytes + kRopeBoxBytes;  // K ring (or whole tile)
   static constexpr int kVStageBytes = 2 * kBoxBytes;                  // V ring (GQLA)
-  static constexpr int kDV = (kMode == MODE_GQLA) ? 128 : 256;  // value columns per CTA
-  static constexpr int kStages = (kMode == MODE_GQLA) ? 2 : (kPair ? 4 : 5);
+  static constexpr int kDV = kHead128 ? 128 : 256;  // value columns per CTA
+  // GTA holds a stage from its load to its PV (K = V), so it gets the ring depth that GQLA
+  // splits between its K ring (2) and V ring (3)
+  static constexpr int kStages = (kMode == MODE_GQLA) ? 2 : (kMode == MODE_GTA ? 4 : (kPair ? 4 : 5));
   // L2 prefetch distance of the producer in tiles (0: off)
   static constexpr int kPrefetch = kPair ? kStages + 1 : 0;
   static constexpr int kVStages = kSplitKV ? 3 : 1;
-  static constexpr int kNope = (kMode == MODE_GQLA) ? 2 : 4;    // non-RoPE Q boxes (in TMEM)
-  static constexpr int kRopeBox = (kMode == MODE_GQLA) ? 2 : 4; // stage box holding k_rope
+  static constexpr int kNope = kHead128 ? 2 : 4;    // non-RoPE Q boxes (in TMEM)
+  static constexpr int kRopeBox = kKBoxes;          // stage box holding k_rope
   static constexpr int kVBox0 = 0;                              // first V box (V ring or stage)
   static constexpr int kNV = kDV / 64;
   static constexpr int kPCols = kTile / 2;                      // bf16 P per buffer
@@ -127,10 +132,13 @@ struct ModeCfg {
 static_assert(ModeCfg<MODE_MLA>::Q0 + 32 * ModeCfg<MODE_MLA>::kNope <= kTmemCols, "TMEM budget");
 static_assert(ModeCfg<MODE_GLA>::Q0 + 32 * ModeCfg<MODE_GLA>::kNope <= kTmemCols, "TMEM budget");
 static_assert(ModeCfg<MODE_GQLA>::Q0 + 32 * ModeCfg<MODE_GQLA>::kNope <= kTmemCols, "TMEM budget");
+static_assert(ModeCfg<MODE_GTA>::Q0 + 32 * ModeCfg<MODE_GTA>::kNope <= kTmemCols, "TMEM budget");
 static_assert(ModeCfg<MODE_MLA>::kTile == 64, "the score exchange rows hold 64 keys");
 static_assert(ModeCfg<MODE_MLA>::kSmemBytes <= 232448, "shared memory budget");
 static_assert(ModeCfg<MODE_GLA>::kSmemBytes <= 232448, "shared memory budget");
 static_assert(ModeCfg<MODE_GQLA>::kSmemBytes <= 232448, "shared memory budget");
+static_assert(ModeCfg<MODE_GTA>::kSmemBytes <= 232448, "shared memory budget");
+static_assert(ModeCfg<MODE_GTA>::kStageBytes == 3 * ModeCfg<MODE_GTA>::kBoxBytes, "GTA stage: tied state + RoPE key");
 
 // Advance a shared-memory descriptor by a byte offset (start-address field, 16-byte units).
 __device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
@@ -380,6 +388,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           tma_prefetch_l2_2d(&map_r, 0, prow);
           tma_prefetch_l2_2d(&map_v, c0, prow);
           tma_prefetch_l2_2d(&map_v, c0 + 64, prow);
+        } else if constexpr (kMode == MODE_GTA) {
+          const int c0 = 128 * psg.k;
+          tma_prefetch_l2_2d(&map_a, c0, prow);
+          tma_prefetch_l2_2d(&map_a, c0 + 64, prow);
+          tma_prefetch_l2_2d(&map_r, 0, prow);
         } else {
           const int c0 = 256 * psg.k;
           for (int bx = 0; bx < 4; ++bx) tma_prefetch_l2_2d(&map_a, c0 + 64 * bx, prow);
@@ -435,6 +448,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tma_load_2d(vdst, &map_v, vb, c0, row);
             tma_load_2d(vdst + kBoxBytes, &map_v, vb, c0 + 64, row);
             ++nv;
+          } else if constexpr (kMode == MODE_GTA) {
+            // the group's tied state (key without RoPE, and value) and the shared RoPE key
+            const int c0 = 128 * sg.k;
+            tma_load_2d(dst, &map_a, fb, c0, row);
+            tma_load_2d(dst + kBoxBytes, &map_a, fb, c0 + 64, row);
+            tma_load_2d(dst + 2 * kBoxBytes, &map_r, fb, 0, row);
           } else {
             const int c0 = 256 * sg.k;
             for (int bx = 0; bx < 4; ++bx) tma_load_2d(dst + bx * kBoxBytes, &map_a, fb, c0 + 64 * bx, row);
