@@ -46,11 +46,28 @@ __device__ __forceinline__ void note_error(int* err, int code) {
 
 __device__ __forceinline__ float clamp_e4m3(float y) { return fminf(fmaxf(y, -kE4m3Max), kE4m3Max); }
 
-// One warp per row: amax by a warp reduction, then 8 codes per lane and chunk.
-__global__ void __launch_bounds__(256) quantize_fp8_kernel(QuantArgs a) {
-  const long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  if (w >= a.n_rows) return;
+// Loads of one source row into registers: latent chunk lane + 32 k (8 bf16 each) and RoPE chunk
+// `lane` (16 bytes); chunks past the row are left zero.
+struct RowRegs {
+  uint4 lat[kMaxChunks];
+  uint4 rope;
+};
+
+__device__ __forceinline__ void load_row(const QuantArgs& a, long long w, int lane, RowRegs& v) {
+  const uint8_t* srow = a.src + w * a.src_rs;
+  const int nch = a.r / kChunkElems;
+#pragma unroll
+  for (int k = 0; k < kMaxChunks; ++k) {
+    const int c = lane + 32 * k;
+    v.lat[k] = c < nch ? *reinterpret_cast<const uint4*>(srow + 16 * c) : make_uint4(0u, 0u, 0u, 0u);
+  }
+  const int rope_chunks = a.d_rope * 2 / 16;
+  v.rope = lane < rope_chunks ? reinterpret_cast<const uint4*>(srow + 2 * static_cast<long long>(a.r))[lane]
+                              : make_uint4(0u, 0u, 0u, 0u);
+}
+
+// Quantise the row held in v (source row w) into its cache row.
+__device__ __forceinline__ void store_row(const QuantArgs& a, long long w, int lane, const RowRegs& v) {
   long long dst_row = w;
   if (a.cu) {
     const int b = static_cast<int>(w / a.s_q), i = static_cast<int>(w % a.s_q);
@@ -66,41 +83,33 @@ __global__ void __launch_bounds__(256) quantize_fp8_kernel(QuantArgs a) {
     if (lane == 0) note_error(a.err, LKV_SITE_BAD_ROW);
     return;
   }
-  const uint8_t* srow = a.src + w * a.src_rs;
   uint8_t* drow = a.dst + dst_row * a.dst_rs;
   const int nch = a.r / kChunkElems;
-
-  float x[kMaxChunks][kChunkElems];
-  float amax = 0.f;
+  float amax = 0.f;  // chunks past the row are zero and do not change it
 #pragma unroll
   for (int k = 0; k < kMaxChunks; ++k) {
-    const int c = lane + 32 * k;
-    if (c < nch) {
-      const uint4 v = *reinterpret_cast<const uint4*>(srow + 16 * c);
-      const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v);
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v.lat[k]);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float2 f = __bfloat1622float2(h[e]);
-        x[k][2 * e] = f.x;
-        x[k][2 * e + 1] = f.y;
-        amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
-      }
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = __bfloat1622float2(h[e]);
+      amax = fmaxf(amax, fmaxf(fabsf(f.x), fabsf(f.y)));
     }
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   const float scale = __fdiv_rn(amax, kE4m3Max);
-
 #pragma unroll
   for (int k = 0; k < kMaxChunks; ++k) {
     const int c = lane + 32 * k;
     if (c < nch) {
       uint32_t word[2] = {0u, 0u};
       if (scale > 0.f) {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&v.lat[k]);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const float y0 = clamp_e4m3(__fdiv_rn(x[k][2 * e], scale));
-          const float y1 = clamp_e4m3(__fdiv_rn(x[k][2 * e + 1], scale));
+          const float2 f = __bfloat1622float2(h[e]);
+          const float y0 = clamp_e4m3(__fdiv_rn(f.x, scale));
+          const float y1 = clamp_e4m3(__fdiv_rn(f.y, scale));
           // .x lands in the low byte: element 2e at the lower address
           const uint32_t pair = __nv_cvt_float2_to_fp8x2(make_float2(y0, y1), __NV_SATFINITE, __NV_E4M3);
           word[e >> 1] |= (pair & 0xffffu) << (16 * (e & 1));
@@ -111,9 +120,32 @@ __global__ void __launch_bounds__(256) quantize_fp8_kernel(QuantArgs a) {
   }
   if (lane == 0) *reinterpret_cast<uint4*>(drow + a.r) = make_uint4(__float_as_uint(scale), 0u, 0u, 0u);
   const int rope_chunks = a.d_rope * 2 / 16;
-  const uint4* rs = reinterpret_cast<const uint4*>(srow + 2 * static_cast<long long>(a.r));
   uint4* rd = reinterpret_cast<uint4*>(drow + a.r + 16);
-  for (int c = lane; c < rope_chunks; c += 32) rd[c] = rs[c];
+  if (lane < rope_chunks) rd[lane] = v.rope;
+  // RoPE keys wider than 32 chunks (d_rope > 256): the rest straight from the source row
+  const uint4* rs = reinterpret_cast<const uint4*>(a.src + w * a.src_rs + 2 * static_cast<long long>(a.r));
+  for (int c = 32 + lane; c < rope_chunks; c += 32) rd[c] = rs[c];
+}
+
+// Grid-stride over rows, one warp per row at a time: the next row's loads are issued before the
+// current row is quantised, so every warp keeps two rows of loads in flight.
+__global__ void __launch_bounds__(256, 3) quantize_fp8_kernel(QuantArgs a) {
+  const int lane = threadIdx.x & 31;
+  const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+  long long w = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  if (w >= a.n_rows) return;
+  RowRegs cur;
+  load_row(a, w, lane, cur);
+  while (true) {
+    const long long wn = w + n_warps;
+    const bool more = wn < a.n_rows;
+    RowRegs nxt;
+    if (more) load_row(a, wn, lane, nxt);
+    store_row(a, w, lane, cur);
+    if (!more) break;
+    cur = nxt;
+    w = wn;
+  }
 }
 
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -129,7 +161,14 @@ lkv_status launch(QuantArgs& a, lkv_stream_t stream) {
   const lkv_status st = lkv_internal_error_word(&err);
   if (st != LKV_OK) return st;
   a.err = err;
-  const unsigned blocks = static_cast<unsigned>((a.n_rows * 32 + 255) / 256);
+  // enough 8-warp blocks for every row, at most the 3 per SM that are resident at once (80
+  // registers a thread); the loop takes the rest
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      sms <= 0)
+    return LKV_ERR_CUDA;
+  const long long need = (a.n_rows + 7) / 8;
+  const unsigned blocks = static_cast<unsigned>(need < 3LL * sms ? need : 3LL * sms);
   quantize_fp8_kernel<<<blocks, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(a);
   const cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? LKV_OK : LKV_ERR_CUDA;
