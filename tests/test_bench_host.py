@@ -1,0 +1,58 @@
+"""bench.py on the CPU: the reference arm's JSON line, the CPU baseline, and the algorithmic
+bytes and FLOPs behind every roofline fraction (checked against the pinned accounting oracle)."""
+import argparse
+import os
+
+import numpy as np
+import pytest
+
+import bench
+import synth
+from oracle import accounting as acc
+
+
+def test_reference_line_keeps_the_contract(monkeypatch):
+    calls = []
+
+    def fake_baseline(w, budget):
+        calls.append(budget)
+        return {"value": 12.5, "unit": "tokens/s", "cores": 4, "kind": "oracle",
+                "sample": f"1 of {w.batch} requests of {w.name} (fp64 numpy oracle)", "seconds": 0.1}
+
+    monkeypatch.setattr(bench, "cpu_baseline", fake_baseline)
+    args = argparse.Namespace(steps=2, warmup=3, workload="mla_b64_l4096")
+    res = bench.bench_reference(args, 0, 1)
+    assert len(calls) == 5                                   # W untimed + K timed samples
+    assert res["impl"] == "reference" and res["metric"] == bench.METRIC
+    assert res["unit"] == "tokens/s" and res["higher_is_better"] is True and res["value"] == 12.5
+    assert res["steps"] == 2 and res["warmup"] == 3 and res["n_gpus"] == 1
+    assert res["config"]["workload"] == "mla_b64_l4096"
+    assert res["e2e"] == {"value": 12.5, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert res["cpu_baseline"]["kind"] == "oracle" and res["cpu_baseline"]["value"] == 12.5
+    assert res["ms_per_step"] == pytest.approx(1e3 * 64 / 12.5)
+    assert bench.bench_reference(args, 1, 2) is None          # only rank 0 runs it
+
+
+def test_cpu_baseline_runs_the_oracle_on_a_bounded_sample():
+    cb = bench.cpu_baseline(synth.workload("tiny_fp32_mla"), 0.2)
+    assert cb["kind"] == "oracle" and cb["unit"] == "tokens/s" and cb["value"] > 0
+    assert cb["cores"] == os.cpu_count()
+    assert "of 2 requests of tiny_fp32_mla" in cb["sample"]
+
+
+@pytest.mark.parametrize("name", ["mla_b64_l4096", "gqla_g8_sq2_l8192", "long_gla2", "gta_g8_sq2_l8192",
+                                  "gqa2_sq2_l8192"])
+def test_roofline_accounting_matches_the_pinned_oracle(name):
+    w = synth.workload(name)
+    lengths = np.full(w.batch, w.seqlen, dtype=np.int64)
+    cache_bytes, io_bytes, flops = bench.workload_accounting(w, lengths)
+    want_bytes = acc.step_bytes(w.kind, lengths, w.s_q, w.h_q, w.groups, w.d_k, w.d_v, w.d_rope)
+    assert cache_bytes + io_bytes == want_bytes
+    assert flops == acc.step_flops(lengths, w.s_q, w.h_q, w.d_k, w.d_v, w.d_rope)
+
+
+def test_source_hash_covers_only_the_decode_sources():
+    h = bench.kernel_source_hash()
+    assert len(h) == 16
+    assert "lkv_proj.cu" not in bench.DECODE_SOURCES and "lkv_fp8.cu" not in bench.DECODE_SOURCES
+    assert bench.kernel_source_hash() == h                   # deterministic
