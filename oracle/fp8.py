@@ -24,7 +24,7 @@ from __future__ import annotations
 import numpy as np
 
 __all__ = ["E4M3_MAX", "e4m3_decode", "e4m3_encode", "quantize_rows", "dequantize_rows",
-           "mla_absorbed_decode_fp8"]
+           "mla_absorbed_decode_fp8", "gta_group_decode_fp8"]
 
 E4M3_MAX = 448.0
 
@@ -100,3 +100,12 @@ def mla_absorbed_decode_fp8(q_nope_abs, q_rope, codes, scales, kpe, cu_seqlens, 
     from .attend import mla_absorbed_decode
     return mla_absorbed_decode(q_nope_abs, q_rope, dequantize_rows(codes, scales), kpe, cu_seqlens, scale,
                                requests=requests)
+
+
+def gta_group_decode_fp8(q, q_rope, codes, scales, kpe, g, cu_seqlens, scale, requests=None):
+    """GTA decode over FP8 rows: the tied states of the g groups are one latent-shaped row per token
+    (codes [T, g*d_h] with one scale per token), dequantised and read as K_j = V_j of group j; the
+    bf16 RoPE key kpe [T, d_R] is shared by all groups."""
+    from .attend import gta_group_decode
+    return gta_group_decode(q, q_rope, dequantize_rows(codes, scales), kpe, g, cu_seqlens, scale,
+                            requests=requests)

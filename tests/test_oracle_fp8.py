@@ -114,3 +114,30 @@ def test_fp8_decode_equals_decode_over_dequantised_latent():
     if sw[0] != sw[1]:
         o2, _ = fp8.mla_absorbed_decode_fp8(q, qr, codes, sw, kpe, cu, 0.3)
         assert np.abs(o2 - out).max() > 1e-6
+
+
+def test_gta_fp8_decode_equals_gta_decode_over_dequantised_states():
+    """Power-of-two scales keep the dequantised tied states exact in bf16: the FP8 GTA decode equals
+    the GTA decode over them; scales are per token across all groups of the row."""
+    rng = np.random.default_rng(3)
+    B, S, H, g, d, dr = 2, 2, 8, 4, 8, 4
+    cu = np.array([0, 6, 13])
+    T = 13
+    codes = rng.integers(0, 0x7E, size=(T, g * d), dtype=np.uint8) | (rng.integers(0, 2, size=(T, g * d), dtype=np.uint8) << 7)
+    scales = (2.0 ** rng.integers(-8, -2, size=T)).astype(np.float32)
+    tied = fp8.e4m3_decode(codes) * scales[:, None].astype(np.float64)
+    q = rng.standard_normal((B, S, H, d))
+    qr = rng.standard_normal((B, S, H, dr))
+    kpe = rng.standard_normal((T, dr))
+    out, lse = fp8.gta_group_decode_fp8(q, qr, codes, scales, kpe, g, cu, 0.35)
+    ref_out, ref_lse = oracle.gta_group_decode(q, qr, tied, kpe, g, cu, 0.35)
+    np.testing.assert_allclose(out, ref_out, atol=1e-12)
+    np.testing.assert_allclose(lse, ref_lse, atol=1e-12)
+    # one scale for the whole row: doubling a token's scale doubles its key and value in every group
+    s2 = scales.copy()
+    s2[7] *= 2
+    out2, _ = fp8.gta_group_decode_fp8(q, qr, codes, s2, kpe, g, cu, 0.35)
+    tied2 = tied.copy()
+    tied2[7] *= 2
+    ref2, _ = oracle.gta_group_decode(q, qr, tied2, kpe, g, cu, 0.35)
+    np.testing.assert_allclose(out2, ref2, atol=1e-12)
