@@ -107,3 +107,30 @@ def test_two_ranks_sum_to_the_full_projection():
         np.testing.assert_allclose(y, y_full, atol=1e-10)         # every rank holds the full sum
         np.testing.assert_allclose(out_local, out[:, :, h0:h1], atol=1e-12)
     assert res[0][3] == (0, 4) and res[1][3] == (4, 8)
+
+
+def test_step_checks_local_shapes_and_single_rank_needs_no_process_group():
+    sh = group_shard(4, 8, 2, 1)                      # groups 2..3, heads 4..7
+    calls = []
+
+    def dec(q, qr, k, v, kpe, cu, scale):
+        calls.append(q.shape)
+        return torch.ones((q.shape[0], q.shape[1], q.shape[2], 3), dtype=torch.float64), None
+
+    tp = GroupAxisTP(sh, decode_fn=dec, proj_fn=lambda o, w: o @ w, allreduce_fn=lambda y: y)
+    q = torch.zeros((2, 1, 8, 3), dtype=torch.float64)
+    k = torch.zeros((5, 4, 3), dtype=torch.float64)
+    with pytest.raises(ValueError):
+        tp.step(q, q, tp.local_cache(k), tp.local_cache(k), None, None, 1.0, torch.zeros((12, 2)))  # all 8 heads
+    with pytest.raises(ValueError):
+        tp.step(tp.local_query(q), tp.local_query(q), k, k, None, None, 1.0, torch.zeros((12, 2)))   # all 4 groups
+    with pytest.raises(ValueError):
+        tp.step(tp.local_query(q), tp.local_query(q), tp.local_cache(k), tp.local_cache(k), None, None, 1.0,
+                torch.zeros((11, 2), dtype=torch.float64))                                        # W_O rows
+    y, out, _ = tp.step(tp.local_query(q), tp.local_query(q), tp.local_cache(k), tp.local_cache(k), None, None, 1.0,
+                        torch.ones((12, 2), dtype=torch.float64))
+    assert calls[-1] == (2, 1, 4, 3) and y.shape == (2, 2) and torch.all(y == 12)
+    # one rank: the default reduction is the identity and needs no process group
+    one = GroupAxisTP(group_shard(4, 8, 1, 0), decode_fn=dec, proj_fn=lambda o, w: o @ w)
+    y1, _, _ = one.step(q, q, k, k, None, None, 1.0, torch.ones((24, 2), dtype=torch.float64))
+    assert torch.all(y1 == 24)
