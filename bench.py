@@ -102,12 +102,13 @@ def job_throughput(tokens_per_rank: int, ms_this_rank: float, world: int, device
 def workload_accounting(w, lengths):
     """Algorithmic bytes (cache rows once, q, out, lse) and FLOPs (visible query-key pairs)."""
     lengths = np.asarray(lengths, dtype=np.int64)
+    elem = 2 if w.dtype == "bf16" else 4
     if w.kind in ("mla", "gla", "gta"):
         row = w.groups * w.d_k + w.d_rope
     else:
         row = w.groups * (w.d_k + w.d_v) + w.d_rope
-    cache_bytes = int(lengths.sum()) * row * 2
-    io_bytes = w.batch * w.s_q * w.h_q * ((w.d_k + w.d_rope) * 2 + w.d_v * 2 + 4)
+    cache_bytes = int(lengths.sum()) * row * elem
+    io_bytes = w.batch * w.s_q * w.h_q * ((w.d_k + w.d_rope) * elem + w.d_v * elem + 4)
     vis = sum(int((lengths - w.s_q + i + 1).sum()) for i in range(w.s_q))
     flops = vis * 2 * w.h_q * (w.d_k + w.d_rope + w.d_v)
     return cache_bytes, io_bytes, flops
@@ -193,7 +194,7 @@ def bench_gpu(args, rank, world, local_rank):
     else:
         k, v, kpe = d["k"].to(dev), d["v"].to(dev), d["kpe"].to(dev)
         new_k, new_v, new_kpe = new["k"].to(dev), new["v"].to(dev), new["kpe"].to(dev)
-    out = torch.empty((B, S, w.h_q, w.d_v), dtype=torch.bfloat16, device=dev)
+    out = torch.empty((B, S, w.h_q, w.d_v), dtype=q.dtype, device=dev)
     lse = torch.empty((B, S, w.h_q), dtype=torch.float32, device=dev)
     nsm = torch.cuda.get_device_properties(dev).multi_processor_count
     if w.kind == "mla":
@@ -281,8 +282,9 @@ def bench_gpu(args, rank, world, local_rank):
     else:
         step_in = [(new["k"].pin_memory(), new_k), (new["v"].pin_memory(), new_v),
                    (new["kpe"].pin_memory(), new_kpe)]
-    h2d = q_h.numel() * 2 + qr_h.numel() * 2 + sum(h.numel() * h.element_size() for h, _ in step_in)
-    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+    h2d = (q_h.numel() * q_h.element_size() + qr_h.numel() * qr_h.element_size()
+           + sum(h.numel() * h.element_size() for h, _ in step_in))
+    d2h = out_h.numel() * out_h.element_size() + lse_h.numel() * lse_h.element_size()
     e2e_steps = max(3, min(args.steps, 200))
 
     def e2e_step():
@@ -385,7 +387,7 @@ def bench_gpu(args, rank, world, local_rank):
             "higher_is_better": True,
             "scaling": "weak",
             "vs_baseline": None,
-            "dtype": "bf16",
+            "dtype": w.dtype,
             "data": "synthetic (seeded Gaussian, shapes of the pages' MLA/GQLA decode workloads)",
             "config": {"workload": w.name, "kind": w.kind, "batch_per_gpu": B, "s_q": S, "h_q": w.h_q,
                        "groups": w.groups, "d_k": w.d_k, "d_v": w.d_v, "d_rope": w.d_rope,

@@ -125,6 +125,13 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
+def _same_dtype(ref: torch.Tensor, **named):
+    """The C ABI takes one storage type per call: every tensor given must have ref's dtype."""
+    for name, t in named.items():
+        if t is not None and t.dtype != ref.dtype:
+            raise TypeError(f"{name} is {t.dtype}, expected {ref.dtype}")
+
+
 def _row_stride(t: torch.Tensor) -> int:
     if t.dim() < 2 or t.stride(-1) != 1:
         raise ValueError("cache rows must have unit stride in the last dimension")
@@ -173,6 +180,7 @@ def mla_absorbed_decode(q_nope_abs, q_rope, ckv, kpe, cu_seqlens, scale, out=Non
     B, s_q, h_q, r_kv = q_nope_abs.shape
     d_r = q_rope.shape[-1]
     dev = q_nope_abs.device
+    _same_dtype(q_nope_abs, q_rope=q_rope, ckv=ckv, kpe=kpe, out=out)
     if out is None:
         out = torch.empty((B, s_q, h_q, r_kv), dtype=q_nope_abs.dtype, device=dev)
     if lse is None:
@@ -191,6 +199,7 @@ def mla_absorbed_decode(q_nope_abs, q_rope, ckv, kpe, cu_seqlens, scale, out=Non
 def gqla_group_decode(q, q_rope, k, v, kpe, cu_seqlens, scale, out=None, lse=None,
                       workspace=None, stream=None):
     """GQLA grouped decode.  q [B,s_q,h_q,d_h], k / v [rows,g,d_h], kpe [rows,d_R]."""
+    _same_dtype(q, q_rope=q_rope, k=k, v=v, kpe=kpe, out=out)
     B, s_q, h_q, d_h = q.shape
     g = k.shape[1]
     d_r = q_rope.shape[-1]
@@ -218,6 +227,7 @@ def gqla_group_decode_noalloc(q, q_rope, k, v, kpe, cu_seqlens, scale, out=None,
     per call.  The library keeps one fixed 8 MiB device scratch array per GPU instead; calls
     that overlap on the GPU race on it, and shapes needing more scratch raise LkvError
     (ERR_WORKSPACE).  `out` and `lse` are still caller-provided (allocated here if omitted)."""
+    _same_dtype(q, q_rope=q_rope, k=k, v=v, kpe=kpe, out=out)
     B, s_q, h_q, d_h = q.shape
     g = k.shape[1]
     d_r = q_rope.shape[-1]
@@ -240,6 +250,7 @@ def gta_group_decode(q, q_rope, kv, kpe, g, cu_seqlens, scale, out=None, lse=Non
                      workspace=None, stream=None):
     """GTA decode over tied groups.  q [B,s_q,h_q,d_h], kv [rows, g*d_h] (tied key/value state
     of each group, contiguous within a row), kpe [rows,d_R]."""
+    _same_dtype(q, q_rope=q_rope, kv=kv, kpe=kpe, out=out)
     B, s_q, h_q, d_h = q.shape
     d_r = q_rope.shape[-1]
     dev = q.device
@@ -262,6 +273,7 @@ def gta_group_decode(q, q_rope, kv, kpe, g, cu_seqlens, scale, out=None, lse=Non
 def gla_group_decode(q, q_rope, clat, kpe, n_lat, cu_seqlens, scale, out=None, lse=None,
                      workspace=None, stream=None):
     """GLA decode.  q [B,s_q,h_q,r_g], clat [rows, n_lat*r_g], kpe [rows,d_R]."""
+    _same_dtype(q, q_rope=q_rope, clat=clat, kpe=kpe, out=out)
     B, s_q, h_q, r_g = q.shape
     d_r = q_rope.shape[-1]
     dev = q.device
@@ -316,6 +328,8 @@ def fp8_cache_fields(cache, r: int, d_rope: int):
 def quantize_latent_fp8(rows, r: int, cache=None, stream=None):
     """Quantise bf16 rows [n, >= r + d_rope] (latent then RoPE key) into FP8 cache rows, row i to
     row i.  Returns the cache [n, row_bytes] uint8 (allocated if not given)."""
+    if rows.dtype != torch.bfloat16 or (cache is not None and cache.dtype != torch.uint8):
+        raise TypeError("quantize_latent_fp8 takes bf16 rows and a uint8 cache")
     n, width = rows.shape
     d_rope = width - r
     rb = fp8_cache_row_bytes(r, d_rope)
@@ -331,6 +345,8 @@ def quantize_latent_fp8(rows, r: int, cache=None, stream=None):
 def latent_cache_append_fp8(new_rows, cache, cu_seqlens, s_q, r: int, stream=None):
     """Quantise row b*s_q+i of the bf16 new_rows [B*s_q, r + d_rope] into FP8 cache row
     cu[b] + L_b - s_q + i of cache [rows, row_bytes] uint8."""
+    if new_rows.dtype != torch.bfloat16 or cache.dtype != torch.uint8:
+        raise TypeError("latent_cache_append_fp8 takes bf16 rows and a uint8 cache")
     n, width = new_rows.shape
     B = cu_seqlens.numel() - 1
     if n != B * s_q:
@@ -370,6 +386,7 @@ def selftest_wait_timeout(limit_ns: int, stream=None):
 def absorb_query(q, w_uk, out=None, stream=None):
     """q_abs[..., h, :] = w_uk[j(h)] @ q[..., h, :].  q [..., h_q, d_h], w_uk [G, r, d_h] (bf16,
     contiguous) -> [..., h_q, r] bf16."""
+    _same_dtype(q, w_uk=w_uk, out=out)
     G, r, d_h = w_uk.shape
     h_q = q.shape[-2]
     if q.shape[-1] != d_h:
@@ -386,6 +403,7 @@ def absorb_query(q, w_uk, out=None, stream=None):
 def unabsorb_output(o_lat, w_uv, out=None, stream=None):
     """out[..., h, :] = w_uv[j(h)]^T @ o_lat[..., h, :].  o_lat [..., h_q, r], w_uv [G, r, d_v]
     (bf16, contiguous) -> [..., h_q, d_v] bf16."""
+    _same_dtype(o_lat, w_uv=w_uv, out=out)
     G, r, d_v = w_uv.shape
     h_q = o_lat.shape[-2]
     if o_lat.shape[-1] != r:
@@ -402,6 +420,7 @@ def unabsorb_output(o_lat, w_uv, out=None, stream=None):
 def expand_latent(c, w, out=None, stream=None):
     """x[t, j, :] = c[t, :] @ w[j].  c [T, r] (unit inner stride; may be a column slice of the
     cache), w [G, r, d] contiguous (bf16) -> x [T, G, d] bf16."""
+    _same_dtype(c, w=w, out=out)
     G, r, d = w.shape
     T = c.shape[0]
     if c.shape[1] != r:

@@ -41,12 +41,13 @@ def test_cpu_baseline_runs_the_oracle_on_a_bounded_sample():
 
 
 @pytest.mark.parametrize("name", ["mla_b64_l4096", "gqla_g8_sq2_l8192", "long_gla2", "gta_g8_sq2_l8192",
-                                  "gqa2_sq2_l8192"])
+                                  "gqa2_sq2_l8192", "tiny_fp32_mla"])
 def test_roofline_accounting_matches_the_pinned_oracle(name):
     w = synth.workload(name)
     lengths = np.full(w.batch, w.seqlen, dtype=np.int64)
     cache_bytes, io_bytes, flops = bench.workload_accounting(w, lengths)
-    want_bytes = acc.step_bytes(w.kind, lengths, w.s_q, w.h_q, w.groups, w.d_k, w.d_v, w.d_rope)
+    elem = 2 if w.dtype == "bf16" else 4
+    want_bytes = acc.step_bytes(w.kind, lengths, w.s_q, w.h_q, w.groups, w.d_k, w.d_v, w.d_rope, elem_bytes=elem)
     assert cache_bytes + io_bytes == want_bytes
     assert flops == acc.step_flops(lengths, w.s_q, w.h_q, w.d_k, w.d_v, w.d_rope)
 
