@@ -6,9 +6,14 @@ One step = one whole decode step of the hot path on one batch: append the s_q ne
 of every request, then decode attention over the full cache (range planning, tensor-core
 split-KV kernel, split combine).  Inputs are seeded synthetic tensors resident in HBM before
 the timed region; the cache (0.30 GB for the default workload) is larger than the 126 MB L2,
-so no flush is done between steps.  Timing: CUDA events on the launching stream over exactly K
-steps, bracketed by a barrier and a device synchronise, max over ranks.  Rank 0 prints one
-JSON line.
+so the timed steps run back to back with no flush.  Timing: CUDA events on the launching stream
+over exactly K steps, bracketed by a barrier and a device synchronise, max over ranks.  Rank 0
+prints one JSON line.
+
+The same line carries, under "workloads", every other decode workload of the build timed on its
+own (the decode call alone, CUDA events, a 256 MB L2-flushing write before each call and outside
+its events), with its roofline fraction and a bounded sample of the CPU oracle on the same
+inputs; and, for the headline workload, the decode call timed the same flushed way.
 
 `--impl reference` times the fp64 CPU oracle (the correctness reference) on the host cores,
 on a bounded sample of the same workload; under torchrun only rank 0 runs it.
@@ -112,6 +117,174 @@ def workload_accounting(w, lengths):
     vis = sum(int((lengths - w.s_q + i + 1).sum()) for i in range(w.s_q))
     flops = vis * 2 * w.h_q * (w.d_k + w.d_rope + w.d_v)
     return cache_bytes, io_bytes, flops
+
+
+# The other workloads timed beside the headline: the five configurations' remaining shapes and the
+# tied / narrow-group variants.
+SIDE_WORKLOADS = ("tiny_fp32_mla", "gqla_g8_sq2_l8192", "varlen_mla_sq1", "varlen_mla_sq2", "long_gla2",
+                  "long_mla", "long_gqla_g8", "gta_g8_sq2_l8192", "gqa2_sq2_l8192")
+L2_FLUSH_BYTES = 256 << 20   # twice the 126 MB L2
+
+
+def roofline_entry(w, lengths, dec_ms, peaks, how):
+    """Algorithmic bytes / FLOPs of one decode call and the fraction of the roofline time
+    max(bytes / HBM peak, FLOPs / tensor peak) that a call of dec_ms milliseconds achieves."""
+    cache_bytes, io_bytes, flops = workload_accounting(w, lengths)
+    alg_bytes = cache_bytes + io_bytes
+    dec_s = dec_ms * 1e-3
+    gbs = alg_bytes / dec_s / 1e9
+    tfl = flops / dec_s / 1e12
+    t_hbm = alg_bytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_hbm >= t_tc else "tensor"
+    achieved = gbs if bound == "hbm" else tfl
+    peak = peaks["hbm_gbs"] if bound == "hbm" else peaks["bf16_tflops"]
+    nominal = max(alg_bytes / (NOMINAL_PEAKS["hbm_gbs"] * 1e9), flops / (NOMINAL_PEAKS["bf16_tflops"] * 1e12)) / dec_s
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
+            "frac": achieved / peak, "traffic": measured_traffic(w.name),
+            "peak_source": f"{how} (MEASURED_PEAKS.json burst)", "nominal": {"frac": nominal},
+            "roofline_ms": max(t_hbm, t_tc) * 1e3, "algorithmic_bytes": alg_bytes, "algorithmic_flops": flops,
+            "kv_gbs": gbs, "tflops": tfl}
+
+
+def device_inputs(w, dev):
+    """Seeded synthetic inputs of workload w drawn on the device (torch's generator seeded with the
+    workload's seed): the shapes, layout and value distribution of synth.make_inputs, without the
+    host draw and copy of multi-GB caches.  Lengths come from synth (the same draw)."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(1000 + w.seed)
+    if w.seqlen is None:
+        lengths = synth.draw_lengths(np.random.default_rng(w.seed), w.batch, w.len_lo, w.len_hi)
+    else:
+        lengths = np.full(w.batch, w.seqlen, dtype=np.int64)
+    cu = synth.prefix_offsets(lengths)
+    T = int(cu[-1])
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def randn(*shape, std):
+        return torch.randn(*shape, generator=g, device=dev, dtype=dt).mul_(std)
+
+    qs = w.input_std if w.q_std is None else w.q_std
+    d = {"workload": w, "lengths": lengths, "cu_seqlens": torch.from_numpy(cu.astype(np.int32)).to(dev),
+         "q": randn(w.batch, w.s_q, w.h_q, w.d_k, std=qs), "q_rope": randn(w.batch, w.s_q, w.h_q, w.d_rope, std=qs)}
+    if w.kind == "gqla":
+        d["k"] = randn(T, w.groups, w.d_k, std=w.input_std)
+        d["v"] = randn(T, w.groups, w.d_v, std=w.input_std)
+        d["kpe"] = randn(T, w.d_rope, std=w.input_std)
+    else:
+        d["cache"] = randn(T, w.groups * w.d_k + w.d_rope, std=w.input_std)
+    return d
+
+
+def make_decoder(lkv, w, d, nsm):
+    """decode(q, q_rope, out, lse) for workload w over the cache tensors in d, workspace allocated here."""
+    dev = d["q"].device
+    B, S = w.batch, w.s_q
+    if w.kind == "mla":
+        ws = torch.empty(lkv.mla_decode_workspace_size(B, S, w.h_q, w.d_k, nsm), dtype=torch.uint8, device=dev)
+    else:
+        kind = {"gqla": lkv.KIND_GQLA, "gla": lkv.KIND_GLA, "gta": lkv.KIND_GTA}[w.kind]
+        ws = torch.empty(lkv.group_decode_workspace_size(kind, B, S, w.h_q, w.groups, w.d_v, nsm),
+                         dtype=torch.uint8, device=dev)
+    cu = d["cu_seqlens"]
+    if w.kind == "gqla":
+        k, v, kpe = d["k"], d["v"], d["kpe"]
+    else:
+        width = w.groups * w.d_k
+        lat, kpe = d["cache"][:, :width], d["cache"][:, width:]
+
+    def decode(qq, qqr, o, l):
+        if w.kind == "mla":
+            lkv.mla_absorbed_decode(qq, qqr, lat, kpe, cu, w.scale, out=o, lse=l, workspace=ws)
+        elif w.kind == "gqla":
+            lkv.gqla_group_decode(qq, qqr, k, v, kpe, cu, w.scale, out=o, lse=l, workspace=ws)
+        elif w.kind == "gta":
+            lkv.gta_group_decode(qq, qqr, lat, kpe, w.groups, cu, w.scale, out=o, lse=l, workspace=ws)
+        else:
+            lkv.gla_group_decode(qq, qqr, lat, kpe, w.groups, cu, w.scale, out=o, lse=l, workspace=ws)
+    return decode
+
+
+def time_flushed(decode, args_, stream, flush, iters: int):
+    """Per-call decode times (ms): each call preceded by an L2-flushing write outside its events."""
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record(stream)
+        decode(*args_)
+        e1.record(stream)
+    torch.cuda.synchronize()
+    return [e0.elapsed_time(e1) for e0, e1 in ev]
+
+
+def cpu_baseline_device(w, d, budget_s: float):
+    """The oracle as it stands on the host cores, on a bounded sample (whole requests, shortest
+    first) of the device-drawn inputs d, copied to the host request by request."""
+    import oracle
+    cu = d["cu_seqlens"].cpu().numpy().astype(np.int64)
+    order = [int(b) for b in np.argsort(d["lengths"], kind="stable")]
+    t0 = time.perf_counter()
+    done = keys = 0
+    for b in order:
+        c0, c1 = int(cu[b]), int(cu[b + 1])
+        one = np.array([0, c1 - c0], dtype=np.int64)
+        q, qr = d["q"][b:b + 1].cpu(), d["q_rope"][b:b + 1].cpu()
+        if w.kind == "gqla":
+            oracle.gqla_group_decode(q, qr, d["k"][c0:c1].cpu(), d["v"][c0:c1].cpu(), d["kpe"][c0:c1].cpu(), one,
+                                     w.scale)
+        else:
+            c = d["cache"][c0:c1].cpu()
+            width = w.groups * w.d_k
+            if w.kind == "mla":
+                oracle.mla_absorbed_decode(q, qr, c[:, :width], c[:, width:], one, w.scale)
+            elif w.kind == "gta":
+                oracle.gta_group_decode(q, qr, c[:, :width], c[:, width:], w.groups, one, w.scale)
+            else:
+                oracle.gla_group_decode(q, qr, c[:, :width], c[:, width:], w.groups, one, w.scale)
+        done += 1
+        keys += c1 - c0
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done * w.s_q / dt, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{done} of {w.batch} requests ({keys} cached tokens) of {w.name}, shortest first "
+                      "(fp64 numpy oracle)", "seconds": dt}
+
+
+def bench_side_workloads(lkv, dev, names, iters: int, cpu_budget: float):
+    """Decode time, roofline fraction and a bounded CPU-oracle sample for each workload in names."""
+    peaks, how = load_peaks()
+    nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    res = {}
+    for name in names:
+        w = synth.workload(name)
+        d = device_inputs(w, dev)
+        out = torch.empty((w.batch, w.s_q, w.h_q, w.d_v), dtype=d["q"].dtype, device=dev)
+        lse = torch.empty((w.batch, w.s_q, w.h_q), dtype=torch.float32, device=dev)
+        decode = make_decoder(lkv, w, d, nsm)
+        for _ in range(3):
+            decode(d["q"], d["q_rope"], out, lse)
+        if lkv.check_device() != 0:
+            raise RuntimeError(f"device error during warm-up of {name}")
+        ms = time_flushed(decode, (d["q"], d["q_rope"], out, lse), stream, flush, iters)
+        if lkv.check_device() != 0:
+            raise RuntimeError(f"device error while timing {name}")
+        med = float(np.median(ms))
+        entry = {"decode_ms": med, "decode_ms_min": float(min(ms)), "decode_ms_max": float(max(ms)),
+                 "calls": iters, "tokens_per_s": w.batch * w.s_q / (med * 1e-3), "dtype": w.dtype,
+                 "shape": {"kind": w.kind, "batch": w.batch, "s_q": w.s_q, "h_q": w.h_q, "groups": w.groups,
+                           "d_k": w.d_k, "d_v": w.d_v, "d_rope": w.d_rope, "seqlen": w.seqlen,
+                           "total_cached_tokens": int(d["lengths"].sum())},
+                 "roofline": roofline_entry(w, d["lengths"], med, peaks, how),
+                 "cpu_baseline": cpu_baseline_device(w, d, cpu_budget)}
+        if w.dtype == "fp32":
+            entry["roofline"]["note"] = "latency-bound CUDA-core fp32 path (0.18 MB); not gated on the roofline"
+        res[name] = entry
+        del d, out, lse, decode
+        torch.cuda.empty_cache()
+    return res
 
 
 class ClockSampler:
@@ -361,6 +534,19 @@ def bench_gpu(args, rank, world, local_rank):
     e2e_ms = time_e2e(e2e_step_pipelined, tail_stream=s_out)
     torch.cuda.synchronize(dev)
 
+    # The headline decode call once more, each call after an L2-flushing write (outside its events),
+    # then every other workload the same way (single process only: they hold up to 4.4 GB each).
+    flushed_ms = None
+    side = None
+    if world == 1 and args.side_iters > 0:
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        flushed_ms = time_flushed(decode, (q, qr, out, lse), stream, flush, args.side_iters)
+        del flush
+        if lkv.check_device() != 0:
+            raise RuntimeError("device error while timing the flushed decode calls")
+        names = [n for n in SIDE_WORKLOADS if n != w.name]
+        side = bench_side_workloads(lkv, dev, names, args.side_iters, args.side_cpu_budget)
+
     tokens = B * S * world
     cache_bytes, io_bytes, flops = workload_accounting(w, lengths)
     res = None
@@ -395,6 +581,13 @@ def bench_gpu(args, rank, world, local_rank):
                        "l2": "inputs larger than L2 (cache >> 126 MB); no flush",
                        "parallelism": f"dp{world}"},
             "decode_kernel_ms": dec_avg_ms,
+            "decode_ms_per_step": {"min": float(np.min(dec_ms)), "median": float(np.median(dec_ms)),
+                                   "max": float(np.max(dec_ms))},
+            "decode_ms_l2_flushed": (None if flushed_ms is None else
+                                     {"median": float(np.median(flushed_ms)), "min": float(np.min(flushed_ms)),
+                                      "calls": len(flushed_ms),
+                                      "frac": roofline_entry(w, lengths, float(np.median(flushed_ms)),
+                                                             *load_peaks())["frac"]}),
             "kv_gbs": gbs,
             "tflops": tfl,
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak,
@@ -414,6 +607,7 @@ def bench_gpu(args, rank, world, local_rank):
                     "serial": {"value": tokens / (e2e_serial_ms * 1e-3), "ms_per_step": e2e_serial_ms}},
             "gpu_launches": launches_per_step * args.steps,
             "clocks": sampler.summary() if sampler else None,
+            "workloads": side,
         }
     if world > 1:
         import torch.distributed as dist
@@ -490,6 +684,10 @@ def main():
     ap.add_argument("--workload", default="mla_b64_l4096", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="lkv", choices=["lkv", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--side-iters", type=int, default=10,
+                    help="calls per workload for the flushed per-workload timings (0: skip them)")
+    ap.add_argument("--side-cpu-budget", type=float, default=1.5,
+                    help="seconds of CPU-oracle work per side workload")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

@@ -35,6 +35,10 @@
  *   - scale must be finite and > 0 (the pages' softmax scale is 1/sqrt of the score width);
  *     a positive scale keeps the order of the raw scores, which the kernels rely on.
  *   - Row strides are in elements and must keep every row 16-byte aligned.
+ *   - The first call on a device sets that device up for the rest of the process (SM count,
+ *     kernel attributes, device addresses of the library's own device variables).  After a
+ *     cudaDeviceReset of a device the library must not be called on that device again in the
+ *     same process: the kept addresses would point into the released context.
  */
 #ifndef LKV_H
 #define LKV_H
@@ -161,8 +165,10 @@ lkv_status lkv_gla_group_decode(const void* q, const void* q_rope, const void* c
  *          [cache_rows, d_rope] row stride kpe_row_stride (kv and kpe may interleave in one
  *          [cache_rows, g*d_h + d_rope] array)
  *   out    [batch, s_q, h_q, d_h]; lse [batch, s_q, h_q]
- * Runs the grouped kernel of lkv_gqla_group_decode with its value stream reading the key rows:
- * same limits, same workspace (lkv_group_decode_workspace_size with kind 1 or 3).
+ * Runs the grouped tensor-core kernel in its tied mode: each tile of tied states (with the RoPE
+ * key) is read once into shared memory and serves as the key operand of QK and the value operand
+ * of PV.  Same limits as lkv_gqla_group_decode, same workspace (lkv_group_decode_workspace_size
+ * with kind 1 or 3).
  */
 lkv_status lkv_gta_group_decode(const void* q, const void* q_rope, const void* kv,
                                 int64_t kv_row_stride, const void* kpe, int64_t kpe_row_stride,
@@ -284,6 +290,15 @@ lkv_status lkv_merge_partials(const float* o_parts, const float* lse_parts, int 
 lkv_status lkv_check_device(int32_t* code_out, int clear);
 
 /*
+ * The same check ordered on one stream only: waits for the work queued on `stream` so far
+ * (cudaStreamSynchronize, not a device-wide synchronise, so other streams keep running), then
+ * reads the device error word with a copy on that stream.  The word is shared by every stream of
+ * the device, so it also shows failures recorded by other streams' finished kernels.
+ * clear != 0 resets it to 0 on that stream afterwards.  code_out may be NULL.
+ */
+lkv_status lkv_check_stream(lkv_stream_t stream, int32_t* code_out, int clear);
+
+/*
  * Failure-detection self test: launches one CTA that waits on an mbarrier no thread
  * arrives at, with the given limit.  The wait gives up, records LKV_SITE_SELFTEST in the
  * device error word and the kernel returns; the context stays usable.
@@ -320,6 +335,10 @@ lkv_status lkv_expand_latent(const void* c, int64_t c_row_stride, const void* w,
 #define LKV_SITE_SELFTEST 1
 #define LKV_SITE_BAD_LENGTH 2     /* a request with L_b < s_q (append or decode)      */
 #define LKV_SITE_BAD_ROW 3        /* a cache row past cache_rows                      */
+/* MLA absorbed decode (bf16): the two halves of a row's scores lie too far apart for the pair's
+ * score exchange -- a tile's best key more than 103 log2 units below the sum of the two halves'
+ * partial maxima, or a partial tile max beyond 16384 log2 units.  Outputs may be inexact. */
+#define LKV_SITE_SCORE_RANGE 4
 #define LKV_SITE_WAIT_BASE 100    /* + kernel-specific wait site: a bounded wait gave up */
 
 #ifdef __cplusplus

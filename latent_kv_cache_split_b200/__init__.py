@@ -32,7 +32,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE = range(6)
 BF16, FP32 = 0, 1
 KIND_MLA, KIND_GQLA, KIND_GLA, KIND_GTA = 0, 1, 2, 3
-SITE_SELFTEST, SITE_BAD_LENGTH, SITE_BAD_ROW, SITE_WAIT_BASE = 1, 2, 3, 100   # device error word
+SITE_SELFTEST, SITE_BAD_LENGTH, SITE_BAD_ROW, SITE_SCORE_RANGE, SITE_WAIT_BASE = 1, 2, 3, 4, 100  # device error word
 
 _vp, _i64, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 
@@ -67,6 +67,7 @@ _append = _sig("lkv_latent_cache_append", _i32, _vp, _i64, _vp, _i64, _i64, _i64
                _i32, _i32, _vp)
 _merge = _sig("lkv_merge_partials", _i32, _vp, _vp, _i32, _i64, _i32, _i32, _vp, _vp, _vp)
 _check = _sig("lkv_check_device", _i32, ctypes.POINTER(ctypes.c_int32), _i32)
+_check_stream = _sig("lkv_check_stream", _i32, _vp, ctypes.POINTER(ctypes.c_int32), _i32)
 _selftest = _sig("lkv_selftest_wait_timeout", _i32, ctypes.c_uint64, _vp)
 _segments = _sig("lkv_plan_segments", _i32, _i32, _vp, _i32, _i32, _i32, _i32, _vp, _i32)
 _absorb = _sig("lkv_absorb_query", _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _vp)
@@ -80,7 +81,8 @@ EXPORTED = ["lkv_version", "lkv_status_string", "lkv_plan_ranges", "lkv_mla_deco
             "lkv_check_device", "lkv_selftest_wait_timeout", "lkv_plan_segments",
             "lkv_gqla_group_decode_noalloc", "lkv_absorb_query", "lkv_unabsorb_output",
             "lkv_expand_latent", "lkv_gta_group_decode", "lkv_fp8_cache_row_bytes",
-            "lkv_quantize_latent_fp8", "lkv_latent_cache_append_fp8", "lkv_output_projection"]
+            "lkv_quantize_latent_fp8", "lkv_latent_cache_append_fp8", "lkv_output_projection",
+            "lkv_check_stream"]
 
 
 class LkvError(RuntimeError):
@@ -376,6 +378,16 @@ def check_device(clear: bool = True) -> int:
     st = _check(ctypes.byref(code), 1 if clear else 0)
     if st not in (OK, ERR_DEVICE):
         raise LkvError(st, "lkv_check_device")
+    return code.value
+
+
+def check_stream(stream=None, clear: bool = True) -> int:
+    """Wait for the work queued on `stream` (not the whole device) and return the device error
+    word (0 = no failure recorded)."""
+    code = ctypes.c_int32(0)
+    st = _check_stream(_stream(stream), ctypes.byref(code), 1 if clear else 0)
+    if st not in (OK, ERR_DEVICE):
+        raise LkvError(st, "lkv_check_stream")
     return code.value
 
 

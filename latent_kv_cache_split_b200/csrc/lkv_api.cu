@@ -689,6 +689,26 @@ lkv_status lkv_check_device(int32_t* code_out, int clear) {
   return v ? LKV_ERR_DEVICE : LKV_OK;
 }
 
+lkv_status lkv_check_stream(lkv_stream_t stream, int32_t* code_out, int clear) {
+  DeviceState* d;
+  lkv_status st = device_state(&d);
+  if (st != LKV_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int v = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return LKV_ERR_CUDA;
+  if (cudaMemcpyFromSymbolAsync(&v, g_lkv_error_word, sizeof(int), 0, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess)
+    return LKV_ERR_CUDA;
+  if (code_out) *code_out = v;
+  if (clear && v) {
+    static const int z = 0;
+    if (cudaMemcpyToSymbolAsync(g_lkv_error_word, &z, sizeof(int), 0, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return LKV_ERR_CUDA;
+  }
+  return v ? LKV_ERR_DEVICE : LKV_OK;
+}
+
 lkv_status lkv_selftest_wait_timeout(uint64_t limit_ns, lkv_stream_t stream) {
   if (limit_ns == 0 || limit_ns > 10000000000ull) return LKV_ERR_INVALID_ARG;
   DeviceState* d;

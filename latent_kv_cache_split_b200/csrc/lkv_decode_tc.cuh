@@ -14,8 +14,9 @@
 //   warps 4-11  softmax / epilogue.  Grouped modes: warp 4 + q + 4h owns TMEM lane quadrant q
 //               and key-column half h of each tile; the two halves of a row agree on the
 //               running max through a bounded shared-memory exchange.  MLA: warps 4-7 (score
-//               warps) turn S into exp2 factors and stage them, warps 8-11 (combine warps) form
-//               P, rescale O and write the output, one tile behind the score warps.
+//               warps) encode S as score codes and stage them, warps 8-11 (combine warps) add
+//               both CTAs' codes, form P, rescale O and write the output, one tile behind the
+//               score warps.
 //
 // TMEM columns: O [0, DV) | S [DV, DV+T) | P0, P1 [DV+T, DV+2T) | Q [DV+2T, ...) for T keys/tile.
 // P is double buffered so the softmax of tile n+1 never waits for the PV of tile n.
@@ -24,11 +25,11 @@
 // 128 x 512 fp32 output accumulator alone fills a whole TMEM, so a CTA pair splits it:
 // rank 0 owns value columns 0..255 and contracts latent columns 0..255 plus RoPE columns 0..31,
 // rank 1 owns value columns 256..511 and contracts latent 256..511 plus RoPE 32..63.  Each CTA
-// turns its partial scores into fp16 factors E = exp2(partial - t) (t its partial row max) and
-// sends them to the peer through distributed shared memory; both CTAs form
-// P = E_own * E_peer * 2^(t_own + t_peer - m) (the same P on both sides) and accumulate their
-// own half of O.  Each CTA streams only the cache columns it needs, so the pair reads every
-// cache byte once.
+// encodes its partial scores as 16-bit offsets below a per-row reference (its partial tile max)
+// and sends them to the peer through distributed shared memory; both CTAs add the two codes of
+// every key (an exact integer sum, so the full score is known to one code step), form the same
+// P = 2^(score - m) and accumulate their own half of O.  Each CTA streams only the cache columns
+// it needs, so the pair reads every cache byte once.
 //
 // GQLA (g groups of expanded K_j, V_j) and GLA (latent groups, K_j = V_j) run one unit per
 // CTA: rows = heads of the group x new tokens (<= 128), padded to the M = 128 UMMA shape.
@@ -44,22 +45,59 @@
 
 namespace lkv {
 
-// Warps: 0 TMA producer, 1 UMMA issuer, 2-3 MLA message sender, 4-11 softmax.  Softmax warp
-// 4 + q + 4 h owns TMEM lane quadrant q (rows 32q..32q+31) and key-column half h of each tile.
+// Warps: 0 TMA producer, 1 QK issuer, 2 PV issuer, 3 MLA message sender, 4-11 softmax (roles in
+// the file header).
 constexpr int kTcThreads = 384;
-// MLA pair message per tile: 128 rows x 64 fp16 of exp2(partial score - partial tile max)
-// (values in (0, 1], so fp16 keeps 11 significant bits where bf16 would keep 8), then the 128
-// partial tile maxima (fp32).
-// One score message: 128 rows x 64 fp16 factors, then the 128 partial row maxima (fp32).
+// One MLA score message: 128 rows x 64 16-bit score codes, then the 128 rows' references (fp32).
 constexpr int kMsgBytes = 128 * 128 + 128 * 4;
 // Slot stride in shared memory: 1024-byte aligned, because the combine warps overwrite the
-// peer's factors in a slot with P (same 128-byte-swizzled rows), the A operand of that tile's PV.
+// peer's codes in a slot with P (same 128-byte-swizzled rows), the A operand of that tile's PV.
 constexpr int kMsgStride = 17 * 1024;
 // Incoming score messages in flight per CTA of the MLA pair.  A CTA sends message m only after
 // it has read the peer's message m-1, which the peer sent after reading message m-2 (and so
 // m-3) from this CTA, so with 3 slots the slot of message m is always free when it is written.
 constexpr int kMsgSlots = 3;
 constexpr int kTmemCols = 512;
+
+// MLA pair score exchange.  A CTA holds only the partial score of each key over its half of the
+// 576 contracted columns; the full score is the sum of both halves.  Each half is sent as a 16-bit
+// code of (reference - partial score) in steps of 2^(e-10) log2 units, the reference being the
+// row's partial tile max.  The step exponent e (0..5) is the smallest whose 65535 steps cover the
+// row's partial scores in this tile; it travels in the low 3 bits of the fp32 reference, and the
+// codes are taken against that very reference.  The receiving side adds the two halves, so the
+// full score of every key is known to within half a step of each half.
+constexpr int kStepBits = 3;                   // low mantissa bits of the reference carrying e
+constexpr float kOffsetMagic = 8388608.f;      // 2^23: an fp32 sum there rounds to an integer
+constexpr float kOffsetRefLimit = 16384.f;     // |reference| beyond this: report, outputs may drift
+
+// 2^(e - 10): the code step of exponent e, in log2 units.
+__device__ __forceinline__ float code_step(uint32_t e) { return __uint_as_float((117u + e) << 23); }
+// 2^(10 - e): code steps per log2 unit.
+__device__ __forceinline__ float code_inv_step(uint32_t e) { return __uint_as_float((137u - e) << 23); }
+
+// Smallest e in [0, 5] whose 65535 steps of 2^(e-10) cover `range` log2 units.
+__device__ __forceinline__ uint32_t code_exponent(float range) {
+  uint32_t e = 0;
+#pragma unroll
+  for (int k = 0; k < 5; ++k) e += (range > 63.99f * static_cast<float>(1 << k)) ? 1u : 0u;
+  return e;
+}
+
+// Codes of two raw scores s0, s1 (round((ref - s * sl2) / step), clamped to [0, 65535]), packed
+// low / high.  nsl = -sl2 / step, refs = ref / step.
+__device__ __forceinline__ uint32_t encode_offsets(float s0, float s1, float nsl, float refs) {
+  const float a = fmaxf(fminf(fmaf(s0, nsl, refs) + kOffsetMagic, kOffsetMagic + 65535.f), kOffsetMagic);
+  const float b = fmaxf(fminf(fmaf(s1, nsl, refs) + kOffsetMagic, kOffsetMagic + 65535.f), kOffsetMagic);
+  return __byte_perm(__float_as_uint(a), __float_as_uint(b), 0x5410);
+}
+// -code * step for a 16-bit code (exact).
+__device__ __forceinline__ float decode_offset(uint32_t code, float step) {
+  return fmaf(__uint_as_float(0x4B000000u | code), -step, kOffsetMagic * step);
+}
+// Sum of the two bf16 values packed in w.
+__device__ __forceinline__ float bf16x2_sum(uint32_t w) {
+  return __uint_as_float(w << 16) + __uint_as_float(w & 0xffff0000u);
+}
 
 // MODE_GTA: grouped-tied attention, the GQLA shapes with K_j = V_j (one tied state per group).
 enum DecodeMode { MODE_MLA = 0, MODE_GQLA = 1, MODE_GLA = 2, MODE_GTA = 3 };
@@ -542,7 +580,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                                           : stage_base + static_cast<uint32_t>(n % KS) * kStageBytes;
             const uint64_t vdesc = sdesc_sw128(vaddr + Cfg::kVBox0 * kBoxBytes, kBoxBytes, 1024);
             if constexpr (kPair) {
-              // P(n) was written over the peer's factors in message slot n % 3 (K-major, 128-byte swizzle)
+              // P(n) was written over the peer's score codes in message slot n % 3 (K-major, 128-byte swizzle)
               const uint64_t pdesc = sdesc_sw128(smem_u32(rbuf + (n % kMsgSlots) * kMsgStride), 16, 1024);
 #pragma unroll
               for (int kk = 0; kk < TN / 16; ++kk)
@@ -631,8 +669,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else if (kPair && warp >= 4 && warp < 12) {
     // ============================================================ MLA softmax
-    // Warps 4-7 (score warps) turn S into this CTA's factors E and stage them for the peer;
-    // warps 8-11 (combine warps) form P from both CTAs' factors, publish it, rescale O and run
+    // Warps 4-7 (score warps) encode S as this CTA's score codes and stage them for the peer;
+    // warps 8-11 (combine warps) form P from both CTAs' codes, publish it, rescale O and run
     // the epilogue.  The two run on different tiles at the same time (the score warps one tile
     // ahead), each warp owns TMEM lane quadrant q = warp % 4 and all 64 key columns.
     const int q4 = warp & 3;
@@ -709,19 +747,33 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             sm.n_armed = n + 1;
           }
           const int rem = sg.keys - t * TN;  // valid keys in this tile
+          // row max and min of the partial scores over the valid keys (the scale is positive)
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          float n4[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
           if (rem < TN) {
 #pragma unroll
-            for (int c = 0; c < TN; ++c) cs[c] = (c < rem) ? cs[c] : -INFINITY;
+            for (int c = 0; c < TN; ++c) {
+              n4[c & 3] = (c < rem) ? fminf(n4[c & 3], cs[c]) : n4[c & 3];
+              cs[c] = (c < rem) ? cs[c] : -INFINITY;
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < TN; ++c) n4[c & 3] = fminf(n4[c & 3], cs[c]);
           }
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int c = 0; c < TN; ++c) m4[c & 3] = fmaxf(m4[c & 3], cs[c]);
           const float tcur = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.sl2;  // log2 units
+          const float tmin = fminf(fminf(n4[0], n4[1]), fminf(n4[2], n4[3])) * p.sl2;
           const float tsub = (tcur == -INFINITY) ? 0.f : tcur;
+          if (!(fabsf(tsub) < kOffsetRefLimit)) record_error(p.err, LKV_SITE_SCORE_RANGE);
+          // The reference carries the step exponent in its low bits; codes are taken against it.
+          const uint32_t ex = code_exponent(tsub - tmin);
+          const float t_ref = __uint_as_float((__float_as_uint(tsub) & ~((1u << kStepBits) - 1u)) | ex);
+          const float inv_step = code_inv_step(ex);
           uint32_t e[TN / 2];
 #pragma unroll
           for (int c = 0; c < TN / 2; ++c)
-            e[c] = ex2_f16x2(fmaf(cs[2 * c], p.sl2, -tsub), fmaf(cs[2 * c + 1], p.sl2, -tsub));
+            e[c] = encode_offsets(cs[2 * c], cs[2 * c + 1], -p.sl2 * inv_step, t_ref * inv_step);
           // the staging copy holds message n-1 until the sender and the combine warps read it
           if (n >= 1 &&
               (!wait_all(smem_u32(&sm.x_stage_free), static_cast<uint32_t>((n - 1) & 1), LKV_WAIT(W_XFREE)) ||
@@ -734,7 +786,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int c = 0; c < 8; ++c)
             *reinterpret_cast<uint4*>(sbuf + r * 128 + ((c ^ (r & 7)) << 4)) =
                 make_uint4(e[4 * c], e[4 * c + 1], e[4 * c + 2], e[4 * c + 3]);
-          reinterpret_cast<float*>(sbuf + 128 * 128)[r] = tcur;
+          reinterpret_cast<float*>(sbuf + 128 * 128)[r] = t_ref;
           warp_arrive(smem_u32(&sm.x_staged));
         }
         if (!ok) break;
@@ -742,7 +794,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
     } else {
       // ---------------------------------------------------------- combine warps
-      float m_run = -INFINITY, l_run = 0.f;
+      float m_run = -INFINITY, l_run = 0.f, lb_run = 0.f;
       int nconsumed = 0;
       while (ok && next_seg(cur, sg)) {
         for (int t = sg.tile_lo; t < sg.tile_hi && ok; ++t, ++n) {
@@ -751,7 +803,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             ok = false;
             break;
           }
-          uint32_t eo[32], ep[32];
+          uint32_t eo[32];
 #pragma unroll
           for (int c = 0; c < 8; ++c) {
             const uint4 x = *reinterpret_cast<const uint4*>(sbuf + r * 128 + ((c ^ (r & 7)) << 4));
@@ -768,47 +820,109 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             break;
           }
           uint8_t* msg = rbuf + xb * kMsgStride;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint4 x = *reinterpret_cast<const uint4*>(msg + r * 128 + ((c ^ (r & 7)) << 4));
-            ep[4 * c] = x.x;
-            ep[4 * c + 1] = x.y;
-            ep[4 * c + 2] = x.z;
-            ep[4 * c + 3] = x.w;
-          }
           const float t_p = reinterpret_cast<const float*>(msg + 128 * 128)[r];
+          const uint32_t e_o = __float_as_uint(t_o) & ((1u << kStepBits) - 1u);
+          const uint32_t e_p = __float_as_uint(t_p) & ((1u << kStepBits) - 1u);
+          const int rem = sg.keys - t * TN;  // valid keys in this tile (>= 1)
+          // Both halves on one step (the usual case): per key the code sum, an exact integer in
+          // common steps, saturated at 65535.  Otherwise each key's offset is formed in fp32.
+          const bool same = __all_sync(0xffffffffu, e_o == e_p) != 0;
+          const float st_o = code_step(e_o), st_p = code_step(e_p);
+          float ybest;         // best key's offset below the reference sum (log2 units, <= 0)
+          uint32_t smin2 = 0;  // same-step path: the best key's code sum in both halves of a word
+          uint32_t nsat = 0;   // keys whose code saturated (the masked keys of a ragged tile excluded)
+          if (same) {
+            uint32_t mn2 = 0xffffffffu;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const uint4 x = *reinterpret_cast<const uint4*>(msg + r * 128 + ((c ^ (r & 7)) << 4));
+              eo[4 * c] = __vaddus2(eo[4 * c], x.x);
+              eo[4 * c + 1] = __vaddus2(eo[4 * c + 1], x.y);
+              eo[4 * c + 2] = __vaddus2(eo[4 * c + 2], x.z);
+              eo[4 * c + 3] = __vaddus2(eo[4 * c + 3], x.w);
+              mn2 = __vminu2(mn2, __vminu2(__vminu2(eo[4 * c], eo[4 * c + 1]), __vminu2(eo[4 * c + 2], eo[4 * c + 3])));
+              nsat += __popc(__vcmpeq2(eo[4 * c], 0xffffffffu)) + __popc(__vcmpeq2(eo[4 * c + 1], 0xffffffffu)) +
+                      __popc(__vcmpeq2(eo[4 * c + 2], 0xffffffffu)) + __popc(__vcmpeq2(eo[4 * c + 3], 0xffffffffu));
+            }
+            // masked keys carry the top code on both sides, so the smallest sum is a valid key's
+            const uint32_t smin = min(mn2 & 0xffffu, mn2 >> 16);
+            smin2 = smin | (smin << 16);
+            ybest = decode_offset(smin, st_o);
+          } else {
+            ybest = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              const uint4 x = *reinterpret_cast<const uint4*>(msg + r * 128 + ((c ^ (r & 7)) << 4));
+              const uint32_t xw[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                const uint32_t wo = eo[4 * c + j], wp = xw[j];
+                const float y0 = decode_offset(wo & 0xffffu, st_o) + decode_offset(wp & 0xffffu, st_p);
+                const float y1 = decode_offset(wo >> 16, st_o) + decode_offset(wp >> 16, st_p);
+                const int k0 = 2 * (4 * c + j);
+                ybest = fmaxf(ybest, fmaxf(k0 < rem ? y0 : -INFINITY, k0 + 1 < rem ? y1 : -INFINITY));
+                nsat += __popc(__vcmpeq2(wo, 0xffffffffu) | __vcmpeq2(wp, 0xffffffffu));
+              }
+            }
+          }
+          nsat = nsat / 16 - (rem < TN ? static_cast<uint32_t>(TN - rem) : 0u);
           ++nconsumed;
           warp_arrive(smem_u32(&sm.x_consumed[n & 1]));
-          // P = E_own * E_peer * 2^(t_own + t_peer - m): t_own + t_peer bounds the row's scores in
-          // this tile; products of two floats commute, so both CTAs get the same P
+          // A saturated key's true offset exceeds its computed one, so its computed weight bounds its
+          // true weight; both lie below 2^-(65535 steps + ...) of the best key.  Report the tile when
+          // those keys together could carry more than 2^-12 of the best key's weight.
+          if (nsat > 0) {
+            const float gap = 65535.f * fminf(st_o, st_p) + ybest;  // log2 units between them, at least
+            if (static_cast<float>(nsat) > ex2_approx(gap - 12.f)) record_error(p.err, LKV_SITE_SCORE_RANGE);
+          }
           if (first) {
             m_run = -INFINITY;
             l_run = 0.f;
+            lb_run = 0.f;
           }
-          const float T = t_o + t_p;  // -inf when every key of this tile is masked for the row
+          const float T = t_o + t_p;  // reference sum (log2 units)
+          const float mx = T + ybest;  // this tile's row max
           bool rescale = false;
           float m_new = m_run;
-          if (T > m_run + 8.f) {  // lazy rescale: keep the running max unless it grows by 2^8
-            m_new = T;
+          if (mx > m_run + 8.f) {  // lazy rescale: keep the running max unless it grows by 2^8
+            m_new = mx;
             rescale = (m_run != -INFINITY);
           }
           const float alpha = rescale ? ex2_approx(m_run - m_new) : 1.f;
-          // f <= 2^8; products below the fp16 range only drop terms under 2^-24 of the max
-          const float f = (T == -INFINITY) ? 0.f : ex2_approx(T - m_new);
-          const uint32_t f2 = pack_f16x2(f, f);
-          float s4[4] = {0.f, 0.f, 0.f, 0.f};
+          // P = 2^(offset - ybest) (exact exponent, <= 0, centred on the tile max) times
+          // f = 2^(mx - m_new) <= 2^8 in fp32
+          const float f = ex2_approx(mx - m_new);
+          float s4[4] = {0.f, 0.f, 0.f, 0.f}, b4[4] = {0.f, 0.f, 0.f, 0.f};
           uint32_t pw[32];
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
-            const uint32_t pr = mul_f16x2(mul_f16x2(eo[c], ep[c]), f2);
-            const float e0 = f16_lo(pr), e1 = f16_hi(pr);
+            float a0, a1;
+            if (same) {
+              const uint32_t dlt = __vsub2(eo[c], smin2);
+              a0 = decode_offset(dlt & 0xffffu, st_o);
+              a1 = decode_offset(dlt >> 16, st_o);
+            } else {
+              const uint32_t wp = *reinterpret_cast<const uint32_t*>(msg + r * 128 + (((c >> 2) ^ (r & 7)) << 4) + 4 * (c & 3));
+              a0 = decode_offset(eo[c] & 0xffffu, st_o) + decode_offset(wp & 0xffffu, st_p) - ybest;
+              a1 = decode_offset(eo[c] >> 16, st_o) + decode_offset(wp >> 16, st_p) - ybest;
+            }
+            if (rem < TN) {
+              a0 = (2 * c < rem) ? a0 : -INFINITY;
+              a1 = (2 * c + 1 < rem) ? a1 : -INFINITY;
+            }
+            const uint32_t pr = ex2_f16x2(a0, a1);
+            const float e0 = f16_lo(pr) * f, e1 = f16_hi(pr) * f;
             s4[c & 3] += e0 + e1;
             pw[c] = pack_bf16x2(e0, e1);
+            b4[c & 3] += bf16x2_sum(pw[c]);
           }
+          // l_run (fp32 weights) gives the lse; lb_run sums the bf16 weights PV actually used, so
+          // that the output is normalised by exactly the weights in O
           l_run = l_run * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+          lb_run = lb_run * alpha + ((b4[0] + b4[1]) + (b4[2] + b4[3]));
           m_run = m_new;
           const int pb = n & 1;
-          // P(n) replaces the peer's factors in slot xb: the same 128-byte swizzled rows are the
+          // P(n) replaces the peer's codes in slot xb: the same 128-byte swizzled rows are the
           // K-major A operand of PV(n) (the sender keeps the peer off this slot until PV(n) is done)
 #pragma unroll
           for (int c = 0; c < 8; ++c)
@@ -825,11 +939,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tc_fence_after();
             tmem_scale_row(tm_addr(tbase, lb, 0), DV, alpha);
           }
-          const int key0 = t * TN;
-          if (key0 + TN > sg.keys) {
+          if (rem < TN) {
             // Rows past the unit's last key belong to another request or to unwritten cache:
             // their P is 0, but 0 * NaN would still poison O, so clear those V rows first.
-            const int firstbad = sg.keys - key0;
+            const int firstbad = rem;
             const int per_box = (TN - firstbad) * 8;  // 16-byte chunks per V box
             uint8_t* vb = dsm + (n % KS) * kStageBytes;
             for (int idx = r; idx < per_box * Cfg::kNV; idx += 128) {
@@ -849,7 +962,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             break;
           }
           tc_fence_after();
-          const float inv_l = l_run > 0.f ? 1.f / l_run : 0.f;
+          const float inv_l = lb_run > 0.f ? 1.f / lb_run : 0.f;
           const float lse_v = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
           const size_t orow = (static_cast<size_t>(sg.b) * p.s_q + sg.k) * p.h_q + r;
           if (sg.complete) {
@@ -961,8 +1074,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       warp_arrive(smem_u32(&sm.q_ready));
     };
 
-    // Running max (shared by both halves of a row) and this half's running sum.
-    float m_run = -INFINITY, l_run = 0.f;
+    // Running max (shared by both halves of a row) and this half's running sums.
+    float m_run = -INFINITY, l_run = 0.f, lb_run = 0.f;
     // Lazy rescale: keep the running max unless the tile max exceeds it by 2^8.
     auto new_max = [&](float mx, bool& rescale, float& alpha) -> float {
       rescale = false;
@@ -981,6 +1094,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (t == sg.tile_lo) {
         m_run = -INFINITY;
         l_run = 0.f;
+        lb_run = 0.f;
       }
       // keys of this half of the tile visible to this row
       const int rem = (sg.L - p.s_q + qi + 1) - (t * TN + c0);
@@ -996,17 +1110,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const float mh = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * p.sl2;
       float mo;
       if (!pair_xchg(mh, mo)) return false;
-      const float m_new = new_max(fmaxf(mh, mo), rescale, alpha);
-      const float msub = (m_new == -INFINITY) ? 0.f : m_new;
-      float s4[4] = {0.f, 0.f, 0.f, 0.f};
+      const float mx = fmaxf(mh, mo);  // this tile's row max
+      const float m_new = new_max(mx, rescale, alpha);
+      // exponents centred on the tile max (<= 0, so the fp16 argument of the best keys is exact
+      // or nearly so), times f = 2^(mx - m_new) <= 2^8 in fp32
+      const float msub = (mx == -INFINITY) ? 0.f : mx;
+      const float f = (mx == -INFINITY) ? 0.f : ex2_approx(mx - m_new);
+      float s4[4] = {0.f, 0.f, 0.f, 0.f}, b4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < HW; ++c) {
         const uint32_t h = ex2_f16x2(fmaf(s[2 * c], p.sl2, -msub), fmaf(s[2 * c + 1], p.sl2, -msub));
-        const float e0 = f16_lo(h), e1 = f16_hi(h);
+        const float e0 = f16_lo(h) * f, e1 = f16_hi(h) * f;
         s4[c & 3] += e0 + e1;
         pw[c] = pack_bf16x2(e0, e1);
+        b4[c & 3] += bf16x2_sum(pw[c]);
       }
+      // l_run (fp32 weights) gives the lse; lb_run sums the bf16 weights PV actually used
       l_run = l_run * alpha + ((s4[0] + s4[1]) + (s4[2] + s4[3]));
+      lb_run = lb_run * alpha + ((b4[0] + b4[1]) + (b4[2] + b4[3]));
       m_run = m_new;
       return true;
     };
@@ -1065,13 +1186,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       warp_arrive(smem_u32(&sm.p_full[pb]));
       if (t != sg.tile_hi - 1) return true;
       // ---------------------------------------------------------- segment epilogue
-      float l_other;
-      if (!pair_xchg(l_run, l_other)) return false;
-      const float l_tot = l_run + l_other;
+      float l_other, lb_other;
+      if (!pair_xchg(l_run, l_other) || !pair_xchg(lb_run, lb_other)) return false;
+      const float l_tot = l_run + l_other, lb_tot = lb_run + lb_other;
       if (!wait_all(smem_u32(&sm.o_done[pb]), static_cast<uint32_t>((n >> 1) & 1), LKV_WAIT(W_ODONE)))
         return false;
       tc_fence_after();
-      const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      const float inv_l = lb_tot > 0.f ? 1.f / lb_tot : 0.f;
       const float lse_v = l_tot > 0.f ? (m_run + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
       const size_t orow = (static_cast<size_t>(sg.b) * p.s_q + qi) * p.h_q + qh;
       if (sg.complete) {

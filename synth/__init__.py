@@ -38,6 +38,9 @@ class Workload:
             in [len_lo, len_hi].
     input_std  standard deviation of every Gaussian input entry before the
             storage rounding.
+    q_std   standard deviation of the query entries (q and q_rope) when it differs
+            from input_std (None: input_std).  Widening only the query widens the
+            score range while the cached values keep their size.
     """
     name: str
     kind: str
@@ -54,6 +57,7 @@ class Workload:
     input_std: float
     len_lo: int = 0
     len_hi: int = 0
+    q_std: float | None = None
 
     @property
     def scale(self) -> float:
@@ -174,8 +178,9 @@ def make_inputs(w: Workload, extra_rows: int = 0, lengths=None) -> dict:
     rows = total + extra_rows
     B, S, H, G = w.batch, w.s_q, w.h_q, w.groups
     std = w.input_std
-    q = _normal(rng, (B, S, H, w.d_k), std, w.dtype)
-    q_rope = _normal(rng, (B, S, H, w.d_rope), std, w.dtype)
+    qs = std if w.q_std is None else w.q_std
+    q = _normal(rng, (B, S, H, w.d_k), qs, w.dtype)
+    q_rope = _normal(rng, (B, S, H, w.d_rope), qs, w.dtype)
     res = {"lengths": lengths, "cu_seqlens": torch.from_numpy(cu.astype(np.int32)),
            "q": q, "q_rope": q_rope, "workload": w}
     tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32

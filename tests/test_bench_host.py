@@ -57,3 +57,45 @@ def test_source_hash_covers_only_the_decode_sources():
     assert len(h) == 16
     assert "lkv_proj.cu" not in bench.DECODE_SOURCES and "lkv_fp8.cu" not in bench.DECODE_SOURCES
     assert bench.kernel_source_hash() == h                   # deterministic
+
+
+def test_roofline_entry_is_the_slower_of_bytes_and_flops():
+    w = synth.workload("mla_b64_l4096")
+    lengths = np.full(w.batch, w.seqlen, dtype=np.int64)
+    peaks = {"hbm_gbs": 1000.0, "bf16_tflops": 100.0}
+    cache_bytes, io_bytes, flops = bench.workload_accounting(w, lengths)
+    t_hbm, t_tc = (cache_bytes + io_bytes) / 1e12, flops / 1e14
+    r = bench.roofline_entry(w, lengths, 2e3 * max(t_hbm, t_tc), peaks, "test")
+    assert r["bound"] == ("hbm" if t_hbm >= t_tc else "tensor")
+    assert r["frac"] == pytest.approx(0.5)                  # twice the roofline time
+    assert r["roofline_ms"] == pytest.approx(1e3 * max(t_hbm, t_tc))
+    assert r["algorithmic_bytes"] == cache_bytes + io_bytes and r["algorithmic_flops"] == flops
+
+
+@pytest.mark.parametrize("name,kw", [("tiny_fp32_mla", {}),
+                                     ("gqla_g8_sq2_l8192", dict(batch=2, seqlen=130)),
+                                     ("gta_g8_sq2_l8192", dict(batch=2, seqlen=70)),
+                                     ("varlen_mla_sq1", dict(batch=3, len_lo=8, len_hi=64))])
+def test_device_inputs_match_the_synth_layout(name, kw):
+    import torch
+    w = synth.workload(name, **kw)
+    d = bench.device_inputs(w, torch.device("cpu"))
+    ref = synth.make_inputs(w)
+    assert np.array_equal(d["lengths"], ref["lengths"])      # the same length draw
+    assert torch.equal(d["cu_seqlens"], ref["cu_seqlens"])
+    for k in ("q", "q_rope", "cache", "k", "v", "kpe"):
+        if k in ref:
+            assert d[k].shape == ref[k][:int(ref["lengths"].sum())].shape if k not in ("q", "q_rope") \
+                else d[k].shape == ref[k].shape
+            assert d[k].dtype == ref[k].dtype
+    x = d["cache"] if "cache" in d else d["k"]
+    assert abs(float(x.float().std()) - w.input_std) < 0.1 * w.input_std
+
+
+def test_cpu_baseline_on_device_inputs_is_bounded():
+    import torch
+    w = synth.workload("gqla_g8_sq2_l8192", batch=3, seqlen=None, len_lo=16, len_hi=64)
+    d = bench.device_inputs(w, torch.device("cpu"))
+    cb = bench.cpu_baseline_device(w, d, 0.0)                # budget spent after the first request
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] == os.cpu_count()
+    assert cb["sample"].startswith("1 of 3 requests")

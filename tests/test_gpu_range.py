@@ -1,0 +1,162 @@
+"""GPU parity at large score ranges: every tensor-core decode entry point against the fp64 oracle
+on inputs built to stress the softmax, with the same gates as the other parity tests.
+
+* Wide score spread: the query drawn with a larger std (scores of std 4, 9 and 16 nat, the spread
+  of N(0,1)*sigma inputs at scale 1/24 for sigma = 2, 3, 4), the cache at std 1/2 so that the
+  output's own bf16 rounding stays well inside the absolute gate.
+* One dominant key per request (+50 nat on every head): the oracle's closed form makes the
+  output the value row of that key.
+* All scores equal (q = 0): the output is the mean of the visible value rows, lse = ln(keys).
+* Cancellation between the two halves of the contracted columns: for every third key the RoPE
+  column 0 adds +c log2 units and RoPE column 32 adds -c, so the full score is unchanged while the
+  partial scores over columns [0, 32) and [32, 64) of the RoPE key move far apart.  The MLA CTA
+  pair contracts those two column ranges in different CTAs, so this is the case where each CTA's
+  partial scores alone say nothing about which keys matter.
+
+The planted values are written into the stored inputs before either side sees them, so the
+oracle and the kernels read identical bf16 values.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from gpu_util import compare, run_lib, run_oracle, to_dev
+
+pytestmark = pytest.mark.gpu
+
+LOG2E = 1.0 / math.log(2.0)
+
+# (base workload, lengths, s_q) per decode form: ragged lengths that span several tiles
+FORMS = {
+    "mla": ("mla_b64_l4096", [1000, 300, 65, 4097], 1),
+    "mla_sq2": ("mla_b64_l4096", [700, 2, 129, 2050], 2),
+    "gqla": ("gqla_g8_sq2_l8192", [900, 130, 2, 2000], 2),
+    "gla": ("long_gla2", [1000, 65, 3000], 1),
+    "gta": ("gta_g8_sq2_l8192", [900, 130, 2, 1500], 2),
+    "gqa2": ("gqa2_sq2_l8192", [700, 129, 2], 2),
+}
+
+
+@pytest.fixture(scope="module")
+def L(gpu):
+    import latent_kv_cache_split_b200 as lib
+    return lib
+
+
+def _workload(form, **kw):
+    name, lengths, s_q = FORMS[form]
+    return synth.workload(name, batch=len(lengths), s_q=s_q, seqlen=None, **kw), lengths
+
+
+def _rope_cache(d):
+    """The stored RoPE-key columns (a view into the cache where it is interleaved)."""
+    w = d["workload"]
+    if w.kind == "gqla":
+        return d["kpe"]
+    return d["cache"][:, w.groups * w.d_k:]
+
+
+def _bf16(x: float) -> float:
+    return float(torch.tensor(x, dtype=torch.float32).to(torch.bfloat16).float())
+
+
+def _check(L, gpu, d, label):
+    out, lse = run_lib(L, to_dev(d, gpu))
+    torch.cuda.synchronize()
+    assert L.check_device() == 0, label
+    ref_out, ref_lse = run_oracle(d)
+    return compare(out, lse, ref_out, ref_lse, label=label)
+
+
+@pytest.mark.parametrize("form", sorted(FORMS))
+@pytest.mark.parametrize("spread", [4.0, 9.0, 16.0])
+def test_wide_score_spread(L, gpu, form, spread):
+    # score std = q_std * cache_std * sqrt(d_k + d_R) * scale = q_std / 2
+    w, lengths = _workload(form, input_std=0.5, q_std=2.0 * spread)
+    d = synth.make_inputs(w, lengths=lengths)
+    _check(L, gpu, d, f"{form} spread {spread}")
+
+
+@pytest.mark.parametrize("form", sorted(FORMS))
+def test_dominant_key(L, gpu, form):
+    w, lengths = _workload(form)
+    d = synth.make_inputs(w, lengths=lengths)
+    kr = _rope_cache(d)
+    d["q_rope"][..., 0] = 1.0
+    kr[:, 0] = 0.0
+    cu = d["cu_seqlens"].numpy()
+    rng = np.random.default_rng(11)
+    star = []
+    for b, n in enumerate(lengths):
+        t = int(rng.integers(0, n - w.s_q + 1))  # visible to every new token
+        kr[int(cu[b]) + t, 0] = _bf16(50.0 / w.scale)
+        star.append(int(cu[b]) + t)
+    r = _check(L, gpu, d, f"{form} dominant key")
+    # the closed form: the output is (up to e^-50 and storage rounding) the dominant key's value row
+    out_ref, _ = run_oracle(d)
+    for b, row in enumerate(star):
+        if w.kind == "gqla":
+            v = d["v"][row].float().numpy()                      # [g, d_h]
+        elif w.kind == "mla":
+            v = d["cache"][row, :w.d_k].float().numpy()[None, :]
+        else:
+            v = d["cache"][row, :w.groups * w.d_k].float().numpy().reshape(w.groups, w.d_k)
+        hpg = w.h_q // w.groups
+        expect = np.repeat(v, hpg, axis=0)                        # [h_q, d_v]
+        assert np.abs(out_ref[b] - expect[None]).max() < 1e-9
+    assert r["max_abs"] <= 1e-2
+
+
+@pytest.mark.parametrize("form", sorted(FORMS))
+def test_all_scores_equal(L, gpu, form):
+    w, lengths = _workload(form)
+    d = synth.make_inputs(w, lengths=lengths)
+    d["q"].zero_()
+    d["q_rope"].zero_()
+    _check(L, gpu, d, f"{form} equal scores")
+    _, lse_ref = run_oracle(d)
+    for b, n in enumerate(lengths):
+        for i in range(w.s_q):
+            assert np.allclose(lse_ref[b, i], math.log(n - w.s_q + i + 1), atol=1e-12)
+
+
+def _plant_cancellation(d, c_log2: float):
+    """Every third key: RoPE column 0 adds +c log2 units to its score on every head, column 32 adds -c."""
+    w = d["workload"]
+    delta = _bf16(c_log2 / (w.scale * LOG2E))
+    kr = _rope_cache(d)
+    d["q_rope"][..., 0] = 1.0
+    d["q_rope"][..., 32] = 1.0
+    kr[:, 0] = 0.0
+    kr[:, 32] = 0.0
+    cu = d["cu_seqlens"].numpy()
+    for b in range(w.batch):
+        rows = np.arange(int(cu[b]), int(cu[b + 1]))[::3]
+        kr[rows, 0] = delta
+        kr[rows, 32] = -delta
+
+
+@pytest.mark.parametrize("form", sorted(FORMS))
+@pytest.mark.parametrize("c_log2", [20.0, 40.0, 90.0])
+def test_cancellation_between_column_halves(L, gpu, form, c_log2):
+    w, lengths = _workload(form)
+    d = synth.make_inputs(w, lengths=lengths)
+    _plant_cancellation(d, c_log2)
+    _check(L, gpu, d, f"{form} cancellation {c_log2}")
+
+
+@pytest.mark.parametrize("form", ["mla", "mla_sq2"])
+def test_cancellation_beyond_the_exchange_range_is_reported(L, gpu, form):
+    """Partial scores 3000 log2 units apart exceed what the MLA pair's 16-bit score codes can carry
+    (65535 steps of at most 2^-5); the kernel records LKV_SITE_SCORE_RANGE instead of failing silently."""
+    w, lengths = _workload(form)
+    d = synth.make_inputs(w, lengths=lengths)
+    _plant_cancellation(d, 3000.0)
+    L.check_device(clear=True)
+    run_lib(L, to_dev(d, gpu))
+    torch.cuda.synchronize()
+    assert L.check_device(clear=True) == L.SITE_SCORE_RANGE
+    assert L.check_device() == 0
