@@ -47,7 +47,8 @@ NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 # The sources the decode kernels and their launch are built from (the projections' translation unit
 # and the header's declarations do not change what a decode launch reads or writes).
-DECODE_SOURCES = ("lkv_api.cu", "lkv_aux.cuh", "lkv_decode_tc.cuh", "lkv_ptx.cuh", "lkv_sched.cuh", "lkv_tma_host.h")
+DECODE_SOURCES = ("lkv_api.cu", "lkv_aux.cuh", "lkv_decode_tc.cuh", "lkv_mla_pair.cuh", "lkv_ptx.cuh", "lkv_sched.cuh",
+                  "lkv_tma_host.h")
 
 
 def kernel_source_hash() -> str:

@@ -83,7 +83,7 @@ int lkv_plan_ranges(int kind, int batch, int s_q, int groups, int num_sms);
  * Host-only view of the same partition (no CUDA call): for host-side cu_seqlens_host [batch+1]
  * and `num_ranges` ranges, writes one record of 8 int32 per segment, in processing order:
  *   (range, request, unit, tile_lo, tile_hi, complete, slot, unit_id)
- * tiles are 64 keys (MLA, GLA) or 128 keys (GQLA, GTA); slot is -1 for a segment that covers its whole unit, else the partial
+ * tiles are 256 keys (MLA), 128 keys (GQLA, GTA) or 64 keys (GLA); slot is -1 for a segment that covers its whole unit, else the partial
  * slot (0 = first segment of its range, 1 = last).  Returns the number of segments (records
  * past max_out are counted but not written), or -1 on bad input.
  */
@@ -110,7 +110,8 @@ size_t lkv_group_decode_workspace_size(int kind, int batch, int s_q, int h_q, in
  *              request is recorded as LKV_SITE_BAD_LENGTH and its outputs are not written)
  *   out        [batch, s_q, h_q, r_kv] (bf16 for LKV_BF16, fp32 for LKV_FP32)
  *   lse        [batch, s_q, h_q] fp32
- * Implemented: LKV_BF16 with r_kv = 512, d_rope = 64, h_q = 128 (tcgen05 kernel, CTA pairs);
+ * Implemented: LKV_BF16 with r_kv = 512, d_rope = 64, h_q = 128 (tcgen05 kernel on CTA pairs that
+ *              share one MMA, 256-key tiles);
  *              LKV_FP32 with r_kv + d_rope <= 1024, r_kv <= 512 (CUDA-core kernel).
  * s_q must be 1 or 2.  workspace_bytes >= lkv_mla_decode_workspace_size(...).
  */
@@ -335,10 +336,6 @@ lkv_status lkv_expand_latent(const void* c, int64_t c_row_stride, const void* w,
 #define LKV_SITE_SELFTEST 1
 #define LKV_SITE_BAD_LENGTH 2     /* a request with L_b < s_q (append or decode)      */
 #define LKV_SITE_BAD_ROW 3        /* a cache row past cache_rows                      */
-/* MLA absorbed decode (bf16): the two halves of a row's scores lie too far apart for the pair's
- * score exchange -- a tile's best key more than 103 log2 units below the sum of the two halves'
- * partial maxima, or a partial tile max beyond 16384 log2 units.  Outputs may be inexact. */
-#define LKV_SITE_SCORE_RANGE 4
 #define LKV_SITE_WAIT_BASE 100    /* + kernel-specific wait site: a bounded wait gave up */
 
 #ifdef __cplusplus

@@ -32,7 +32,7 @@ _lib = ctypes.CDLL(LIB_PATH)
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_DEVICE = range(6)
 BF16, FP32 = 0, 1
 KIND_MLA, KIND_GQLA, KIND_GLA, KIND_GTA = 0, 1, 2, 3
-SITE_SELFTEST, SITE_BAD_LENGTH, SITE_BAD_ROW, SITE_SCORE_RANGE, SITE_WAIT_BASE = 1, 2, 3, 4, 100  # device error word
+SITE_SELFTEST, SITE_BAD_LENGTH, SITE_BAD_ROW, SITE_WAIT_BASE = 1, 2, 3, 100   # device error word
 
 _vp, _i64, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
 

@@ -10,6 +10,7 @@
 #include "../../include/lkv.h"
 #include "lkv_aux.cuh"
 #include "lkv_decode_tc.cuh"
+#include "lkv_mla_pair.cuh"
 #include "lkv_ptx.cuh"
 #include "lkv_tma_host.h"
 
@@ -39,8 +40,7 @@ unsigned long long wait_limit_ns() {
 }
 
 constexpr size_t tc_smem_bytes(int mode) {
-  return mode == MODE_MLA    ? ModeCfg<MODE_MLA>::kSmemBytes
-         : mode == MODE_GQLA ? ModeCfg<MODE_GQLA>::kSmemBytes
+  return mode == MODE_GQLA ? ModeCfg<MODE_GQLA>::kSmemBytes
          : mode == MODE_GTA  ? ModeCfg<MODE_GTA>::kSmemBytes
                              : ModeCfg<MODE_GLA>::kSmemBytes;
 }
@@ -56,14 +56,14 @@ lkv_status device_state(DeviceState** out) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_lkv_error_word) != cudaSuccess) return LKV_ERR_CUDA;
     d.err = static_cast<int*>(p);
-    if (cudaFuncSetAttribute(decode_tc_kernel<MODE_MLA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(tc_smem_bytes(MODE_MLA))) != cudaSuccess ||
-        cudaFuncSetAttribute(decode_tc_kernel<MODE_GQLA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(decode_tc_kernel<MODE_GQLA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(tc_smem_bytes(MODE_GQLA))) != cudaSuccess ||
         cudaFuncSetAttribute(decode_tc_kernel<MODE_GLA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(tc_smem_bytes(MODE_GLA))) != cudaSuccess ||
         cudaFuncSetAttribute(decode_tc_kernel<MODE_GTA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(tc_smem_bytes(MODE_GTA))) != cudaSuccess)
+                             static_cast<int>(tc_smem_bytes(MODE_GTA))) != cudaSuccess ||
+        cudaFuncSetAttribute(mla_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(kPairSmemBytes)) != cudaSuccess)
       return LKV_ERR_CUDA;
     d.ready = true;
   }
@@ -107,6 +107,28 @@ lkv_status launch_err(cudaError_t e) {
   return LKV_ERR_CUDA;
 }
 
+// Merge the partial outputs of units split across ranges (units handled whole are left alone).
+lkv_status launch_combine(const TcParams& p, int units_per_req, int per_query_units, cudaStream_t stream) {
+  CombineParams c;
+  c.seg_info = p.seg_info;
+  c.part_lse = p.part_lse;
+  c.part_o = p.part_o;
+  c.P = p.P;
+  c.rmax = p.rmax;
+  c.dv_total = p.dv_total;
+  c.R = p.R;
+  c.per_query_units = per_query_units;
+  c.units_per_req = units_per_req;
+  c.s_q = p.s_q;
+  c.h_q = p.h_q;
+  c.hpg = p.hpg;
+  c.out = p.out;
+  c.lse = p.lse;
+  const dim3 cgrid(p.B * units_per_req, (p.R + kCombineWarps - 1) / kCombineWarps);
+  combine_kernel<<<cgrid, kCombineWarps * 32, 0, stream>>>(c);
+  return launch_err(cudaGetLastError());
+}
+
 struct TcLaunch {
   int mode;
   CUtensorMap map_a, map_r, map_v;
@@ -115,24 +137,15 @@ struct TcLaunch {
   int per_query_units;
 };
 
+// Grouped decode (one CTA per range), then the split combine.
 lkv_status run_tc(TcLaunch& L, const DeviceState& d, cudaStream_t stream) {
-  const int grid = L.mode == MODE_MLA ? 2 * L.p.P : L.p.P;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(grid);
+  cfg.gridDim = dim3(L.p.P);
   cfg.blockDim = dim3(kTcThreads);
   cfg.dynamicSmemBytes = tc_smem_bytes(L.mode);
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
   cudaError_t e;
-  if (L.mode == MODE_MLA) {
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<MODE_MLA>, L.map_a, L.map_r, L.map_v, L.p);
-  } else if (L.mode == MODE_GQLA) {
+  if (L.mode == MODE_GQLA) {
     e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<MODE_GQLA>, L.map_a, L.map_r, L.map_v, L.p);
   } else if (L.mode == MODE_GTA) {
     e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<MODE_GTA>, L.map_a, L.map_r, L.map_v, L.p);
@@ -140,24 +153,26 @@ lkv_status run_tc(TcLaunch& L, const DeviceState& d, cudaStream_t stream) {
     e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<MODE_GLA>, L.map_a, L.map_r, L.map_v, L.p);
   }
   if (e != cudaSuccess) return launch_err(e);
-  CombineParams c;
-  c.seg_info = L.p.seg_info;
-  c.part_lse = L.p.part_lse;
-  c.part_o = L.p.part_o;
-  c.P = L.p.P;
-  c.rmax = L.p.rmax;
-  c.dv_total = L.p.dv_total;
-  c.R = L.p.R;
-  c.per_query_units = L.per_query_units;
-  c.units_per_req = L.units_per_req;
-  c.s_q = L.p.s_q;
-  c.h_q = L.p.h_q;
-  c.hpg = L.p.hpg;
-  c.out = L.p.out;
-  c.lse = L.p.lse;
-  const dim3 cgrid(L.p.B * L.units_per_req, (L.p.R + kCombineWarps - 1) / kCombineWarps);
-  combine_kernel<<<cgrid, kCombineWarps * 32, 0, stream>>>(c);
-  return launch_err(cudaGetLastError());
+  return launch_combine(L.p, L.units_per_req, L.per_query_units, stream);
+}
+
+// MLA absorbed decode on CTA pairs sharing one MMA (lkv_mla_pair.cuh), then the split combine.
+lkv_status run_pair(const TcParams& p, const CUtensorMap (&maps)[5], cudaStream_t stream) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * p.P);
+  cfg.blockDim = dim3(kPairThreads);
+  cfg.dynamicSmemBytes = kPairSmemBytes;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, mla_pair_kernel, maps[0], maps[1], maps[2], maps[3], maps[4], p);
+  if (e != cudaSuccess) return launch_err(e);
+  return launch_combine(p, p.s_q, 1, stream);
 }
 
 lkv_status run_simt(SimtParams& s, cudaStream_t stream) {
@@ -229,7 +244,7 @@ int lkv_plan_segments(int kind, const int32_t* cu_seqlens_host, int batch, int s
   a.units_per_req = kind == 0 ? s_q : groups;
   a.per_query_units = kind == 0 ? 1 : 0;
   a.P = num_ranges;
-  a.tile = kind == 0 ? ModeCfg<MODE_MLA>::kTile : (kind == 1 ? ModeCfg<MODE_GQLA>::kTile : ModeCfg<MODE_GLA>::kTile);
+  a.tile = kind == 0 ? kPairTile : (kind == 1 ? ModeCfg<MODE_GQLA>::kTile : ModeCfg<MODE_GLA>::kTile);
   const bool lockstep = lockstep_groups(a);
   const SchedArgs ar = request_space(a);
   int n = 0;
@@ -326,15 +341,18 @@ lkv_status lkv_mla_absorbed_decode(const void* q_nope_abs, const void* q_rope, c
   const int P = plan_ranges(0, batch, s_q, 1, d->num_sms);
   const WsLayout w = ws_layout(P, h_q, r_kv);
   if (!workspace || !al16(workspace) || workspace_bytes < w.total) return LKV_ERR_WORKSPACE;
-  TcLaunch L;
-  L.mode = MODE_MLA;
-  constexpr int TN = ModeCfg<MODE_MLA>::kTile;
-  if (!make_tmap_bf16(&L.map_a, ckv, r_kv, cache_rows, ckv_row_stride * 2, 64, TN) ||
-      !make_tmap_bf16(&L.map_r, kpe, d_rope, cache_rows, kpe_row_stride * 2, 32, TN))  // one RoPE half per CTA
+  // Query rows (b, i, h) as 2-D [batch * s_q * h_q, width] maps in 64-row boxes (one CTA's heads);
+  // cache rows in 128-row boxes for QK (one CTA's keys of a 256-key tile) and 64-row boxes for PV.
+  const uint64_t qrows = static_cast<uint64_t>(batch) * s_q * h_q;
+  CUtensorMap maps[5];
+  if (!make_tmap_bf16(&maps[0], q_nope_abs, r_kv, qrows, static_cast<uint64_t>(r_kv) * 2, 64, 64) ||
+      !make_tmap_bf16(&maps[1], q_rope, d_rope, qrows, static_cast<uint64_t>(d_rope) * 2, 64, 64) ||
+      !make_tmap_bf16(&maps[2], ckv, r_kv, cache_rows, ckv_row_stride * 2, 64, 128) ||
+      !make_tmap_bf16(&maps[3], kpe, d_rope, cache_rows, kpe_row_stride * 2, 64, 128) ||
+      !make_tmap_bf16(&maps[4], ckv, r_kv, cache_rows, ckv_row_stride * 2, 64, 64))
     return LKV_ERR_CUDA;
-  L.map_v = L.map_a;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  TcParams& p = L.p;
+  TcParams p;
   p.q_nope = static_cast<const __nv_bfloat16*>(q_nope_abs);
   p.q_rope = static_cast<const __nv_bfloat16*>(q_rope);
   p.dq = r_kv;
@@ -356,9 +374,7 @@ lkv_status lkv_mla_absorbed_decode(const void* q_nope_abs, const void* q_rope, c
   p.P = P;
   p.err = d->err;
   p.wait_limit_ns = wait_limit_ns();
-  L.units_per_req = s_q;
-  L.per_query_units = 1;
-  return run_tc(L, *d, s);
+  return run_pair(p, maps, s);
 }
 
 lkv_status lkv_gqla_group_decode(const void* q, const void* q_rope, const void* k,

@@ -30,9 +30,9 @@ int main(void) {
   CHECK(lkv_plan_ranges(3, 64, 2, 8, 148) == 144);
   CHECK(lkv_plan_ranges(7, 64, 2, 8, 148) == -1);
 
-  /* segments of two MLA requests (100 and 200 keys, 64-key tiles) over 3 ranges: every tile once */
+  /* segments of two MLA requests (300 and 600 keys, 256-key tiles) over 3 ranges: every tile once */
   {
-    const int32_t cu[3] = {0, 100, 300};
+    const int32_t cu[3] = {0, 300, 900};
     int32_t rec[8 * 32];
     const int n = lkv_plan_segments(0, cu, 2, 1, 1, 3, rec, 32);
     CHECK(n > 0 && n <= 32);
@@ -44,7 +44,7 @@ int main(void) {
       CHECK(r[3] >= 0 && r[3] < r[4]);          /* tile_lo < tile_hi */
       tiles += r[4] - r[3];
     }
-    CHECK(tiles == 2 + 4);
+    CHECK(tiles == 2 + 3);
     CHECK(lkv_plan_segments(0, NULL, 2, 1, 1, 3, rec, 32) == -1);
   }
 

@@ -79,7 +79,7 @@ def test_workspace_sizes(lkv):
 def _check_partition(segs, cu, kind, s_q, G, P):
     """Every tile of every unit is covered exactly once; slot rules hold."""
     B = len(cu) - 1
-    T = 128 if kind == 1 else 64
+    T = {0: 256, 1: 128, 2: 64}[kind]   # keys per tile: MLA pair kernel, GQLA / GTA, GLA
     upr = s_q if kind == 0 else G
     covered = {}
     by_range = {}

@@ -7,11 +7,11 @@ on inputs built to stress the softmax, with the same gates as the other parity t
 * One dominant key per request (+50 nat on every head): the oracle's closed form makes the
   output the value row of that key.
 * All scores equal (q = 0): the output is the mean of the visible value rows, lse = ln(keys).
-* Cancellation between the two halves of the contracted columns: for every third key the RoPE
-  column 0 adds +c log2 units and RoPE column 32 adds -c, so the full score is unchanged while the
-  partial scores over columns [0, 32) and [32, 64) of the RoPE key move far apart.  The MLA CTA
-  pair contracts those two column ranges in different CTAs, so this is the case where each CTA's
-  partial scores alone say nothing about which keys matter.
+* Cancellation inside the contraction: for every third key the RoPE column 0 adds +c log2 units
+  and RoPE column 32 adds -c, so the full score is unchanged while partial sums over the
+  contracted columns move far apart.  A kernel that combined separately normalised partial
+  scores (as an earlier form of the MLA pair did) loses those keys; the fp32 accumulation of the
+  tensor-core products must keep them.
 
 The planted values are written into the stored inputs before either side sees them, so the
 oracle and the kernels read identical bf16 values.
@@ -146,17 +146,3 @@ def test_cancellation_between_column_halves(L, gpu, form, c_log2):
     d = synth.make_inputs(w, lengths=lengths)
     _plant_cancellation(d, c_log2)
     _check(L, gpu, d, f"{form} cancellation {c_log2}")
-
-
-@pytest.mark.parametrize("form", ["mla", "mla_sq2"])
-def test_cancellation_beyond_the_exchange_range_is_reported(L, gpu, form):
-    """Partial scores 3000 log2 units apart exceed what the MLA pair's 16-bit score codes can carry
-    (65535 steps of at most 2^-5); the kernel records LKV_SITE_SCORE_RANGE instead of failing silently."""
-    w, lengths = _workload(form)
-    d = synth.make_inputs(w, lengths=lengths)
-    _plant_cancellation(d, 3000.0)
-    L.check_device(clear=True)
-    run_lib(L, to_dev(d, gpu))
-    torch.cuda.synchronize()
-    assert L.check_device(clear=True) == L.SITE_SCORE_RANGE
-    assert L.check_device() == 0
