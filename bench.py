@@ -63,6 +63,14 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+def decode_kernel_name(w) -> str:
+    """The tensor-core kernel a bf16 decode call of this workload launches."""
+    if w.kind == "mla":
+        return "mla_pair_kernel"
+    return {"gqla": "decode_tc_kernel<MODE_GQLA>", "gla": "decode_tc_kernel<MODE_GLA>",
+            "gta": "decode_tc_kernel<MODE_GTA>"}.get(w.kind, "decode_tc_kernel")
+
+
 def measured_traffic(workload: str):
     """DRAM bytes (read + write) per decode-kernel launch from an ncu capture recorded in
     profiles/traffic.json, or None when absent or taken on other kernel sources."""
@@ -204,6 +212,96 @@ def make_decoder(lkv, w, d, nsm):
         else:
             lkv.gla_group_decode(qq, qqr, lat, kpe, w.groups, cu, w.scale, out=o, lse=l, workspace=ws)
     return decode
+
+
+TP_WORKLOAD = "gqla_g8_sq2_l8192"
+TP_D_MODEL = 7168   # model width the output projection maps the heads' outputs back to
+
+
+def tp_local_inputs(w, sh, dev, d_model: int):
+    """One rank's share of the group-axis TP step, drawn on the device (seeded by workload and rank):
+    the query heads of its groups, the expanded K_j, V_j of its groups, the RoPE key every rank
+    keeps, and the rows of W_O [h_q * d_v, d_model] that multiply its heads."""
+    g = torch.Generator(device=dev)
+    g.manual_seed(2000 + 17 * w.seed + sh.rank)
+    lengths = np.full(w.batch, w.seqlen, dtype=np.int64)
+    cu = synth.prefix_offsets(lengths)
+    T = int(cu[-1])
+
+    def randn(*shape, std):
+        return torch.randn(*shape, generator=g, device=dev, dtype=torch.bfloat16).mul_(std)
+
+    return {"lengths": lengths, "cu_seqlens": torch.from_numpy(cu.astype(np.int32)).to(dev),
+            "q": randn(w.batch, w.s_q, sh.heads, w.d_k, std=w.input_std),
+            "q_rope": randn(w.batch, w.s_q, sh.heads, w.d_rope, std=w.input_std),
+            "k": randn(T, sh.groups, w.d_k, std=w.input_std), "v": randn(T, sh.groups, w.d_v, std=w.input_std),
+            "kpe": randn(T, w.d_rope, std=w.input_std),
+            "w_o": randn(sh.heads * w.d_v, d_model, std=(w.h_q * w.d_v) ** -0.5)}
+
+
+def bench_tp(lkv, dev, rank: int, world: int, steps: int, warmup: int):
+    """Group-axis tensor parallelism of the GQA path (GQLA explainer, section 2): the GQLA decode
+    step of one fixed batch with its g groups split over the ranks, each rank's heads projected by
+    its rows of W_O and the partial outputs summed by one NCCL all-reduce.  Total work is fixed
+    (strong scaling).  Times are device times, the max over ranks: the whole step, and the decode,
+    the projection and the all-reduce each timed alone."""
+    from latent_kv_cache_split_b200.tp import GroupAxisTP, group_shard
+    w = synth.workload(TP_WORKLOAD)
+    if w.groups % world:
+        return {"workload": w.name, "tp": world, "skipped": f"{world} ranks do not divide g = {w.groups}"}
+    sh = group_shard(w.groups, w.h_q, world, rank)
+    d = tp_local_inputs(w, sh, dev, TP_D_MODEL)
+    B, S = w.batch, w.s_q
+    nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+    ws = torch.empty(lkv.group_decode_workspace_size(lkv.KIND_GQLA, B, S, sh.heads, sh.groups, w.d_v, nsm),
+                     dtype=torch.uint8, device=dev)
+    out = torch.empty((B, S, sh.heads, w.d_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, S, sh.heads), dtype=torch.float32, device=dev)
+    y = torch.empty((B * S, TP_D_MODEL), dtype=torch.float32, device=dev)
+
+    def decode_fn(q, qr, k, v, kpe, cu, scale):
+        lkv.gqla_group_decode(q, qr, k, v, kpe, cu, scale, out=out, lse=lse, workspace=ws)
+        return out, lse
+
+    def proj_fn(o, w_o):
+        return lkv.output_projection(o, w_o, out=y)
+
+    tp = GroupAxisTP(sh, decode_fn=decode_fn, proj_fn=proj_fn)
+    args_ = (d["q"], d["q_rope"], d["k"], d["v"], d["kpe"], d["cu_seqlens"], w.scale, d["w_o"])
+    stream = torch.cuda.current_stream(dev)
+
+    def sync_all():
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    def timed(fn, n):
+        sync_all()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        sync_all()
+        return reduce_max(e0.elapsed_time(e1) / n, world, dev)
+
+    for _ in range(warmup):
+        tp.step(*args_)
+    step_ms = timed(lambda: tp.step(*args_), steps)
+    dec_ms = timed(lambda: decode_fn(*args_[:7]), steps)
+    o2 = out.reshape(B * S, sh.heads * w.d_v)
+    proj_ms = timed(lambda: proj_fn(o2, d["w_o"]), steps)
+    ar_ms = timed(lambda: tp.allreduce_fn(y), steps)
+    if lkv.check_device() != 0:
+        raise RuntimeError("device error in the group-axis TP step")
+    return {"workload": w.name, "tp": world, "groups_per_rank": sh.groups, "heads_per_rank": sh.heads,
+            "d_model": TP_D_MODEL, "scaling": "strong", "steps": steps,
+            "tokens_per_s": B * S / (step_ms * 1e-3), "ms_per_step": step_ms,
+            "decode_ms": dec_ms, "projection_ms": proj_ms, "allreduce_ms": ar_ms,
+            "allreduce_bytes": B * S * TP_D_MODEL * 4,
+            "collective": "torch.distributed all_reduce (NCCL) of the fp32 partial projection" if world > 1
+            else "none (one rank)"}
 
 
 def time_flushed(decode, args_, stream, flush, iters: int):
@@ -548,6 +646,10 @@ def bench_gpu(args, rank, world, local_rank):
         names = [n for n in SIDE_WORKLOADS if n != w.name]
         side = bench_side_workloads(lkv, dev, names, args.side_iters, args.side_cpu_budget)
 
+    # Group-axis TP of the GQLA step over all ranks (every rank takes the same collective steps).
+    del d
+    tp_res = bench_tp(lkv, dev, rank, world, args.tp_steps, 3) if args.tp_steps > 0 else None
+
     tokens = B * S * world
     cache_bytes, io_bytes, flops = workload_accounting(w, lengths)
     res = None
@@ -600,7 +702,7 @@ def bench_gpu(args, rank, world, local_rank):
                                                  flops / (NOMINAL_PEAKS["bf16_tflops"] * 1e12)) / dec_s},
                          "roofline_ms": max(t_hbm, t_tc) * 1e3,
                          "frac_of_step_roofline": max(t_hbm, t_tc) * 1e3 / ms,
-                         "kernel": "decode_tc_kernel + split combine (one lkv_*_decode call)",
+                         "kernel": decode_kernel_name(w) + " + split combine (one lkv_*_decode call)",
                          "algorithmic_bytes": alg_bytes, "algorithmic_flops": flops},
             "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                     "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms,
@@ -609,6 +711,7 @@ def bench_gpu(args, rank, world, local_rank):
             "gpu_launches": launches_per_step * args.steps,
             "clocks": sampler.summary() if sampler else None,
             "workloads": side,
+            "tp": tp_res,
         }
     if world > 1:
         import torch.distributed as dist
@@ -689,6 +792,8 @@ def main():
                     help="calls per workload for the flushed per-workload timings (0: skip them)")
     ap.add_argument("--side-cpu-budget", type=float, default=1.5,
                     help="seconds of CPU-oracle work per side workload")
+    ap.add_argument("--tp-steps", type=int, default=20,
+                    help="timed steps of the group-axis TP workload on all ranks (0: skip it)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

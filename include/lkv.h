@@ -179,6 +179,25 @@ lkv_status lkv_gta_group_decode(const void* q, const void* q_rope, const void* k
                                 lkv_stream_t stream);
 
 /*
+ * GTA decode over FP8 cache rows (the row format of lkv_fp8_cache_row_bytes below, with
+ * r = g * d_h): the tied state of group j is the dequantised columns [128 j, 128 j + 128) of the
+ * row's latent, e4m3(code) * s, used as key (with the row's bf16 RoPE key) and as value, exactly as
+ * lkv_gta_group_decode uses its bf16 tied rows.  FP8 halves the bytes of the tied states (the pages
+ * run their latent models in FP8 for serving: Grouped Latent Attention article, section on the
+ * GLA-vs-MLA decoding test).
+ *   cache  [cache_rows] FP8 rows of cache_row_stride_bytes (a multiple of 16), 16-byte aligned
+ *   q, q_rope, cu_seqlens, out, lse, workspace: as lkv_gta_group_decode (bf16); the workspace size
+ *          is lkv_group_decode_workspace_size with kind 3.
+ * Implemented: d_h = 128, d_rope = 64, g * d_h <= 1024, s_q * h_q / g <= 64 (LKV_ERR_UNSUPPORTED
+ * otherwise).  Rows past a unit's keys are never read as values (their codes are not converted).
+ */
+lkv_status lkv_gta_group_decode_fp8(const void* q, const void* q_rope, const void* cache,
+                                    int64_t cache_row_stride_bytes, int64_t cache_rows,
+                                    const int32_t* cu_seqlens, int batch, int s_q, int h_q, int g, int d_h,
+                                    int d_rope, float scale, void* out, float* lse, void* workspace,
+                                    size_t workspace_bytes, lkv_stream_t stream);
+
+/*
  * GQLA grouped decode that allocates nothing and takes no workspace.
  *
  * No counterpart on the source pages.  It serves callers that cannot allocate device memory
@@ -223,14 +242,15 @@ lkv_status lkv_latent_cache_append(const void* new_rows, int64_t new_row_stride_
                                    lkv_stream_t stream);
 
 /*
- * Output projection y = o W_O (bf16 operands, fp32 accumulation; cuBLAS, as the other projections).
+ * Output projection y = o W_O (bf16 operands, fp32 accumulation; the tensor-core GEMM of the other
+ * projections).
  *   o    [n_tok, k] bf16 row-major: the heads' attention outputs side by side (k = heads * d_v)
  *   w_o  [k, d_model] bf16 row-major
  *   y    [n_tok, d_model], bf16 (out_dtype LKV_BF16) or fp32 (LKV_FP32)
  * With the heads split along the group axis across GPUs (GQLA explainer, section 2, GQA path), each
  * GPU passes its heads' columns of o and the matching row block of W_O and gets a partial y; the sum
- * over GPUs is the full projection.  LKV_ERR_INVALID_ARG for NULL pointers, non-positive sizes or
- * another out_dtype; LKV_ERR_UNSUPPORTED if cuBLAS cannot be opened.
+ * over GPUs is the full projection.  LKV_ERR_INVALID_ARG for NULL pointers, non-positive sizes,
+ * another out_dtype, o or w_o not 16-byte aligned, or k or d_model not a multiple of 8.
  */
 lkv_status lkv_output_projection(const void* o, const void* w_o, void* y, int n_tok, int k, int d_model,
                                  int out_dtype, lkv_stream_t stream);
@@ -240,11 +260,13 @@ lkv_status lkv_output_projection(const void* o, const void* w_o, void* y, int n_
  * section on the GLA-vs-MLA decoding test -- but fix no format; this is the library's reading).
  * One row per token of lkv_fp8_cache_row_bytes(r, d_rope) = r + 16 + 2*d_rope bytes:
  *   bytes [0, r)          e4m3 codes of the latent row (OCP E4M3: bias 7, largest finite 448)
- *   bytes [r, r + 4)      fp32 scale s = max|latent row| / 448 (0 for an all-zero row)
+ *   bytes [r, r + 4)      fp32 scale s: the smallest power of two with max|latent row| / s <= 448
+ *                         (0 for an all-zero row)
  *   bytes [r + 4, r + 16) zero
  *   bytes [r + 16, ...)   the bf16 RoPE key, copied unchanged
- * The dequantised latent is e4m3(code) * s.  Codes are taken in fp32: y = x / s (IEEE division),
- * clamped to [-448, 448], rounded to the nearest e4m3 value with ties to the even code.
+ * The dequantised latent is e4m3(code) * s, exact in bf16 (a power of two times a 4-bit
+ * significand).  Codes: y = x / s (exact), rounded to the nearest e4m3 value with ties to the even
+ * code.
  * lkv_fp8_cache_row_bytes returns 0 unless r is a multiple of 16 in [16, 1024] and d_rope a
  * non-negative multiple of 8 (host-only, no CUDA call).
  */
@@ -311,10 +333,9 @@ lkv_status lkv_selftest_wait_timeout(uint64_t limit_ns, lkv_stream_t stream);
  * absorbed path folds W_UK into the query and applies W_UV after attention; the GQA path expands
  * the latent into per-group keys and values).  j(h) = h / (h_q / groups).  bf16 operands, fp32
  * accumulation, bf16 results (dtype must be LKV_BF16, else LKV_ERR_UNSUPPORTED); all arrays are
- * contiguous device arrays unless a row stride is given.  These are plain GEMMs run by cuBLAS,
- * which the library opens (dlopen "libcublas.so.12") at the first projection call: LKV_ERR_UNSUPPORTED
- * if it cannot be loaded.  The first call on a device creates that device's cuBLAS handle, which
- * allocates cuBLAS's own workspace; later calls allocate nothing.  Asynchronous on `stream`.
+ * contiguous device arrays unless a row stride is given.  Each call is one launch of the library's
+ * tensor-core GEMM (tcgen05, TMA-fed, persistent over 128-row tiles); nothing is allocated.
+ * Asynchronous on `stream`; a bounded wait that gives up is recorded in the device error word.
  *
  * lkv_absorb_query:    q [n_tok, h_q, d_h], w_uk [groups, r, d_h] -> q_abs [n_tok, h_q, r],
  *                      q_abs[t, h, :] = w_uk[j(h)] q[t, h, :]
@@ -322,8 +343,10 @@ lkv_status lkv_selftest_wait_timeout(uint64_t limit_ns, lkv_stream_t stream);
  *                      out[t, h, :] = w_uv[j(h)]^T o_lat[t, h, :]
  * lkv_expand_latent:   c [n_rows, r] (row stride c_row_stride elements >= r), w [groups, r, d]
  *                      -> x [n_rows, groups, d],  x[t, j, :] = c[t, :] w[j]
- * Errors: LKV_ERR_INVALID_ARG for NULL pointers, non-positive sizes, h_q % groups != 0 or
- * leading dimensions beyond int range (checked before any launch); LKV_ERR_CUDA if cuBLAS fails.
+ * Errors (checked before any launch): LKV_ERR_INVALID_ARG for NULL pointers, non-positive sizes,
+ * h_q % groups != 0, leading dimensions beyond int range, operand pointers not 16-byte aligned, or
+ * an operand row whose length or stride (d_h for absorb; r and d_v for unabsorb; c_row_stride and
+ * d for expand) is not a multiple of 8 elements; LKV_ERR_CUDA if the launch fails.
  */
 lkv_status lkv_absorb_query(const void* q, const void* w_uk, void* q_abs, int n_tok, int h_q, int groups,
                             int d_h, int r, int dtype, lkv_stream_t stream);

@@ -57,6 +57,8 @@ _gla = _sig("lkv_gla_group_decode", _i32, _vp, _vp, _vp, _i64, _vp, _i64, _i64, 
             _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp)
 _gta = _sig("lkv_gta_group_decode", _i32, _vp, _vp, _vp, _i64, _vp, _i64, _i64, _vp,
             _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _vp, _vp, _sz, _vp)
+_gta_fp8 = _sig("lkv_gta_group_decode_fp8", _i32, _vp, _vp, _vp, _i64, _i64, _vp, _i32, _i32, _i32, _i32,
+                _i32, _i32, _f32, _vp, _vp, _vp, _sz, _vp)
 _fp8_row_bytes = _sig("lkv_fp8_cache_row_bytes", _sz, _i32, _i32)
 _quant_fp8 = _sig("lkv_quantize_latent_fp8", _i32, _vp, _i64, _vp, _i64, _i64, _i32, _i32, _vp)
 _append_fp8 = _sig("lkv_latent_cache_append_fp8", _i32, _vp, _i64, _vp, _i64, _i64, _i32, _i32, _vp,
@@ -82,7 +84,7 @@ EXPORTED = ["lkv_version", "lkv_status_string", "lkv_plan_ranges", "lkv_mla_deco
             "lkv_gqla_group_decode_noalloc", "lkv_absorb_query", "lkv_unabsorb_output",
             "lkv_expand_latent", "lkv_gta_group_decode", "lkv_fp8_cache_row_bytes",
             "lkv_quantize_latent_fp8", "lkv_latent_cache_append_fp8", "lkv_output_projection",
-            "lkv_check_stream"]
+            "lkv_check_stream", "lkv_gta_group_decode_fp8"]
 
 
 class LkvError(RuntimeError):
@@ -269,6 +271,32 @@ def gta_group_decode(q, q_rope, kv, kpe, g, cu_seqlens, scale, out=None, lse=Non
     _ck(_gta(_ptr(q), _ptr(q_rope), _ptr(kv), _row_stride(kv), _ptr(kpe), _row_stride(kpe), kv.shape[0],
              _ptr(cu_seqlens), B, s_q, h_q, g, d_h, d_r, float(scale), _dtype_code(q), _ptr(out), _ptr(lse),
              _ptr(workspace), ws_bytes, _stream(stream)), "lkv_gta_group_decode")
+    return out, lse
+
+
+def gta_group_decode_fp8(q, q_rope, cache, g, cu_seqlens, scale, out=None, lse=None, workspace=None,
+                         stream=None):
+    """GTA decode over FP8 cache rows.  q [B,s_q,h_q,d_h] and q_rope [B,s_q,h_q,d_R] bf16; cache
+    [rows, >= fp8_cache_row_bytes(g*d_h, d_R)] uint8 (row stride a multiple of 16 bytes)."""
+    _same_dtype(q, q_rope=q_rope, out=out)
+    if q.dtype != torch.bfloat16 or cache.dtype != torch.uint8:
+        raise TypeError("gta_group_decode_fp8 takes a bf16 query and a uint8 FP8 cache")
+    B, s_q, h_q, d_h = q.shape
+    d_r = q_rope.shape[-1]
+    dev = q.device
+    if cache.stride(-1) != 1:
+        raise ValueError("cache rows must be contiguous")
+    if out is None:
+        out = torch.empty((B, s_q, h_q, d_h), dtype=q.dtype, device=dev)
+    if lse is None:
+        lse = torch.empty((B, s_q, h_q), dtype=torch.float32, device=dev)
+    if workspace is None:
+        workspace = _alloc_ws(group_decode_workspace_size(KIND_GTA, B, s_q, h_q, g, d_h, _num_sms(dev)), dev)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    _contig(q, q_rope, out, lse)
+    _ck(_gta_fp8(_ptr(q), _ptr(q_rope), _ptr(cache), cache.stride(0), cache.shape[0], _ptr(cu_seqlens), B, s_q,
+                 h_q, g, d_h, d_r, float(scale), _ptr(out), _ptr(lse), _ptr(workspace), ws_bytes, _stream(stream)),
+        "lkv_gta_group_decode_fp8")
     return out, lse
 
 

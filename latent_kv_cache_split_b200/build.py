@@ -3,10 +3,9 @@
     python latent_kv_cache_split_b200/build.py [--verbose]
 
 The library is three translation units: csrc/lkv_api.cu (the decode path; it includes the kernel
-headers), csrc/lkv_proj.cu (the projections, which open cuBLAS at run time) and csrc/lkv_fp8.cu
-(FP8 latent cache rows).  All link the
-static CUDA runtime, so the .so only needs the NVIDIA driver at run time (and cuBLAS for the
-projections).
+headers), csrc/lkv_proj.cu (the projections, on the tensor-core GEMM of csrc/lkv_gemm.cuh) and
+csrc/lkv_fp8.cu (FP8 latent cache rows).  All link the static CUDA runtime, so the .so only needs
+the NVIDIA driver at run time.
 """
 from __future__ import annotations
 
@@ -20,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "liblkv.so")
 SOURCES = ["lkv_api.cu", "lkv_proj.cu", "lkv_fp8.cu"]
-HEADERS = ["lkv_ptx.cuh", "lkv_sched.cuh", "lkv_decode_tc.cuh", "lkv_mla_pair.cuh", "lkv_aux.cuh", "lkv_tma_host.h"]
+HEADERS = ["lkv_ptx.cuh", "lkv_sched.cuh", "lkv_decode_tc.cuh", "lkv_mla_pair.cuh", "lkv_gemm.cuh", "lkv_aux.cuh", "lkv_tma_host.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -40,8 +40,9 @@ unsigned long long wait_limit_ns() {
 }
 
 constexpr size_t tc_smem_bytes(int mode) {
-  return mode == MODE_GQLA ? ModeCfg<MODE_GQLA>::kSmemBytes
+  return mode == MODE_GQLA   ? ModeCfg<MODE_GQLA>::kSmemBytes
          : mode == MODE_GTA  ? ModeCfg<MODE_GTA>::kSmemBytes
+         : mode == MODE_GTA8 ? ModeCfg<MODE_GTA8>::kSmemBytes
                              : ModeCfg<MODE_GLA>::kSmemBytes;
 }
 
@@ -62,6 +63,8 @@ lkv_status device_state(DeviceState** out) {
                              static_cast<int>(tc_smem_bytes(MODE_GLA))) != cudaSuccess ||
         cudaFuncSetAttribute(decode_tc_kernel<MODE_GTA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(tc_smem_bytes(MODE_GTA))) != cudaSuccess ||
+        cudaFuncSetAttribute(decode_tc_kernel<MODE_GTA8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(tc_smem_bytes(MODE_GTA8))) != cudaSuccess ||
         cudaFuncSetAttribute(mla_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(kPairSmemBytes)) != cudaSuccess)
       return LKV_ERR_CUDA;
@@ -149,6 +152,8 @@ lkv_status run_tc(TcLaunch& L, const DeviceState& d, cudaStream_t stream) {
     e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<MODE_GQLA>, L.map_a, L.map_r, L.map_v, L.p);
   } else if (L.mode == MODE_GTA) {
     e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<MODE_GTA>, L.map_a, L.map_r, L.map_v, L.p);
+  } else if (L.mode == MODE_GTA8) {
+    e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<MODE_GTA8>, L.map_a, L.map_r, L.map_v, L.p);
   } else {
     e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<MODE_GLA>, L.map_a, L.map_r, L.map_v, L.p);
   }
@@ -206,6 +211,17 @@ lkv_status lkv_internal_error_word(int** err) {
   DeviceState* d;
   const lkv_status st = device_state(&d);
   if (st == LKV_OK) *err = d->err;
+  return st;
+}
+// The same, with the device's SM count and the bounded-wait limit of the kernels.
+lkv_status lkv_internal_device_info(int** err, int* num_sms, unsigned long long* wait_ns) {
+  DeviceState* d;
+  const lkv_status st = device_state(&d);
+  if (st == LKV_OK) {
+    *err = d->err;
+    *num_sms = d->num_sms;
+    *wait_ns = wait_limit_ns();
+  }
   return st;
 }
 
@@ -342,14 +358,14 @@ lkv_status lkv_mla_absorbed_decode(const void* q_nope_abs, const void* q_rope, c
   const WsLayout w = ws_layout(P, h_q, r_kv);
   if (!workspace || !al16(workspace) || workspace_bytes < w.total) return LKV_ERR_WORKSPACE;
   // Query rows (b, i, h) as 2-D [batch * s_q * h_q, width] maps in 64-row boxes (one CTA's heads);
-  // cache rows in 128-row boxes for QK (one CTA's keys of a 256-key tile) and 64-row boxes for PV.
+  // cache rows in 128-row boxes for QK (one CTA's keys of a 256-key tile) and PV (a value chunk).
   const uint64_t qrows = static_cast<uint64_t>(batch) * s_q * h_q;
   CUtensorMap maps[5];
   if (!make_tmap_bf16(&maps[0], q_nope_abs, r_kv, qrows, static_cast<uint64_t>(r_kv) * 2, 64, 64) ||
       !make_tmap_bf16(&maps[1], q_rope, d_rope, qrows, static_cast<uint64_t>(d_rope) * 2, 64, 64) ||
       !make_tmap_bf16(&maps[2], ckv, r_kv, cache_rows, ckv_row_stride * 2, 64, 128) ||
       !make_tmap_bf16(&maps[3], kpe, d_rope, cache_rows, kpe_row_stride * 2, 64, 128) ||
-      !make_tmap_bf16(&maps[4], ckv, r_kv, cache_rows, ckv_row_stride * 2, 64, 64))
+      !make_tmap_bf16(&maps[4], ckv, r_kv, cache_rows, ckv_row_stride * 2, 64, 128))
     return LKV_ERR_CUDA;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   TcParams p;
@@ -529,6 +545,71 @@ lkv_status lkv_gta_group_decode(const void* q, const void* q_rope, const void* k
   p.P = P;
   p.err = d->err;
   p.wait_limit_ns = wait_limit_ns();
+  L.units_per_req = g;
+  L.per_query_units = 0;
+  return run_tc(L, *d, reinterpret_cast<cudaStream_t>(stream));
+}
+
+lkv_status lkv_gta_group_decode_fp8(const void* q, const void* q_rope, const void* cache,
+                                    int64_t cache_row_stride_bytes, int64_t cache_rows,
+                                    const int32_t* cu_seqlens, int batch, int s_q, int h_q, int g, int d_h,
+                                    int d_rope, float scale, void* out, float* lse, void* workspace,
+                                    size_t workspace_bytes, lkv_stream_t stream) {
+  lkv_status st = common_checks(q, q_rope, cu_seqlens, out, lse, batch, s_q, h_q, g, d_rope,
+                                cache_rows, LKV_BF16, scale);
+  if (st != LKV_OK) return st;
+  if (!cache || d_h <= 0) return LKV_ERR_INVALID_ARG;
+  const int hpg = h_q / g;
+  const int r = g * d_h;
+  // the converter warps are the softmax slots a unit of <= 64 rows leaves free
+  if (d_h != 128 || d_rope != 64 || r > 1024 || s_q * hpg > 64) return LKV_ERR_UNSUPPORTED;
+  const size_t row_bytes = lkv_fp8_cache_row_bytes(r, d_rope);
+  if (row_bytes == 0 || cache_row_stride_bytes < static_cast<int64_t>(row_bytes) || cache_row_stride_bytes % 16 ||
+      !al16(q) || !al16(q_rope) || !al16(cache) || !al16(out))
+    return LKV_ERR_INVALID_ARG;
+  DeviceState* d;
+  if ((st = device_state(&d)) != LKV_OK) return st;
+  const int P = plan_ranges(1, batch, s_q, g, d->num_sms);
+  const int R = s_q * hpg;
+  const WsLayout w = ws_layout(P, R, d_h);
+  if (!workspace || !al16(workspace) || workspace_bytes < w.total) return LKV_ERR_WORKSPACE;
+  // The row's fields as three maps: the codes (bytes, 128 per group), the scale with its 12 zero
+  // bytes (fp32, 4 per row) and the RoPE key (bf16, 64 per row), 128-row boxes.
+  TcLaunch L;
+  L.mode = MODE_GTA8;
+  constexpr int TN = ModeCfg<MODE_GTA8>::kTile;
+  const uint64_t rs = static_cast<uint64_t>(cache_row_stride_bytes);
+  if (!make_tmap_2d(&L.map_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, cache, row_bytes, cache_rows, rs, 128, TN,
+                    CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_tmap_2d(&L.map_v, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, cache, row_bytes / 4, cache_rows, rs, 4, TN,
+                    CU_TENSOR_MAP_SWIZZLE_NONE) ||
+      !make_tmap_bf16(&L.map_r, cache, row_bytes / 2, cache_rows, rs, 64, TN))
+    return LKV_ERR_CUDA;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  TcParams& p = L.p;
+  p.q_nope = static_cast<const __nv_bfloat16*>(q);
+  p.q_rope = static_cast<const __nv_bfloat16*>(q_rope);
+  p.dq = d_h;
+  p.cu = cu_seqlens;
+  p.B = batch;
+  p.s_q = s_q;
+  p.h_q = h_q;
+  p.G = g;
+  p.hpg = hpg;
+  p.R = R;
+  p.sl2 = scale * 1.4426950408889634f;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.lse = lse;
+  p.dv_total = d_h;
+  p.seg_info = reinterpret_cast<int*>(ws + w.seg);
+  p.part_lse = reinterpret_cast<float*>(ws + w.lse);
+  p.part_o = reinterpret_cast<float*>(ws + w.o);
+  p.rmax = R;
+  p.P = P;
+  p.err = d->err;
+  p.wait_limit_ns = wait_limit_ns();
+  p.fp8_scale_col = r / 4;
+  p.fp8_rope_col = (r + 16) / 2;
   L.units_per_req = g;
   L.per_query_units = 0;
   return run_tc(L, *d, reinterpret_cast<cudaStream_t>(stream));

@@ -18,9 +18,16 @@
 //
 // TMEM columns: O [0, DV) | S [DV, DV+T) | P0, P1 [DV+T, DV+2T) | Q [DV+2T, ...) for T keys/tile.
 // P is double buffered so the softmax of tile n+1 never waits for the PV of tile n.
+//
+// GTA over FP8 cache rows (MODE_GTA8): the producer loads the group's e4m3 codes, the tokens'
+// power-of-two scales and the RoPE key; warps 6, 7, 10 and 11 (idle in the other modes when a unit
+// has at most 64 rows) convert the codes into the bf16 tied state of the stage, exactly (a 4-bit
+// significand times a power of two), after which the tile is used as in MODE_GTA.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 #include "lkv_ptx.cuh"
 #include "lkv_sched.cuh"
 #include "../../include/lkv.h"
@@ -40,11 +47,12 @@ __device__ __forceinline__ float bf16x2_sum(uint32_t w) {
 
 // MODE_GTA: grouped-tied attention, the GQLA shapes with K_j = V_j (one tied state per group).
 // (Mode 0, the MLA absorbed path, runs in lkv_mla_pair.cuh; the numbering keeps wait-site codes stable.)
-enum DecodeMode { MODE_GQLA = 1, MODE_GLA = 2, MODE_GTA = 3 };
+// MODE_GTA8: MODE_GTA over FP8 (e4m3) cache rows.
+enum DecodeMode { MODE_GQLA = 1, MODE_GLA = 2, MODE_GTA = 3, MODE_GTA8 = 5 };
 
 // Wait sites (added to LKV_SITE_WAIT_BASE in the error word).
 enum WaitSite {
-  W_EMPTY = 1, W_FULL, W_SFREE, W_QREADY, W_PFULL, W_OFREE, W_SFULL, W_ODONE, W_DRAIN = 11, W_XCHG = 13
+  W_EMPTY = 1, W_FULL, W_SFREE, W_QREADY, W_PFULL, W_OFREE, W_SFULL, W_ODONE, W_DRAIN = 11, W_XCHG = 13, W_CONV
 };
 
 struct TcParams {
@@ -64,11 +72,15 @@ struct TcParams {
   int P;
   int* err;
   unsigned long long wait_limit_ns;
+  int fp8_scale_col;            // MODE_GTA8: column (4-byte units) of a row's scale
+  int fp8_rope_col;             // MODE_GTA8: column (bf16 units) of a row's RoPE key
 };
 
 template <int kMode>
 struct ModeCfg {
-  static constexpr bool kHead128 = (kMode == MODE_GQLA || kMode == MODE_GTA);  // d_h = 128 groups
+  static constexpr bool kFp8 = (kMode == MODE_GTA8);
+  static constexpr bool kTied128 = (kMode == MODE_GTA || kMode == MODE_GTA8);  // one tied 128-wide state
+  static constexpr bool kHead128 = (kMode == MODE_GQLA || kTied128);  // d_h = 128 groups
   // Keys per tile.  GQLA runs 128-key tiles so that every QK UMMA is N = 128 (one issuing
   // thread then keeps the tensor pipe at full rate); GLA keeps 64-key tiles because a
   // 128-column S tile would not fit next to its 256-column O accumulator and resident Q.
@@ -79,12 +91,18 @@ struct ModeCfg {
   static constexpr bool kSplitKV = (kMode == MODE_GQLA);
   static constexpr int kKBoxes = kHead128 ? 2 : 4;  // 64-column boxes of the non-RoPE key per stage
   static constexpr int kRopeBoxBytes = kBoxBytes;  // the whole 64-column RoPE key
-  static constexpr int kStageBytes = kKBoxes * kBoxBytes + kRopeBoxBytes;  // K ring (or whole tile)
+  // FP8 stages also hold the codes (kTile rows x 128 bytes) and scales (kTile rows x 16 bytes) that
+  // the bf16 state is converted from
+  static constexpr int kCodesOff = kKBoxes * kBoxBytes + kRopeBoxBytes;
+  static constexpr int kScalesOff = kCodesOff + kTile * 128;
+  static constexpr int kStageBytes = kKBoxes * kBoxBytes + kRopeBoxBytes + (kFp8 ? kTile * (128 + 16) : 0);
+  // bytes the producer's copies bring into a stage
+  static constexpr int kTmaBytes = kFp8 ? kTile * (128 + 16) + kRopeBoxBytes : kStageBytes;
   static constexpr int kVStageBytes = 2 * kBoxBytes;                  // V ring (GQLA)
   static constexpr int kDV = kHead128 ? 128 : 256;  // value columns per CTA
   // GTA holds a stage from its load to its PV (K = V), so it gets the ring depth that GQLA
   // splits between its K ring (2) and V ring (3)
-  static constexpr int kStages = (kMode == MODE_GQLA) ? 2 : (kMode == MODE_GTA ? 4 : 5);
+  static constexpr int kStages = (kMode == MODE_GQLA) ? 2 : (kMode == MODE_GTA ? 4 : (kFp8 ? 3 : 5));
   static constexpr int kVStages = kSplitKV ? 3 : 1;
   static constexpr int kNope = kHead128 ? 2 : 4;    // non-RoPE Q boxes (in TMEM)
   static constexpr int kRopeBox = kKBoxes;          // stage box holding k_rope
@@ -107,14 +125,25 @@ static_assert(ModeCfg<MODE_GLA>::kSmemBytes <= 232448, "shared memory budget");
 static_assert(ModeCfg<MODE_GQLA>::kSmemBytes <= 232448, "shared memory budget");
 static_assert(ModeCfg<MODE_GTA>::kSmemBytes <= 232448, "shared memory budget");
 static_assert(ModeCfg<MODE_GTA>::kStageBytes == 3 * ModeCfg<MODE_GTA>::kBoxBytes, "GTA stage: tied state + RoPE key");
+static_assert(ModeCfg<MODE_GTA8>::Q0 + 32 * ModeCfg<MODE_GTA8>::kNope <= kTmemCols, "TMEM budget");
+static_assert(ModeCfg<MODE_GTA8>::kSmemBytes <= 232448, "shared memory budget");
+static_assert(ModeCfg<MODE_GTA8>::kScalesOff % 1024 == 0 && ModeCfg<MODE_GTA8>::kStageBytes % 1024 == 0,
+              "FP8 stage fields on 1024-byte boundaries");
+
+// Two e4m3 codes (the low byte first) times a power-of-two scale, packed as bf16x2: exact, since
+// every e4m3 value is an f16 normal (or zero) with a 4-bit significand.
+__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two_codes, float s) {
+  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_codes & 0xffffu), __NV_E4M3);
+  const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+  return pack_bf16x2(f.x * s, f.y * s);
+}
 
 // Advance a shared-memory descriptor by a byte offset (start-address field, 16-byte units).
-__device__ __forceinline__ uint64_t desc_add(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
-
 template <int kStagesT, int kVStagesT>
 struct __align__(16) TcSmem {
   uint64_t full[kStagesT];
   uint64_t empty[kStagesT];
+  uint64_t conv[kStagesT];          // MODE_GTA8: the stage's codes are converted to bf16
   uint64_t vfull[kVStagesT];
   uint64_t vempty[kVStagesT];
   uint64_t s_full, s_free;         // the S buffer
@@ -248,6 +277,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     for (int s = 0; s < KS; ++s) {
       mbar_init(smem_u32(&sm.full[s]), 1);
       mbar_init(smem_u32(&sm.empty[s]), 1);
+      mbar_init(smem_u32(&sm.conv[s]), 4);  // one arrival per converter warp
     }
     for (int s = 0; s < VS; ++s) {
       mbar_init(smem_u32(&sm.vfull[s]), 1);
@@ -283,7 +313,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       p.seg_info[2 * range + 1] = -1;
       tma_prefetch_desc(&map_a);
       tma_prefetch_desc(&map_r);
-      if (kMode == MODE_GQLA) tma_prefetch_desc(&map_v);
+      if (kMode == MODE_GQLA || kMode == MODE_GTA8) tma_prefetch_desc(&map_v);
     }
   }
   if (warp == 1) {
@@ -307,7 +337,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 0) {
     // ============================================================ TMA producer
     if (lane == 0) {
-      const uint32_t bytes = Cfg::kStageBytes;
+      const uint32_t bytes = Cfg::kTmaBytes;
       SegCursor cur = cur0;
       Segment sg;
       int n = 0, nv = 0;   // K (or whole) tiles and V tiles issued (a CTA's tile count fits an int)
@@ -349,6 +379,12 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             tma_load_2d(dst, &map_a, fb, c0, row);
             tma_load_2d(dst + kBoxBytes, &map_a, fb, c0 + 64, row);
             tma_load_2d(dst + 2 * kBoxBytes, &map_r, fb, 0, row);
+          } else if constexpr (kMode == MODE_GTA8) {
+            // the group's 128 codes per row, the rows' scales (with their 12 zero bytes) and the
+            // shared RoPE key; the converter warps fill the bf16 state at the stage's start
+            tma_load_2d(dst + Cfg::kCodesOff, &map_a, fb, 128 * sg.k, row);
+            tma_load_2d(dst + Cfg::kScalesOff, &map_v, fb, p.fp8_scale_col, row);
+            tma_load_2d(dst + 2 * kBoxBytes, &map_r, fb, p.fp8_rope_col, row);
           } else {
             const int c0 = 256 * sg.k;
             for (int bx = 0; bx < 4; ++bx) tma_load_2d(dst + bx * kBoxBytes, &map_a, fb, c0 + 64 * bx, row);
@@ -388,7 +424,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
             const int st = static_cast<int>(n % KS);
             // one S buffer: tile n's QK waits until the softmax has read tile n-1's scores
-            if (!mbar_wait(smem_u32(&sm.full[st]), static_cast<uint32_t>((n / KS) & 1), wc, LKV_WAIT(W_FULL)) ||
+            const uint32_t kbar = Cfg::kFp8 ? smem_u32(&sm.conv[st]) : smem_u32(&sm.full[st]);
+            if (!mbar_wait(kbar, static_cast<uint32_t>((n / KS) & 1), wc, LKV_WAIT(Cfg::kFp8 ? W_CONV : W_FULL)) ||
                 (n >= 1 && !mbar_wait(smem_u32(&sm.s_free), static_cast<uint32_t>((n - 1) & 1), wc, LKV_WAIT(W_SFREE))) ||
                 (t == sg.tile_lo &&
                  !mbar_wait(smem_u32(&sm.q_ready), static_cast<uint32_t>(seg & 1), wc, LKV_WAIT(W_QREADY)))) {
@@ -448,6 +485,49 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint32_t zero = 0;
       const WaitCtl dc{&zero, p.err, p.wait_limit_ns};
       mbar_wait(smem_u32(&sm.drain), 0, dc, LKV_WAIT(W_DRAIN));
+    }
+  } else if (Cfg::kFp8 && warp >= 4 && warp < 12 && ((warp - 4) & 3) >= 2) {
+    // ============================================================ FP8 converters (MODE_GTA8)
+    // Thread `row` turns key row `row` of each tile from 128 e4m3 codes (128-byte swizzled box)
+    // into 128 bf16 values in the stage's two 64-column state boxes (the layout a TMA copy with
+    // 128-byte swizzle writes).  Rows past the unit's keys become zeros.
+    const int row = 64 * ((warp - 4) >> 2) + 32 * (((warp - 4) & 3) - 2) + lane;
+    SegCursor cur = cur0;
+    Segment sg;
+    int n = 0;
+    bool ok = true;
+    while (ok && next_seg(cur, sg)) {
+      for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
+        const int st = static_cast<int>(n % KS);
+        if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&sm.full[st]), static_cast<uint32_t>((n / KS) & 1), wc,
+                                               LKV_WAIT(W_FULL)))) {
+          ok = false;
+          break;
+        }
+        uint8_t* sb = dsm + st * kStageBytes;
+        const bool valid = t * TN + row < sg.keys;
+        const float sc = valid ? *reinterpret_cast<const float*>(sb + Cfg::kScalesOff + row * 16) : 0.f;
+        const int sw = row & 7;
+        const uint8_t* crow = sb + Cfg::kCodesOff + row * 128;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {  // codes 16 j .. 16 j + 15 -> bf16 chunks 2 (j % 4), +1 of box j / 4
+          const uint4 c = valid ? *reinterpret_cast<const uint4*>(crow + ((j ^ sw) << 4)) : make_uint4(0u, 0u, 0u, 0u);
+          const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+          uint32_t o[8];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            o[2 * k] = e4m3x2_to_bf16x2(cw[k], sc);
+            o[2 * k + 1] = e4m3x2_to_bf16x2(cw[k] >> 16, sc);
+          }
+          uint8_t* box = sb + (j >> 2) * kBoxBytes + row * 128;
+          const int cc = 2 * (j & 3);
+          *reinterpret_cast<uint4*>(box + ((cc ^ sw) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(box + (((cc + 1) ^ sw) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sm.conv[st]));
+      }
     }
   } else if (warp >= 4 && warp < 12 && ((warp - 4) & 3) < n_row_warps) {
     // ============================================================ softmax / epilogue
@@ -620,7 +700,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
         }
       }
-      if (key0 + TN > sg.keys) {
+      if (!Cfg::kFp8 && key0 + TN > sg.keys) {
+        // (The FP8 converters write zeros there themselves.)
         // Rows past the unit's last key belong to another request or to unwritten cache:
         // their P is 0, but 0 * NaN would still poison O, so clear those V rows first.
         const int first = sg.keys - key0;

@@ -4,13 +4,15 @@
 // section on the GLA-vs-MLA decoding test) but fix no cache format.  The format here: one row per
 // token of row_bytes = r + 16 + 2 * d_rope bytes,
 //   [0, r)            e4m3 codes of the latent c_KV[t, :]
-//   [r, r + 4)        fp32 scale s_t = amax_t / 448 (amax_t = max |c_KV[t, :]|; 0 for a zero row)
+//   [r, r + 4)        fp32 scale s_t: the smallest power of two with amax_t / s_t <= 448
+//                     (amax_t = max |c_KV[t, :]|; 0 for a zero row)
 //   [r + 4, r + 16)   zero
 //   [r + 16, ...)     the bf16 RoPE key, unchanged
 // so every field starts on a 16-byte boundary (TMA boxes can address each one) and the dequantised
-// latent is e4m3(code) * s_t.  Codes: y = x / s_t rounded to fp32, clamped to [-448, 448], rounded
-// to the nearest e4m3 value with ties to even (OCP E4M3: bias 7, 3 mantissa bits, largest finite
-// 448, no infinities).
+// latent is e4m3(code) * s_t, exact in bf16 (a power of two times a 4-bit significand), so a decode
+// can dequantise into bf16 tensor-core operands without rounding.  Codes: y = x / s_t (exact),
+// rounded to the nearest e4m3 value with ties to even (OCP E4M3: bias 7, 3 mantissa bits, largest
+// finite 448, no infinities).
 #include <cstdint>
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
@@ -45,6 +47,15 @@ __device__ __forceinline__ void note_error(int* err, int code) {
 }
 
 __device__ __forceinline__ float clamp_e4m3(float y) { return fminf(fmaxf(y, -kE4m3Max), kE4m3Max); }
+
+// The smallest power of two s with amax / s <= 448, for a finite amax > 0: with amax = m * 2^E
+// (m in [0.5, 1)), amax <= 448 * 2^e = 0.875 * 2^(9 + e) first holds at e = E - 9 when m <= 0.875,
+// else at e = E - 8.  frexpf and ldexpf are exact.
+__device__ __forceinline__ float pow2_scale(float amax) {
+  int E;
+  const float m = frexpf(amax, &E);
+  return ldexpf(1.f, m <= 0.875f ? E - 9 : E - 8);
+}
 
 // Loads of one source row into registers: latent chunk lane + 32 k (8 bf16 each) and RoPE chunk
 // `lane` (16 bytes); chunks past the row are left zero.
@@ -97,7 +108,7 @@ __device__ __forceinline__ void store_row(const QuantArgs& a, long long w, int l
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const float scale = __fdiv_rn(amax, kE4m3Max);
+  const float scale = amax > 0.f ? pow2_scale(amax) : 0.f;
 #pragma unroll
   for (int k = 0; k < kMaxChunks; ++k) {
     const int c = lane + 32 * k;

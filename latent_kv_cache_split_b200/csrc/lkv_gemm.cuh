@@ -1,0 +1,273 @@
+// Projection GEMM on the 5th-generation tensor cores: D = A B with bf16 operands, fp32 accumulation
+// in TMEM and a bf16 (or fp32) result, for the projections either side of the decode path (GQLA
+// explainer, section 2 "Methodology": W_UK folded into the query, W_UV after attention, the latent
+// expanded into per-group keys and values; and the output projection after attention).
+//
+// Every projection is written with the large dimension as the MMA's M (rows of A, 128 per tile):
+//   A rows   are K-major (the contraction is the row's unit-stride axis) and addressed through a
+//            3-D tensor map {K, n1, n2}: a tile is a box of b1 x b2 rows (b1 * b2 = 128), which lets a
+//            tile gather the rows of one head group across tokens (q[t, h, :] for h in a group).
+//   B        is either K-major ([N, K] rows, W_UK[j]) or MN-major ([K, N] with unit stride along N,
+//            W_UV[j], the expansion weights, W_O), 3-D {.., .., matrix index}.  The matrix a tile
+//            uses comes from its rows (the head group) or from its columns (the expansion's groups
+//            side by side).
+// A tile is 128 rows x tn columns (tn a multiple of 64, <= 256); the K loop streams 64-wide blocks
+// of A (16 KB) and B (tn x 128 bytes) through a ring of shared-memory stages.
+//
+// Warps: 0 TMA producer; 1 TMEM allocator and MMA issuer; 2-9 epilogue (warp w reads TMEM lane
+// quadrant w % 4, column half (w - 2) / 4).  The kernel is persistent over tiles (grid = SM count at
+// most) and double-buffers the accumulator in TMEM (2 x 256 columns), so a tile's epilogue overlaps
+// the next tile's MMAs.  Every wait is bounded and records its site in the device error word.
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include "lkv_ptx.cuh"
+#include "../../include/lkv.h"
+
+namespace lkv {
+
+constexpr int kGemmThreads = 320;
+constexpr int kGemmStages = 4;
+constexpr int kGemmABytes = 16384;      // 128 rows x 64 K (bf16)
+constexpr int kGemmBBytes = 32768;      // up to 256 N x 64 K (bf16)
+constexpr int kGemmStageBytes = kGemmABytes + kGemmBBytes;
+constexpr size_t kGemmSmemBytes = 1024 + static_cast<size_t>(kGemmStages) * kGemmStageBytes;
+constexpr uint32_t kGemmTmemCols = 512;  // two accumulators of up to 256 columns
+static_assert(kGemmSmemBytes <= 232448 - 1024, "shared memory budget");
+
+// Wait sites of this kernel (added to LKV_SITE_WAIT_BASE in the error word; above the decode kernels').
+enum GemmWaitSite { GW_EMPTY = LKV_SITE_WAIT_BASE + 120, GW_FULL, GW_TEMPTY, GW_TFULL, GW_DRAIN };
+
+struct GemmParams {
+  int k_blocks;       // ceil(K / 64)
+  int tn;             // columns per tile (multiple of 64, <= 256)
+  int n_tiles;        // tiles along the columns
+  int n_valid;        // columns of the result (per group on the group axis)
+  int b1, lg_b1, b2;  // rows of a tile along A's dims 1 and 2 (b1 a power of two, b1 * b2 = 128)
+  int n1, n2;         // A's row extents
+  int t1, t2;         // tiles along A's dims 1 and 2
+  int rows_per_b;     // rows of dim 1 that share one B matrix (heads per group); 0: not row-selected
+  int groups;         // B matrices applied to every row as separate column blocks (else 1)
+  int nb;             // columns of one B matrix when the column axis spans several side by side
+  int b_mn;           // B is MN-major
+  int b_bytes;        // B bytes per stage
+  int out_fp32;
+  int vec_ok;         // every row start and column block is 16-byte aligned
+  long long os1, os2; // result offset (elements) per unit of A's dims 1 and 2
+  long long ocol;     // result column offset per group
+  int total_tiles;
+  void* out;
+  int* err;
+  unsigned long long wait_limit_ns;
+};
+
+struct __align__(8) GemmSmem {
+  uint64_t full[kGemmStages];   // A and B of the stage landed
+  uint64_t empty[kGemmStages];  // the MMAs reading the stage are done
+  uint64_t tfull[2];            // accumulator b holds a finished tile
+  uint64_t tempty[2];           // the 8 epilogue warps read accumulator b
+  uint64_t drain;               // every MMA issued is complete
+  uint32_t tmem_base;
+  uint32_t abort;
+  uint32_t zero;                // abort flag of the drain waits: never set
+  int fills, consumed;
+};
+
+struct GemmTile {
+  int nt, i1, i2, g;
+};
+__device__ __forceinline__ GemmTile gemm_tile(const GemmParams& p, int t) {
+  GemmTile x;
+  x.nt = t % p.n_tiles;
+  t /= p.n_tiles;
+  x.i1 = t % p.t1;
+  t /= p.t1;
+  x.i2 = t % p.t2;
+  x.g = t / p.t2;
+  return x;
+}
+
+// 32 consecutive fp32 results of one row (`n` of them in range) to global memory.
+__device__ __forceinline__ void gemm_store32(const GemmParams& p, long long off, const uint32_t (&v)[32], int n) {
+  if (n <= 0) return;
+  if (p.out_fp32) {
+    float* o = static_cast<float*>(p.out) + off;
+    if (p.vec_ok && n >= 32) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        reinterpret_cast<uint4*>(o)[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if (i < n) o[i] = __uint_as_float(v[i]);
+    }
+    return;
+  }
+  uint32_t h[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) h[i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+  uint16_t* o = static_cast<uint16_t*>(p.out) + off;
+  if (p.vec_ok && n >= 32) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      reinterpret_cast<uint4*>(o)[i] = make_uint4(h[4 * i], h[4 * i + 1], h[4 * i + 2], h[4 * i + 3]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 32; ++i)
+      if (i < n) o[i] = static_cast<uint16_t>(h[i >> 1] >> (16 * (i & 1)));
+  }
+}
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    proj_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                     const GemmParams p) {
+  extern __shared__ __align__(1024) uint8_t gemm_smem_raw[];
+  __shared__ GemmSmem sm;
+  uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gemm_smem_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  const uint32_t ring = smem_u32(dsm);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr int S = kGemmStages;
+  auto bar = [](const uint64_t& b) { return smem_u32(&b); };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(bar(sm.full[s]), 1);
+      mbar_init(bar(sm.empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(sm.tfull[b]), 1);
+      mbar_init(bar(sm.tempty[b]), 8);
+    }
+    mbar_init(bar(sm.drain), 1);
+    sm.abort = 0;
+    sm.zero = 0;
+    sm.fills = 0;
+    sm.consumed = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&sm.tmem_base), kGemmTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const WaitCtl wc{&sm.abort, p.err, p.wait_limit_ns};
+  const WaitCtl wd{&sm.zero, p.err, p.wait_limit_ns};
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&map_a);
+      tma_prefetch_desc(&map_b);
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x) {
+        const GemmTile x = gemm_tile(p, t);
+        const int row_b = p.rows_per_b ? (x.i1 * p.b1) / p.rows_per_b : 0;
+        const int c_tile = x.nt * p.tn;
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(bar(sm.empty[s]), ((it / S) & 1) ^ 1, wc, GW_EMPTY)) {
+            ok = false;
+            break;
+          }
+          const uint32_t a_dst = ring + s * kGemmStageBytes;
+          const uint32_t b_dst = a_dst + kGemmABytes;
+          const uint32_t fb = bar(sm.full[s]);
+          mbar_arrive_expect_tx(fb, kGemmABytes + p.b_bytes);
+          tma_load_3d(a_dst, &map_a, fb, kb * 64, x.i1 * p.b1, x.i2 * p.b2);
+          if (p.b_mn) {
+            for (int a = 0; a < (p.tn >> 6); ++a) {
+              const int c0 = c_tile + 64 * a;
+              tma_load_3d(b_dst + a * 8192, &map_b, fb, c0 % p.nb, kb * 64, x.g + row_b + c0 / p.nb);
+            }
+          } else {
+            tma_load_3d(b_dst, &map_b, fb, kb * 64, c_tile, x.g + row_b);
+          }
+          sm.fills = it + 1;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, p.tn, 0, p.b_mn);
+      const uint32_t bstep = p.b_mn ? 2048u : 32u;  // one K step of 16: 16 rows of 128 B, or 32 B in a row
+      const uint32_t blbo = p.b_mn ? 8192u : 16u;   // MN-major: 64-column blocks 8 KB apart
+      int it = 0, lt = 0;
+      bool issued = false, ok = true;
+      for (int t = blockIdx.x; ok && t < p.total_tiles; t += gridDim.x, ++lt) {
+        const int buf = lt & 1;
+        if (!mbar_wait(bar(sm.tempty[buf]), ((lt >> 1) & 1) ^ 1, wc, GW_TEMPTY)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + 256u * buf;
+        for (int kb = 0; kb < p.k_blocks; ++kb, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(bar(sm.full[s]), (it / S) & 1, wc, GW_FULL)) {
+            ok = false;
+            break;
+          }
+          sm.consumed = it + 1;
+          tc_fence_after();
+          const uint32_t a_addr = ring + s * kGemmStageBytes;
+          const uint64_t ad = sdesc_sw128(a_addr, 16, 1024);
+          const uint64_t bd = sdesc_sw128(a_addr + kGemmABytes, blbo, 1024);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            umma_ss(d, desc_add(ad, kk * 32), desc_add(bd, kk * bstep), idesc, (kb | kk) ? 1u : 0u);
+          issued = true;
+          umma_commit(bar(sm.empty[s]));
+        }
+        if (ok) umma_commit(bar(sm.tfull[buf]));
+      }
+      if (issued) {
+        umma_commit(bar(sm.drain));
+        mbar_wait(bar(sm.drain), 0, wd, GW_DRAIN);
+      }
+    }
+  } else {
+    // ---------------- epilogue: TMEM -> registers -> global ----------------
+    const int qd = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int m = 32 * qd + lane;
+    const int hc = p.tn >> 1;
+    int lt = 0;
+    for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++lt) {
+      const GemmTile x = gemm_tile(p, t);
+      const int buf = lt & 1;
+      if (!mbar_wait(bar(sm.tfull[buf]), (lt >> 1) & 1, wc, GW_TFULL)) break;
+      tc_fence_after();
+      const int u1 = x.i1 * p.b1 + (m & (p.b1 - 1));
+      const int u2 = x.i2 * p.b2 + (m >> p.lg_b1);
+      const bool row_ok = u1 < p.n1 && u2 < p.n2;
+      const long long row_off = u1 * p.os1 + u2 * p.os2 + x.g * p.ocol;
+      for (int c = half * hc; c < (half + 1) * hc; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * qd) << 16) + 256u * buf + c, v);
+        tmem_wait_ld();
+        const int col = x.nt * p.tn + c;
+        if (row_ok) gemm_store32(p, row_off + col, v, p.n_valid - col);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(sm.tempty[buf]));
+    }
+  }
+
+  // Loads the MMA never waited for (after an abort) must land before the CTA's shared memory goes.
+  __syncthreads();
+  if (warp == 0 && lane == 0)
+    for (int i = sm.consumed; i < sm.fills; ++i) mbar_wait(bar(sm.full[i % S]), (i / S) & 1, wd, GW_DRAIN);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kGemmTmemCols);
+  }
+}
+
+}  // namespace lkv

@@ -11,7 +11,7 @@
 //   QK:  S[128 heads, 256 keys] += Q[heads, 64 cols] K[keys, 64 cols]^T, per 64-column chunk.
 //        CTA c streams keys 128c .. 128c+127 of the tile (all 576 columns); the pair reads every
 //        key row once.
-//   PV:  O[128 heads, 256 dims] += P[heads, 64 keys] V[64 keys, 256 dims], for the dims 0..255
+//   PV:  O[128 heads, 256 dims] += P[heads, 128 keys] V[128 keys, 256 dims], for the dims 0..255
 //        and 256..511.  CTA c streams dims 256b + 128c .. +127 of the tile's keys (a second read
 //        of latent rows the pair fetched for QK a moment before, served by L2).
 // There is no score exchange between the CTAs: each has exact fp32 scores of its own heads.
@@ -26,8 +26,8 @@
 // row max through a bounded shared-memory exchange.
 //
 // Shared memory per CTA: Q (9 chunks of 64 heads x 64 columns), P (4 chunks of 64 heads x 64 keys)
-// and a ring of 16 KB stages that carries, in the MMA's order, the 9 QK chunks of tile n+1 and
-// then the PV chunks of tile n.  Ring stages are counted on the even CTA's barriers (the pair load
+// and a ring of 32 KB stages that carries, in the MMA's order, the QK chunks of tile n+1 and then
+// the PV chunks of tile n; every load is a 16 KB box of 128 rows x 64 columns.  Ring stages are counted on the even CTA's barriers (the pair load
 // form), released to both CTAs by the MMA's multicast commit.
 #pragma once
 #include <cstdint>
@@ -43,12 +43,13 @@ constexpr int kPairTile = 256;             // keys per tile (N of the QK MMA)
 // Ring of 32 KB stages.  The even CTA learns of every stage of both CTAs on one barrier and both
 // CTAs learn of its release from one multicast commit; that hand-off has a fixed cost per stage, so
 // stages carry 32 KB (measured: 16 KB stages stream at under half the rate of 32 KB ones, and
-// three 32 KB stages already stream at HBM speed).  Per 256-key tile a CTA fills 4 stages of two
-// 64-column key chunks, 1 stage with the RoPE key chunk, and 1 stage per 64-key value chunk with
-// both dims blocks.
+// three 32 KB stages already stream at HBM speed), in boxes of 16 KB (8 KB boxes stream at about
+// two thirds of that rate).  Per 256-key tile a CTA fills 4 stages of two 64-column key chunks,
+// 1 stage with the RoPE key chunk, and 1 stage per 128-key value chunk and dims block: this CTA's
+// 128 dims of the block as two 64-dim boxes.
 constexpr int kPairStages = 3;             // ring stages
 constexpr int kPairStageBytes = 32768;
-constexpr int kPairChunkBytes = 16384;     // 128 keys x 64 columns, or 64 keys x 128 dims
+constexpr int kPairChunkBytes = 16384;     // one box: 128 keys x 64 columns
 constexpr int kPairQBytes = 9 * 8192;      // 64 heads x (512 + 64) columns
 constexpr int kPairPBytes = 4 * 8192;      // 64 heads x 256 keys
 constexpr int kPairQOff = 0;
@@ -83,7 +84,8 @@ struct __align__(16) PairSmem {
   float xch[2][4][64];          // [buffer][lane half * 2 + column half][head row]
   uint32_t tmem_base;
   uint32_t abort;
-  int vzero_stage, vzero_first; // stage of the chunk to clear, first row to clear
+  int vzero_stage[2];           // the two stages (dims blocks) of the chunk to clear
+  int vzero_first;              // its first row to clear
   int peer_chunks, peer_units;  // odd CTA's producer counts, for the even CTA's drain
   int own_chunks, own_units;    // even CTA's producer counts
   int stage_bytes[kPairStages]; // even CTA: bytes per CTA of the last phase armed on each stage
@@ -97,17 +99,20 @@ __device__ __forceinline__ int pair_tile_keys(const Segment& sg, int t) {
   const int k = sg.keys - t * kPairTile;
   return k < kPairTile ? k : kPairTile;
 }
+// 128-key value chunks of tile t (1 or 2).
+__device__ __forceinline__ int pair_pv_chunks(const Segment& sg, int t) { return (pair_tile_keys(sg, t) + 127) >> 7; }
 // Does the PV of tile t read latent rows past the end of the last request (row T = cu[B])?  Those
 // rows can hold anything, even NaN, and a zero weight times NaN is NaN: they are cleared first.
 __device__ __forceinline__ bool pair_crosses_end(const Segment& sg, int t, int T) {
-  const int nkc = (pair_tile_keys(sg, t) + 63) >> 6;
-  const int r1 = sg.cu_b + t * kPairTile + 64 * nkc;  // one past the last row PV reads
+  const int r1 = sg.cu_b + t * kPairTile + 128 * pair_pv_chunks(sg, t);  // one past the last row PV reads
   return r1 > T;
 }
-// PV stage i (0 .. nkc - 1) of a tile: its 64-key chunk.  A tile that crosses the cache end takes
-// its last key chunk first, so that chunk is resident before the softmax clears it.
+// PV stage i (0 .. 2 nkc - 1) of a tile: value chunk (128 keys) i / 2 in processing order, dims block
+// i % 2.  A tile that crosses the cache end takes its last chunk first (both blocks), so those two
+// stages are resident before the softmax clears the rows past the end.
 __device__ __forceinline__ int pair_pv_chunk(int i, int nkc, bool cross) {
-  return cross ? (i == 0 ? nkc - 1 : i - 1) : i;
+  const int c = i >> 1;
+  return cross ? (c == 0 ? nkc - 1 : c - 1) : c;
 }
 // Stages per tile for QK: 4 of two latent chunks, then 1 with the RoPE chunk.
 constexpr int kPairQkStages = 5;
@@ -117,7 +122,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                     const __grid_constant__ CUtensorMap map_qr,  // q_rope [rows, 64], box 64 x 64
                     const __grid_constant__ CUtensorMap map_k,   // ckv [T, 512], box 64 x 128
                     const __grid_constant__ CUtensorMap map_kr,  // kpe [T, 64], box 64 x 128
-                    const __grid_constant__ CUtensorMap map_v,   // ckv [T, 512], box 64 x 64
+                    const __grid_constant__ CUtensorMap map_v,   // ckv [T, 512], box 64 x 128
                     const TcParams p) {
   extern __shared__ __align__(1024) uint8_t pair_smem_raw[];
   __shared__ PairSmem sm;
@@ -234,21 +239,19 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         return true;
       };
       auto issue_pv = [&](const Segment& s, int t) -> bool {
-        const int nkc = (pair_tile_keys(s, t) + 63) >> 6;
+        const int nkc = pair_pv_chunks(s, t);
         const bool cross = pair_crosses_end(s, t, T_end);
-        for (int i = 0; i < nkc; ++i) {
+        for (int i = 0; i < 2 * nkc; ++i) {
           const int kc = pair_pv_chunk(i, nkc, cross);
           int st;
           if (!stage_acquire(st, kPairStageBytes)) return false;
           const uint32_t dst = ring_base + st * kPairStageBytes;
           const uint32_t fb = lead(sm.full[st]);
-          const int row = s.cu_b + t * kPairTile + 64 * kc;
-          // dims block b = 0, 1: this CTA's 128 dims of it as two 64-dim boxes
-          for (int b = 0; b < 2; ++b) {
-            const int x0 = 256 * b + 128 * static_cast<int>(rank);
-            tma_load_2d_pair(dst + b * kPairChunkBytes, &map_v, fb, x0, row);
-            tma_load_2d_pair(dst + b * kPairChunkBytes + 8192, &map_v, fb, x0 + 64, row);
-          }
+          const int row = s.cu_b + t * kPairTile + 128 * kc;
+          // this CTA's 128 dims of dims block i % 2 as two 64-dim boxes
+          const int x0 = 256 * (i & 1) + 128 * static_cast<int>(rank);
+          tma_load_2d_pair(dst, &map_v, fb, x0, row);
+          tma_load_2d_pair(dst + kPairChunkBytes, &map_v, fb, x0 + 64, row);
           ++chunks;
         }
         return true;
@@ -329,15 +332,18 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             !mbar_wait<true>(smem_u32(&sm.o_free), static_cast<uint32_t>((sidx - 1) & 1), wc,
                              LKV_WAIT_BASE_PAIR(PW_OFREE)))
           return false;
-        const int nkc = (pair_tile_keys(s, t) + 63) >> 6;
+        const int nkc = pair_pv_chunks(s, t);
         const bool cross = pair_crosses_end(s, t, T_end);
         if (cross) {
-          // the chunk past the cache end must be resident before the softmax warps clear it
-          if (!full_wait(ch)) return false;
-          const int first_bad = T_end - (s.cu_b + t * kPairTile + 64 * (nkc - 1));
-          sm.vzero_stage = ch % KS;
+          // the chunk past the cache end (its two stages) must be resident before the softmax
+          // warps clear it
+          if (!full_wait(ch) || !full_wait(ch + 1)) return false;
+          const int first_bad = T_end - (s.cu_b + t * kPairTile + 128 * (nkc - 1));
+          for (int b = 0; b < 2; ++b) {
+            sm.vzero_stage[b] = (ch + b) % KS;
+            st_cluster_u32(map_to_peer(smem_u32(&sm.vzero_stage[b]), 1u), static_cast<uint32_t>((ch + b) % KS));
+          }
           sm.vzero_first = first_bad;
-          st_cluster_u32(map_to_peer(smem_u32(&sm.vzero_stage), 1u), static_cast<uint32_t>(ch % KS));
           st_cluster_u32(map_to_peer(smem_u32(&sm.vzero_first), 1u), static_cast<uint32_t>(first_bad));
           mbar_arrive_remote(lead(sm.vland));
           mbar_arrive_remote(map_to_peer(smem_u32(&sm.vland), 1u));
@@ -345,18 +351,18 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         if (!mbar_wait<true>(smem_u32(&sm.p_full), static_cast<uint32_t>(m & 1), wc, LKV_WAIT_BASE_PAIR(PW_PFULL)))
           return false;
         tc_fence_after();
-        for (int i = 0; i < nkc; ++i) {
+        for (int i = 0; i < 2 * nkc; ++i) {
           const int kc = pair_pv_chunk(i, nkc, cross);
+          const int b = i & 1;
           if (!full_wait(ch)) return false;
           tc_fence_after();
-          const uint64_t pd = sdesc_sw128(p_base + kc * 8192, 16, 1024);
+          // P keys 128 kc + 16 kk: 64-key chunk 2 kc + kk / 4; V: two 64-dim boxes 16 KB apart
+          const uint64_t vd = sdesc_sw128(ring_base + (ch % KS) * kPairStageBytes, kPairChunkBytes, 1024);
 #pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            const uint64_t vd = sdesc_sw128(ring_base + (ch % KS) * kPairStageBytes + b * kPairChunkBytes, 8192, 1024);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk)
-              umma_pair_ss(tbase + 128 * b, desc_add(pd, kk * 32), desc_add(vd, kk * 2048), id_pv,
-                           (first && i == 0 && kk == 0) ? 0u : 1u);
+          for (int kk = 0; kk < 8; ++kk) {
+            const uint64_t pd = sdesc_sw128(p_base + (2 * kc + (kk >> 2)) * 8192, 16, 1024);
+            umma_pair_ss(tbase + 128 * b, desc_add(pd, (kk & 3) * 32), desc_add(vd, kk * 2048), id_pv,
+                         (first && i < 2 && kk == 0) ? 0u : 1u);
           }
           umma_pair_commit(smem_u32(&sm.empty[ch % KS]), kBothCtas);
           ++ch;
@@ -537,22 +543,24 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
         fence_proxy_async_smem();
         if (pair_crosses_end(sg, t, T_end)) {
-          // clear this CTA's latent rows past the cache end in the tile's last key chunk (one stage:
-          // two dims blocks of two 64-dim boxes each) once the MMA issuer reports them resident
+          // clear this CTA's latent rows past the cache end in the tile's last value chunk (two
+          // stages, one per dims block, of two 64-dim boxes each) once the MMA issuer reports them
+          // resident
           if (!wait_all(smem_u32(&sm.vland), static_cast<uint32_t>(ncross & 1), LKV_WAIT_BASE_PAIR(PW_VLAND))) {
             ok = false;
             break;
           }
           ++ncross;
-          const int st0 = *reinterpret_cast<volatile int*>(&sm.vzero_stage);
+          const int stz0 = *reinterpret_cast<volatile int*>(&sm.vzero_stage[0]);
+          const int stz1 = *reinterpret_cast<volatile int*>(&sm.vzero_stage[1]);
           const int first = *reinterpret_cast<volatile int*>(&sm.vzero_first);
-          const int rows = 64 - (first > 0 ? first : 0);
+          const int rows = 128 - (first > 0 ? first : 0);
           const int per_box = rows * 8;  // 16-byte chunks
           const int sidx = (warp - 2) * 32 + lane;
           for (int idx = sidx; idx < 4 * per_box; idx += 256) {
-            const int box = idx / per_box, r2 = idx % per_box;  // the stage's four 64-row, 64-dim boxes
-            uint8_t* base = ring + st0 * kPairStageBytes + box * 8192;
-            *reinterpret_cast<uint4*>(base + (64 - rows + r2 / 8) * 128 + (r2 % 8) * 16) = make_uint4(0u, 0u, 0u, 0u);
+            const int box = idx / per_box, r2 = idx % per_box;  // two stages x two 128-row, 64-dim boxes
+            uint8_t* base = ring + ((box >> 1) ? stz1 : stz0) * kPairStageBytes + (box & 1) * kPairChunkBytes;
+            *reinterpret_cast<uint4*>(base + (128 - rows + r2 / 8) * 128 + (r2 % 8) * 16) = make_uint4(0u, 0u, 0u, 0u);
           }
           fence_proxy_async_smem();
         }

@@ -5,88 +5,94 @@
 // with j(h) = h / (h_q / G), and the output projection that follows attention,
 //                   y[t, :]        = o[t, :] W_O                  (o = the heads' outputs side by side)
 // which, with the heads split across GPUs along the group axis, gives each GPU a partial y to be summed
-// (GQLA explainer, section 2, GQA path: tensor parallelism along the group axis).  These are plain GEMMs (bf16 operands, fp32 accumulation, bf16
-// result), run by cuBLAS.  cuBLAS is opened at the first projection call (dlopen), so the decode path
-// and the rest of the library never depend on it; each device gets one cuBLAS handle, created at its
-// first projection call (cuBLAS allocates its own workspace then).
+// (GQLA explainer, section 2, GQA path: tensor parallelism along the group axis).
+//
+// Each is one launch of the tensor-core GEMM of lkv_gemm.cuh (bf16 operands, fp32 accumulation in
+// TMEM): the host describes the rows of A (which may gather the heads of one group across tokens),
+// which B matrix a tile takes, and where each result row goes.
+#include <climits>
 #include <cstdint>
-#include <cstring>
-#include <dlfcn.h>
 #include <mutex>
-#include <cublas_v2.h>
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/lkv.h"
+#include "lkv_gemm.cuh"
+#include "lkv_tma_host.h"
+
+lkv_status lkv_internal_device_info(int** err, int* num_sms, unsigned long long* wait_ns);  // lkv_api.cu
 
 namespace {
 
-// The C entry points used (32-bit sizes, 64-bit batch strides).
-typedef cublasStatus_t (*CreateFn)(cublasHandle_t*);
-typedef cublasStatus_t (*SetStreamFn)(cublasHandle_t, cudaStream_t);
-typedef cublasStatus_t (*GemmFn)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int, int, const void*,
-                                 const void*, cudaDataType, int, long long, const void*, cudaDataType, int, long long,
-                                 const void*, void*, cudaDataType, int, long long, int, cublasComputeType_t,
-                                 cublasGemmAlgo_t);
-struct CublasApi {
-  CreateFn create = nullptr;
-  SetStreamFn set_stream = nullptr;
-  GemmFn gemm = nullptr;
-  bool ok = false;
-};
-
-const CublasApi& cublas_api() {
-  static CublasApi api;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* h = dlopen("libcublas.so.12", RTLD_NOW | RTLD_GLOBAL);
-    if (!h) h = dlopen("libcublas.so", RTLD_NOW | RTLD_GLOBAL);
-    if (!h) return;
-    api.create = reinterpret_cast<decltype(api.create)>(dlsym(h, "cublasCreate_v2"));
-    api.set_stream = reinterpret_cast<decltype(api.set_stream)>(dlsym(h, "cublasSetStream_v2"));
-    api.gemm = reinterpret_cast<decltype(api.gemm)>(dlsym(h, "cublasGemmStridedBatchedEx"));
-    api.ok = api.create && api.set_stream && api.gemm;
-  });
-  return api;
-}
+using namespace lkv;
 
 constexpr int kMaxDevices = 64;
-
-// Serialises the projection calls of all host threads: a device's one handle is re-bound to the
-// caller's stream at every call, so the binding and the GEMMs it enqueues must not interleave with
-// another thread's.  Only the enqueueing is serialised, not the GPU work.
-std::mutex& proj_mutex() {
-  static std::mutex mu;
-  return mu;
-}
-
-// The cuBLAS handle of the current device, bound to `stream`.  Call with proj_mutex() held.
-lkv_status handle_for(cudaStream_t stream, cublasHandle_t* out) {
-  const CublasApi& api = cublas_api();
-  if (!api.ok) return LKV_ERR_UNSUPPORTED;
-  static cublasHandle_t handles[kMaxDevices] = {};
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LKV_ERR_CUDA;
-  if (!handles[dev] && api.create(&handles[dev]) != CUBLAS_STATUS_SUCCESS) {
-    handles[dev] = nullptr;
-    return LKV_ERR_CUDA;
-  }
-  if (api.set_stream(handles[dev], stream) != CUBLAS_STATUS_SUCCESS) return LKV_ERR_CUDA;
-  *out = handles[dev];
-  return LKV_OK;
-}
-
-// One strided-batched GEMM of bf16 operands in cuBLAS's column-major terms: C = op(A) op(B), fp32
-// accumulate, C in bf16 (or fp32 when c_fp32).
-lkv_status gemm(cublasHandle_t h, cublasOperation_t ta, int m, int n, int k, const void* A, int lda, long long sA,
-                const void* B, int ldb, long long sB, void* C, int ldc, long long sC, int batch, bool c_fp32 = false) {
-  const float one = 1.f, zero = 0.f;
-  const cublasStatus_t s = cublas_api().gemm(h, ta, CUBLAS_OP_N, m, n, k, &one, A, CUDA_R_16BF, lda, sA, B, CUDA_R_16BF,
-                                             ldb, sB, &zero, C, c_fp32 ? CUDA_R_32F : CUDA_R_16BF, ldc, sC, batch,
-                                             CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT);
-  return s == CUBLAS_STATUS_SUCCESS ? LKV_OK : LKV_ERR_CUDA;
-}
+constexpr int kNoColumnGroups = 1 << 30;  // nb when the column axis stays inside one B matrix
 
 bool fits_int(long long v) { return v > 0 && v <= 0x7fffffffLL; }
+bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+int cdiv(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+// Row tiling: a tile takes b1 consecutive rows of A's dim 1 (a power of two that divides
+// rows_per_b, so one tile never spans two B matrices; 128 when rows do not select B) times b2 = 128 / b1
+// rows of dim 2.
+void set_rows(GemmParams& p, int n1, int n2, int rows_per_b) {
+  int b1 = 128;
+  if (rows_per_b) {
+    b1 = 1;
+    while (b1 < 128 && rows_per_b % (2 * b1) == 0) b1 *= 2;
+  }
+  p.b1 = b1;
+  p.lg_b1 = 31 - __builtin_clz(static_cast<unsigned>(b1));
+  p.b2 = 128 / b1;
+  p.n1 = n1;
+  p.n2 = n2;
+  p.t1 = cdiv(n1, b1);
+  p.t2 = cdiv(n2, p.b2);
+  p.rows_per_b = rows_per_b;
+}
+
+// Column tiling: as few tiles of <= 256 columns as cover n, each a multiple of 64 wide.
+void set_cols(GemmParams& p, int n) {
+  p.n_tiles = cdiv(n, 256);
+  p.tn = 64 * cdiv(cdiv(n, p.n_tiles), 64);
+  p.b_bytes = p.tn * 128;
+}
+
+lkv_status launch(const CUtensorMap& ma, const CUtensorMap& mb, GemmParams& p, int k, cudaStream_t s) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LKV_ERR_CUDA;
+  int num_sms = 0;
+  lkv_status st = lkv_internal_device_info(&p.err, &num_sms, &p.wait_limit_ns);
+  if (st != LKV_OK) return st;
+  static std::mutex mu;
+  static bool attr_set[kMaxDevices] = {};
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!attr_set[dev]) {
+      if (cudaFuncSetAttribute(proj_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kGemmSmemBytes)) != cudaSuccess)
+        return LKV_ERR_CUDA;
+      attr_set[dev] = true;
+    }
+  }
+  p.k_blocks = cdiv(k, 64);
+  const long long tiles = static_cast<long long>(p.n_tiles) * p.t1 * p.t2 * p.groups;
+  if (tiles <= 0 || tiles > INT_MAX) return LKV_ERR_INVALID_ARG;
+  p.total_tiles = static_cast<int>(tiles);
+  const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
+  proj_gemm_kernel<<<grid, kGemmThreads, kGemmSmemBytes, s>>>(ma, mb, p);
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? LKV_OK : LKV_ERR_CUDA;
+}
+
+GemmParams base_params(void* out) {
+  GemmParams p{};
+  p.groups = 1;
+  p.nb = kNoColumnGroups;
+  p.out = out;
+  return p;
+}
 
 }  // namespace
 
@@ -98,23 +104,20 @@ lkv_status lkv_absorb_query(const void* q, const void* w_uk, void* q_abs, int n_
       h_q % groups != 0 || !fits_int(static_cast<long long>(h_q) * r) || !fits_int(static_cast<long long>(h_q) * d_h))
     return LKV_ERR_INVALID_ARG;
   if (dtype != LKV_BF16) return LKV_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(proj_mutex());
-  cublasHandle_t h;
-  lkv_status st = handle_for(static_cast<cudaStream_t>(stream), &h);
-  if (st != LKV_OK) return st;
-  const int hpg = h_q / groups;
-  const auto* qb = static_cast<const uint16_t*>(q);
-  const auto* wb = static_cast<const uint16_t*>(w_uk);
-  auto* ob = static_cast<uint16_t*>(q_abs);
-  if (groups == 1 && fits_int(static_cast<long long>(n_tok) * h_q))  // one shared W: a single GEMM over every (t, h)
-    return gemm(h, CUBLAS_OP_T, r, n_tok * h_q, d_h, wb, d_h, 0, qb, d_h, 0, ob, r, 0, 1);
-  for (int j = 0; j < groups && st == LKV_OK; ++j) {
-    // per head of group j: (q_abs_h)^T [r x n] = W [r x d_h] * (q_h)^T [d_h x n]
-    st = gemm(h, CUBLAS_OP_T, r, n_tok, d_h, wb + static_cast<size_t>(j) * r * d_h, d_h, 0,
-              qb + static_cast<size_t>(j) * hpg * d_h, h_q * d_h, d_h, ob + static_cast<size_t>(j) * hpg * r, h_q * r, r,
-              hpg);
-  }
-  return st;
+  if (d_h % 8 != 0 || !al16(q) || !al16(w_uk)) return LKV_ERR_INVALID_ARG;
+  // rows (h, t) of q; B = W_UK[j] as [r, d_h] rows (K-major)
+  GemmParams p = base_params(q_abs);
+  set_rows(p, h_q, n_tok, h_q / groups);
+  set_cols(p, r);
+  p.n_valid = r;
+  p.os1 = r;
+  p.os2 = static_cast<long long>(h_q) * r;
+  p.vec_ok = (r % 8 == 0) && al16(q_abs);
+  CUtensorMap ma, mb;
+  if (!make_tmap_bf16_3d(&ma, q, d_h, h_q, n_tok, 2ull * d_h, 2ull * d_h * h_q, p.b1, p.b2) ||
+      !make_tmap_bf16_3d(&mb, w_uk, d_h, r, groups, 2ull * d_h, 2ull * d_h * r, p.tn, 1))
+    return LKV_ERR_INVALID_ARG;
+  return launch(ma, mb, p, d_h, static_cast<cudaStream_t>(stream));
 }
 
 lkv_status lkv_unabsorb_output(const void* o_lat, const void* w_uv, void* out, int n_tok, int h_q, int groups, int r,
@@ -123,23 +126,21 @@ lkv_status lkv_unabsorb_output(const void* o_lat, const void* w_uv, void* out, i
       h_q % groups != 0 || !fits_int(static_cast<long long>(h_q) * r) || !fits_int(static_cast<long long>(h_q) * d_v))
     return LKV_ERR_INVALID_ARG;
   if (dtype != LKV_BF16) return LKV_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(proj_mutex());
-  cublasHandle_t h;
-  lkv_status st = handle_for(static_cast<cudaStream_t>(stream), &h);
-  if (st != LKV_OK) return st;
-  const int hpg = h_q / groups;
-  const auto* ob = static_cast<const uint16_t*>(o_lat);
-  const auto* wb = static_cast<const uint16_t*>(w_uv);
-  auto* yb = static_cast<uint16_t*>(out);
-  if (groups == 1 && fits_int(static_cast<long long>(n_tok) * h_q))
-    return gemm(h, CUBLAS_OP_N, d_v, n_tok * h_q, r, wb, d_v, 0, ob, r, 0, yb, d_v, 0, 1);
-  for (int j = 0; j < groups && st == LKV_OK; ++j) {
-    // per head of group j: (out_h)^T [d_v x n] = W^T [d_v x r] * (o_h)^T [r x n]
-    st = gemm(h, CUBLAS_OP_N, d_v, n_tok, r, wb + static_cast<size_t>(j) * r * d_v, d_v, 0,
-              ob + static_cast<size_t>(j) * hpg * r, h_q * r, r, yb + static_cast<size_t>(j) * hpg * d_v, h_q * d_v, d_v,
-              hpg);
-  }
-  return st;
+  if (r % 8 != 0 || d_v % 8 != 0 || !al16(o_lat) || !al16(w_uv)) return LKV_ERR_INVALID_ARG;
+  // rows (h, t) of o_lat; B = W_UV[j] as [r, d_v] (MN-major)
+  GemmParams p = base_params(out);
+  set_rows(p, h_q, n_tok, h_q / groups);
+  set_cols(p, d_v);
+  p.b_mn = 1;
+  p.n_valid = d_v;
+  p.os1 = d_v;
+  p.os2 = static_cast<long long>(h_q) * d_v;
+  p.vec_ok = al16(out);
+  CUtensorMap ma, mb;
+  if (!make_tmap_bf16_3d(&ma, o_lat, r, h_q, n_tok, 2ull * r, 2ull * r * h_q, p.b1, p.b2) ||
+      !make_tmap_bf16_3d(&mb, w_uv, d_v, r, groups, 2ull * d_v, 2ull * d_v * r, 64, 1))
+    return LKV_ERR_INVALID_ARG;
+  return launch(ma, mb, p, r, static_cast<cudaStream_t>(stream));
 }
 
 lkv_status lkv_expand_latent(const void* c, int64_t c_row_stride, const void* w, void* x, int64_t n_rows, int groups,
@@ -148,25 +149,53 @@ lkv_status lkv_expand_latent(const void* c, int64_t c_row_stride, const void* w,
       !fits_int(n_rows) || !fits_int(c_row_stride) || !fits_int(static_cast<long long>(groups) * d))
     return LKV_ERR_INVALID_ARG;
   if (dtype != LKV_BF16) return LKV_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(proj_mutex());
-  cublasHandle_t h;
-  const lkv_status st = handle_for(static_cast<cudaStream_t>(stream), &h);
-  if (st != LKV_OK) return st;
-  // per group j: (X_j)^T [d x T] = W_j^T [d x r] * c^T [r x T]
-  return gemm(h, CUBLAS_OP_N, d, static_cast<int>(n_rows), r, w, d, static_cast<long long>(r) * d, c,
-              static_cast<int>(c_row_stride), 0, x, groups * d, d, groups);
+  if (c_row_stride % 8 != 0 || d % 8 != 0 || !al16(c) || !al16(w)) return LKV_ERR_INVALID_ARG;
+  // rows t of c; B = W[j] as [r, d] (MN-major).  With d a multiple of 64 the G matrices sit side by
+  // side along the columns (one tile may span two groups: x[t] is [G, d] contiguous); else one
+  // column block per group.
+  GemmParams p = base_params(x);
+  set_rows(p, static_cast<int>(n_rows), 1, 0);
+  p.b_mn = 1;
+  p.os1 = static_cast<long long>(groups) * d;
+  if (d % 64 == 0) {
+    set_cols(p, groups * d);
+    p.nb = d;
+    p.n_valid = groups * d;
+  } else {
+    set_cols(p, d);
+    p.groups = groups;
+    p.ocol = d;
+    p.n_valid = d;
+  }
+  p.vec_ok = al16(x);
+  const uint64_t cs = 2ull * static_cast<uint64_t>(c_row_stride);
+  CUtensorMap ma, mb;
+  if (!make_tmap_bf16_3d(&ma, c, r, n_rows, 1, cs, cs * static_cast<uint64_t>(n_rows), 128, 1) ||
+      !make_tmap_bf16_3d(&mb, w, d, r, groups, 2ull * d, 2ull * d * r, 64, 1))
+    return LKV_ERR_INVALID_ARG;
+  return launch(ma, mb, p, r, static_cast<cudaStream_t>(stream));
 }
 
 lkv_status lkv_output_projection(const void* o, const void* w_o, void* y, int n_tok, int k, int d_model,
                                  int out_dtype, lkv_stream_t stream) {
   if (!o || !w_o || !y || n_tok <= 0 || k <= 0 || d_model <= 0) return LKV_ERR_INVALID_ARG;
   if (out_dtype != LKV_BF16 && out_dtype != LKV_FP32) return LKV_ERR_INVALID_ARG;
-  std::lock_guard<std::mutex> lock(proj_mutex());
-  cublasHandle_t h;
-  const lkv_status st = handle_for(static_cast<cudaStream_t>(stream), &h);
-  if (st != LKV_OK) return st;
-  // y^T [d_model x n] = W_O^T [d_model x k] * o^T [k x n]
-  return gemm(h, CUBLAS_OP_N, d_model, n_tok, k, w_o, d_model, 0, o, k, 0, y, d_model, 0, 1, out_dtype == LKV_FP32);
+  if (k % 8 != 0 || d_model % 8 != 0 || !al16(o) || !al16(w_o)) return LKV_ERR_INVALID_ARG;
+  // rows t of o; B = W_O as [k, d_model] (MN-major)
+  GemmParams p = base_params(y);
+  set_rows(p, n_tok, 1, 0);
+  set_cols(p, d_model);
+  p.b_mn = 1;
+  p.out_fp32 = out_dtype == LKV_FP32;
+  p.n_valid = d_model;
+  p.os1 = d_model;
+  p.vec_ok = al16(y);
+  const uint64_t os = 2ull * static_cast<uint64_t>(k);
+  CUtensorMap ma, mb;
+  if (!make_tmap_bf16_3d(&ma, o, k, n_tok, 1, os, os * static_cast<uint64_t>(n_tok), 128, 1) ||
+      !make_tmap_bf16_3d(&mb, w_o, d_model, k, 1, 2ull * d_model, 2ull * d_model * k, 64, 1))
+    return LKV_ERR_INVALID_ARG;
+  return launch(ma, mb, p, k, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

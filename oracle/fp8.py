@@ -6,24 +6,27 @@ What the pages fix and what is read into them:
 * The serving comparison in the Grouped Latent Attention article (news page, section on the
   GLA-vs-MLA decoding test) runs DeepSeek-Coder-V2 in FP8; the pages give no cache format.
 * Reading: the latent part of each cached token is stored as e4m3 codes with one fp32 scale per
-  token, s_t = amax_t / 448 (amax_t = max |c_KV[t, :]|), so that the largest entry maps to the
-  largest finite e4m3 value; the RoPE key stays bf16.  Dequantised value = e4m3(code) * s_t.
+  token, s_t = the smallest power of two with amax_t / s_t <= 448 (amax_t = max |c_KV[t, :]|), so
+  that the largest entry lands in the top binade of e4m3 (224, 448]; the RoPE key stays bf16.
+  Dequantised value = e4m3(code) * s_t.  A power of two (as in the OCP microscaling formats' shared
+  scales) makes the dequantised value exact in bf16: a decode may dequantise into bf16 operands and
+  still compute on exactly the values this oracle reads.
 * e4m3 is the OCP 8-bit floating-point E4M3 format: 1 sign bit, 4 exponent bits with bias 7,
   3 mantissa bits; exponent field 0 holds subnormals m * 2^-9; fields 1..15 hold
   (1 + m/8) * 2^(e-7); the all-ones pattern S.1111.111 is NaN; there are no infinities, so the
   largest finite magnitude is 1.75 * 2^8 = 448.
 
-Quantisation arithmetic (the same steps the CUDA kernel takes, in fp32, so that the codes, which
-floating point decides, come out identical): amax in fp32 (exact: a max of stored bf16 values),
-s = amax / 448 rounded to fp32, y = x / s rounded to fp32, y clamped to [-448, 448], code = y
-rounded to the nearest e4m3 value with ties to the even code.  A row whose amax is 0 gets s = 0
-and all codes 0.
+Quantisation arithmetic (the same steps the CUDA kernel takes, so that the codes, which floating
+point decides, come out identical): amax in fp32 (exact: a max of stored bf16 values), s the
+power of two above (exact), y = x / s (exact: a power-of-two division), y clamped to [-448, 448]
+(a no-op), code = y rounded to the nearest e4m3 value with ties to the even code.  A row whose
+amax is 0 gets s = 0 and all codes 0.
 """
 from __future__ import annotations
 
 import numpy as np
 
-__all__ = ["E4M3_MAX", "e4m3_decode", "e4m3_encode", "quantize_rows", "dequantize_rows",
+__all__ = ["E4M3_MAX", "e4m3_decode", "e4m3_encode", "pow2_scale", "quantize_rows", "dequantize_rows",
            "mla_absorbed_decode_fp8", "gta_group_decode_fp8"]
 
 E4M3_MAX = 448.0
@@ -71,6 +74,17 @@ def e4m3_encode(y) -> np.ndarray:
     return np.where(np.signbit(y), mag | 0x80, mag).astype(np.uint8)
 
 
+def pow2_scale(amax) -> np.ndarray:
+    """Per-token scale: the smallest power of two s with amax / s <= 448 (0 where amax is 0).
+
+    With amax = m * 2^E (m in [0.5, 1), numpy's frexp), amax <= 448 * 2^e = 0.875 * 2^(9 + e) holds
+    for e = E - 9 when m <= 0.875 and first for e = E - 8 otherwise."""
+    a = np.asarray(amax, dtype=np.float64)
+    m, E = np.frexp(a)
+    e = np.where(m <= 0.875, E - 9, E - 8)
+    return np.where(a > 0, np.ldexp(1.0, e), 0.0).astype(np.float32)
+
+
 def quantize_rows(x):
     """Per-row e4m3 quantisation of stored latent rows x [n, r] (bf16 or fp32 values).
 
@@ -79,11 +93,11 @@ def quantize_rows(x):
     if x32.ndim != 2:
         raise ValueError("x must be [n, r]")
     amax = np.abs(x32).max(axis=1)                        # exact in fp32
-    scales = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    scales = pow2_scale(amax)
     codes = np.zeros(x32.shape, dtype=np.uint8)
     nz = scales > 0
     if np.any(nz):
-        y = (x32[nz] / scales[nz, None]).astype(np.float32)   # fp32 division, per element
+        y = (x32[nz] / scales[nz, None]).astype(np.float32)   # exact: division by a power of two
         y = np.clip(y, -E4M3_MAX, E4M3_MAX)
         codes[nz] = e4m3_encode(y)
     return codes, scales

@@ -214,7 +214,7 @@ def test_validation_errors_need_no_gpu(lkv):
 
 
 def test_projection_argument_errors_need_no_gpu(lkv):
-    """The projection entry points reject bad arguments before any CUDA or cuBLAS call."""
+    """The projection entry points reject bad arguments before any CUDA call."""
     P = _fake(1 << 20)
     st = ctypes.c_void_p(0)
     assert lkv._absorb(None, P, P, 4, 8, 4, 8, 16, 0, st) == lkv.ERR_INVALID_ARG
@@ -227,6 +227,19 @@ def test_projection_argument_errors_need_no_gpu(lkv):
     assert lkv._expand(P, 8, P, P, 4, 2, 16, 8, 0, st) == lkv.ERR_INVALID_ARG      # row stride < r
     assert lkv._expand(P, 16, P, P, 0, 2, 16, 8, 0, st) == lkv.ERR_INVALID_ARG
     assert lkv._expand(P, 16, P, P, 4, 2, 16, 8, 1, st) == lkv.ERR_UNSUPPORTED
+    # the tensor-core GEMM's TMA operands: 16-byte aligned pointers, rows of a multiple of 8 elements
+    M = _fake((1 << 20) + 8)
+    assert lkv._absorb(M, P, P, 4, 8, 4, 8, 16, 0, st) == lkv.ERR_INVALID_ARG      # misaligned q
+    assert lkv._absorb(P, P, P, 4, 8, 4, 12, 16, 0, st) == lkv.ERR_INVALID_ARG     # d_h = 12
+    assert lkv._unabsorb(P, P, P, 4, 8, 4, 20, 8, 0, st) == lkv.ERR_INVALID_ARG    # r = 20
+    assert lkv._unabsorb(P, P, P, 4, 8, 4, 16, 12, 0, st) == lkv.ERR_INVALID_ARG   # d_v = 12
+    assert lkv._unabsorb(P, M, P, 4, 8, 4, 16, 8, 0, st) == lkv.ERR_INVALID_ARG    # misaligned w_uv
+    assert lkv._expand(P, 20, P, P, 4, 2, 16, 8, 0, st) == lkv.ERR_INVALID_ARG     # row stride 20
+    assert lkv._expand(P, 16, P, P, 4, 2, 16, 12, 0, st) == lkv.ERR_INVALID_ARG    # d = 12
+    assert lkv._expand(M, 16, P, P, 4, 2, 16, 8, 0, st) == lkv.ERR_INVALID_ARG     # misaligned c
+    assert lkv._oproj(P, P, P, 4, 12, 8, 0, st) == lkv.ERR_INVALID_ARG             # k = 12
+    assert lkv._oproj(P, P, P, 4, 16, 12, 1, st) == lkv.ERR_INVALID_ARG            # d_model = 12
+    assert lkv._oproj(P, M, P, 4, 16, 8, 1, st) == lkv.ERR_INVALID_ARG             # misaligned w_o
 
 
 def test_fp8_cache_rows_host_side(lkv):

@@ -99,3 +99,22 @@ def test_cpu_baseline_on_device_inputs_is_bounded():
     cb = bench.cpu_baseline_device(w, d, 0.0)                # budget spent after the first request
     assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["cores"] == os.cpu_count()
     assert cb["sample"].startswith("1 of 3 requests")
+
+
+@pytest.mark.parametrize("world,rank", [(1, 0), (2, 1), (8, 7)])
+def test_tp_local_inputs_hold_one_ranks_groups_and_heads(world, rank):
+    """The group-axis TP workload's per-rank inputs: g / world groups of K_j and V_j, the heads of
+    those groups, the full RoPE key and the matching h_q / world * d_v rows of W_O."""
+    import torch
+    from latent_kv_cache_split_b200.tp import group_shard
+    w = synth.workload(bench.TP_WORKLOAD, batch=2, seqlen=40)
+    sh = group_shard(w.groups, w.h_q, world, rank)
+    d = bench.tp_local_inputs(w, sh, torch.device("cpu"), 64)
+    T = 2 * 40
+    assert d["q"].shape == (2, w.s_q, w.h_q // world, w.d_k)
+    assert d["q_rope"].shape == (2, w.s_q, w.h_q // world, w.d_rope)
+    assert d["k"].shape == (T, w.groups // world, w.d_k) and d["v"].shape == (T, w.groups // world, w.d_v)
+    assert d["kpe"].shape == (T, w.d_rope)
+    assert d["w_o"].shape == (w.h_q // world * w.d_v, 64)
+    assert d["cu_seqlens"].tolist() == [0, 40, 80]
+    assert all(t.dtype == torch.bfloat16 for k, t in d.items() if k not in ("lengths", "cu_seqlens"))

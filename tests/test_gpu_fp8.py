@@ -1,6 +1,8 @@
-"""GPU tests for FP8 (e4m3) latent cache rows: the quantisation kernel against the oracle's fp32
-steps, bit for bit (the codes are integers that floating point decides, and both sides take the
-same IEEE fp32 division and round-to-nearest-even), in bulk and at append."""
+"""GPU tests for FP8 (e4m3) latent cache rows: the quantisation kernel against the oracle's steps,
+bit for bit (the codes are integers that floating point decides; the power-of-two scale makes the
+division exact on both sides, and both round to nearest even), in bulk and at append; and the GTA
+decode over FP8 rows against the oracle's decode over the dequantised states (rows built on the
+host by the oracle's quantiser, so no input comes from the GPU path)."""
 import numpy as np
 import pytest
 import torch
@@ -124,3 +126,118 @@ def test_quantize_throughput(L, gpu):
     ms = e0.elapsed_time(e1) / 20
     moved = T * ((r + d_rope) * 2 + cache.shape[1])
     print(f"quantize {T} rows: {ms * 1e3:.1f} us, {moved / ms / 1e6:.0f} GB/s (bytes read + written)")
+
+
+# ---------------------------------------------------------------------------------------------
+# GTA decode over FP8 rows
+import math  # noqa: E402
+
+from gpu_util import compare  # noqa: E402
+
+
+def _fp8_gta_case(lengths, s_q=2, groups=8, h_q=128, seed=0, extra_rows=0, std=None, q_std=None):
+    """bf16 GTA inputs of the given shape, their tied states quantised into FP8 rows by the oracle."""
+    kw = {} if std is None else {"input_std": std}
+    if q_std is not None:
+        kw["q_std"] = q_std
+    w = synth.workload("gta_g8_sq2_l8192", batch=len(lengths), s_q=s_q, seqlen=None, groups=groups, h_q=h_q,
+                       seed=seed, **kw)
+    d = synth.make_inputs(w, lengths=lengths, extra_rows=extra_rows)
+    width = w.groups * w.d_k
+    tied = d["cache"][:, :width].float().numpy()
+    kpe = d["cache"][:, width:].contiguous()
+    codes, scales = fp8.quantize_rows(tied)
+    rb = 16 * ((width + 16 + 2 * w.d_rope + 15) // 16)
+    rows = np.zeros((tied.shape[0], rb), dtype=np.uint8)
+    rows[:, :width] = codes
+    rows[:, width:width + 4] = scales.view(np.uint8).reshape(-1, 4)
+    rows[:, width + 16:width + 16 + 2 * w.d_rope] = kpe.view(torch.uint8).numpy()
+    return w, d, torch.from_numpy(rows), codes, scales, kpe
+
+
+def _run_fp8_gta(L, gpu, w, d, rows):
+    return L.gta_group_decode_fp8(d["q"].to(gpu), d["q_rope"].to(gpu), rows.to(gpu), w.groups,
+                                  d["cu_seqlens"].to(gpu), w.scale)
+
+
+def _oracle_fp8_gta(w, d, codes, scales, kpe, requests=None):
+    cu = d["cu_seqlens"].numpy().astype(np.int64)
+    return fp8.gta_group_decode_fp8(d["q"], d["q_rope"], codes, scales, kpe, w.groups, cu, w.scale,
+                                    requests=requests)
+
+
+@pytest.mark.parametrize("lengths,s_q,groups", [([900, 130, 2, 1500], 2, 8), ([257, 1, 128, 129], 1, 8),
+                                                ([700, 64, 3], 2, 4), ([1, 2, 3, 4000], 1, 2)])
+def test_gta_fp8_decode_parity(L, gpu, lengths, s_q, groups):
+    """Ragged lengths over several 128-key tiles and a tail, s_q 1 and 2, 8 / 4 / 2 groups (units of
+    32, 64 and 64 rows)."""
+    w, d, rows, codes, scales, kpe = _fp8_gta_case(lengths, s_q=s_q, groups=groups, h_q=128 if groups > 2 else 64)
+    out, lse = _run_fp8_gta(L, gpu, w, d, rows)
+    torch.cuda.synchronize()
+    assert L.check_device() == 0
+    ref_out, ref_lse = _oracle_fp8_gta(w, d, codes, scales, kpe)
+    compare(out, lse, ref_out, ref_lse, label=f"gta fp8 {lengths} s_q={s_q} g={groups}")
+
+
+@pytest.mark.parametrize("spread", [4.0, 16.0])
+def test_gta_fp8_decode_wide_score_spread(L, gpu, spread):
+    w, d, rows, codes, scales, kpe = _fp8_gta_case([900, 130, 2, 1500], std=0.5, q_std=2.0 * spread, seed=5)
+    out, lse = _run_fp8_gta(L, gpu, w, d, rows)
+    ref_out, ref_lse = _oracle_fp8_gta(w, d, codes, scales, kpe)
+    compare(out, lse, ref_out, ref_lse, label=f"gta fp8 spread {spread}")
+
+
+def test_gta_fp8_decode_full_size_sampled(L, gpu):
+    """The GTA workload at full size (64 requests of 8192 keys, s_q = 2) in FP8: eight requests
+    against the oracle."""
+    w, d, rows, codes, scales, kpe = _fp8_gta_case([8192] * 64, seed=2)
+    out, lse = _run_fp8_gta(L, gpu, w, d, rows)
+    torch.cuda.synchronize()
+    assert L.check_device() == 0
+    req = [0, 9, 18, 27, 36, 45, 54, 63]
+    ref_out, ref_lse = _oracle_fp8_gta(w, d, codes, scales, kpe, requests=req)
+    compare(out, lse, ref_out, ref_lse, requests=req, label="gta fp8 full size")
+
+
+def test_gta_fp8_rows_past_the_cache_do_not_leak(L, gpu):
+    """NaN codes and an infinite scale in the rows after the last request give bitwise the result of
+    zero rows there."""
+    lengths = [100, 37, 129]
+    w, d, rows, codes, scales, kpe = _fp8_gta_case(lengths, extra_rows=70)
+    out0, lse0 = (t.clone() for t in _run_fp8_gta(L, gpu, w, d, rows))
+    T = sum(lengths)
+    bad = rows.clone()
+    width = w.groups * w.d_k
+    bad[T:, :width] = 0x7F                                    # e4m3 NaN
+    bad[T:, width:width + 4] = torch.tensor(np.array([np.inf], dtype=np.float32).view(np.uint8))
+    out1, lse1 = _run_fp8_gta(L, gpu, w, d, bad)
+    torch.cuda.synchronize()
+    assert torch.isfinite(out1.float()).all()
+    assert torch.equal(out0, out1) and torch.equal(lse0, lse1)
+
+
+def test_gta_fp8_agrees_with_bf16_gta_on_the_dequantised_states(L, gpu):
+    """The FP8 decode and the bf16 GTA decode over the dequantised (bf16-exact) states compute on
+    the same values: outputs agree to the bf16 rounding of the results."""
+    w, d, rows, codes, scales, kpe = _fp8_gta_case([700, 64, 3], seed=7)
+    deq = torch.from_numpy(fp8.dequantize_rows(codes, scales)).bfloat16()
+    assert torch.equal(deq.double(), torch.from_numpy(fp8.dequantize_rows(codes, scales)))
+    out8, lse8 = _run_fp8_gta(L, gpu, w, d, rows)
+    cache = torch.cat([deq, kpe], 1).to(gpu)
+    width = w.groups * w.d_k
+    out16, lse16 = L.gta_group_decode(d["q"].to(gpu), d["q_rope"].to(gpu), cache[:, :width], cache[:, width:],
+                                      w.groups, d["cu_seqlens"].to(gpu), w.scale)
+    torch.cuda.synchronize()
+    assert torch.equal(out8, out16) and torch.equal(lse8, lse16)
+
+
+def test_gta_fp8_argument_errors(L, gpu):
+    w, d, rows, codes, scales, kpe = _fp8_gta_case([40, 50])
+    q, qr, cu = d["q"].to(gpu), d["q_rope"].to(gpu), d["cu_seqlens"].to(gpu)
+    short = torch.zeros((rows.shape[0], 1152), dtype=torch.uint8, device=gpu)
+    with pytest.raises(L.LkvError) as e:   # rows shorter than the 1168-byte FP8 row
+        L.gta_group_decode_fp8(q, qr, short, w.groups, cu, w.scale)
+    assert e.value.status == L.ERR_INVALID_ARG
+    with pytest.raises(L.LkvError) as e:   # one group: 256 rows per unit, more than the converters leave room for
+        L.gta_group_decode_fp8(q, qr, rows.to(gpu), 1, cu, w.scale)
+    assert e.value.status == L.ERR_UNSUPPORTED

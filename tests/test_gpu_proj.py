@@ -67,6 +67,59 @@ def test_expand_latent_from_interleaved_cache(L, gpu, T, G, r, d):
     _check(L.expand_latent(c, w), oracle.expand_latent(_f64(c), _f64(w)))
 
 
+def _nan_out(shape, gpu, dtype=torch.bfloat16):
+    return torch.full(shape, float("nan"), dtype=dtype, device=gpu)
+
+
+@pytest.mark.parametrize("n_tok,h_q,G,d_h,r", [(9, 12, 2, 64, 520), (3, 24, 8, 128, 64), (200, 4, 1, 32, 256)])
+def test_absorb_every_element_written_once(L, gpu, n_tok, h_q, G, d_h, r):
+    """Odd heads per group (6, 3: tiles of 2 and 1 head rows x tokens), r over several column tiles,
+    a NaN-filled output: every element is written, by the right group's weights."""
+    rng = np.random.default_rng(h_q + r)
+    q = _bf(rng.standard_normal((n_tok, h_q, d_h)), gpu)
+    w = _bf(rng.standard_normal((G, r, d_h)) / math.sqrt(d_h), gpu)
+    out = L.absorb_query(q, w, out=_nan_out((n_tok, h_q, r), gpu))
+    assert not torch.isnan(out).any()
+    _check(out, oracle.absorb_query(_f64(q), _f64(w), G))
+
+
+@pytest.mark.parametrize("n_tok,h_q,G,r,d_v", [(5, 12, 3, 136, 200), (33, 128, 8, 512, 128), (2, 2, 2, 64, 8)])
+def test_unabsorb_every_element_written_once(L, gpu, n_tok, h_q, G, r, d_v):
+    rng = np.random.default_rng(h_q + d_v)
+    o = _bf(rng.standard_normal((n_tok, h_q, r)), gpu)
+    w = _bf(rng.standard_normal((G, r, d_v)) / math.sqrt(r), gpu)
+    out = L.unabsorb_output(o, w, out=_nan_out((n_tok, h_q, d_v), gpu))
+    assert not torch.isnan(out).any()
+    _check(out, oracle.unabsorb_output(_f64(o), _f64(w), G))
+
+
+@pytest.mark.parametrize("T,G,r,d", [(130, 3, 64, 40), (257, 5, 128, 64), (129, 1, 512, 512)])
+def test_expand_every_element_written_once(L, gpu, T, G, r, d):
+    """d not a multiple of 64 (one column block per group), groups side by side across a tile edge
+    (5 x 64 columns in tiles of 192), one wide group over two column tiles."""
+    rng = np.random.default_rng(T + d)
+    c = _bf(rng.standard_normal((T, r)), gpu)
+    w = _bf(rng.standard_normal((G, r, d)) / math.sqrt(r), gpu)
+    x = L.expand_latent(c, w, out=_nan_out((T, G, d), gpu))
+    assert not torch.isnan(x).any()
+    _check(x, oracle.expand_latent(_f64(c), _f64(w)))
+
+
+def test_expand_full_cache_sampled_rows(L, gpu):
+    """The expansion of a long cache (65536 rows of the interleaved [T, 576] cache into 8 groups of
+    128): 512 sampled rows against the oracle, and no row left unwritten."""
+    rng = np.random.default_rng(17)
+    T, G, r, d = 65536, 8, 512, 128
+    cache = torch.randn((T, r + 64), generator=torch.Generator(device=gpu).manual_seed(3), device=gpu).bfloat16()
+    w = _bf(rng.standard_normal((G, r, d)) / math.sqrt(r), gpu)
+    x = L.expand_latent(cache[:, :r], w, out=_nan_out((T, G, d), gpu))
+    assert not torch.isnan(x).any()
+    rows = np.sort(rng.choice(T, 512, replace=False))
+    rows[-1] = T - 1
+    rows_t = torch.from_numpy(rows).to(gpu)
+    _check(x[rows_t], oracle.expand_latent(_f64(cache[rows_t, :r]), _f64(w)))
+
+
 def test_projection_argument_errors(L, gpu):
     q = torch.zeros((4, 6, 8), dtype=torch.bfloat16, device=gpu)
     w = torch.zeros((4, 16, 8), dtype=torch.bfloat16, device=gpu)
@@ -130,6 +183,12 @@ def test_projection_throughput(L, gpu):
     cases.append(("unabsorb 64 tok x 128 heads, g=8", lambda: L.unabsorb_output(o, wv), 2 * 64 * 128 * 512 * 128))
     c = _bf(rng.standard_normal((4096, 512)), gpu)
     cases.append(("expand 4096 rows to g=8 x 128", lambda: L.expand_latent(c, wk), 2 * 4096 * 512 * 8 * 128))
+    cl = torch.randn((65536, 512), device=gpu).bfloat16()
+    cases.append(("expand 65536 rows to g=8 x 128", lambda: L.expand_latent(cl, wk), 2 * 65536 * 512 * 8 * 128))
+    ob = _bf(rng.standard_normal((64, 128 * 128)), gpu)
+    wo = _bf(rng.standard_normal((128 * 128, 7168)) / 128, gpu)
+    cases.append(("output projection 64 tok, 16384 -> 7168", lambda: L.output_projection(ob, wo),
+                  2 * 64 * 16384 * 7168))
     for name, fn, flops in cases:
         for _ in range(3):
             fn()

@@ -1,6 +1,6 @@
 """Pin the FP8 (e4m3) oracle: every code against torch's float8_e4m3fn conversion (an independent
 library routine), closed-form values of the format, round-to-nearest-even ties, the error bound of a
-3-bit mantissa, and the per-token scale rules."""
+3-bit mantissa, and the per-token power-of-two scale (its defining property and closed forms)."""
 import math
 
 import numpy as np
@@ -69,16 +69,33 @@ def test_quantize_rows_scale_and_error_bound():
     rng = np.random.default_rng(1)
     x = torch.from_numpy(rng.standard_normal((64, 512)).astype(np.float32) / 24).bfloat16().float().numpy()
     x[3] *= 1e-30                                            # tiny row: scale still exact in fp32
+    x[5] *= 2.0 ** 40
     codes, scales = fp8.quantize_rows(x)
-    amax = np.abs(x).max(axis=1)
-    np.testing.assert_array_equal(scales, (amax / np.float32(448)).astype(np.float32))
-    # the largest entry of every row maps to +-448 exactly
+    amax = np.abs(x).max(axis=1).astype(np.float64)
+    s64 = scales.astype(np.float64)
+    # the scale's defining property, checked directly: a power of two, the smallest one that
+    # brings amax within 448
+    m, _ = np.frexp(s64)
+    assert (m == 0.5).all()
+    assert (amax / s64 <= 448).all() and (amax / (s64 / 2) > 448).all()
+    # the largest entry of every row lands in the top binade of e4m3, (224, 448]
     mag = codes & 0x7F
-    assert (mag.max(axis=1) == 0x7E).all()
+    assert ((mag.max(axis=1) >= 0x70) & (mag.max(axis=1) <= 0x7E)).all()
     deq = fp8.dequantize_rows(codes, scales)
     # 3 mantissa bits: half an ulp is 2^-4 relative for normals, 2^-10 * s absolute below 2^-6 * s
-    bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * scales[:, None].astype(np.float64)) * (1 + 1e-6)
+    bound = np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10 * s64[:, None]) * (1 + 1e-6)
     assert (np.abs(deq - x) <= bound + 1e-300).all()
+    # and the dequantised values are exact in bf16 (a power-of-two scale times a 4-bit significand)
+    assert np.array_equal(torch.from_numpy(deq).bfloat16().double().numpy(), deq)
+
+
+def test_pow2_scale_closed_forms():
+    assert fp8.pow2_scale([448.0])[0] == 1.0                  # 448 / 1 fits, 448 / 0.5 does not
+    assert fp8.pow2_scale([449.0])[0] == 2.0
+    assert fp8.pow2_scale([1.0])[0] == 2.0 ** -8              # 1 / 2^-8 = 256 <= 448 < 512
+    assert fp8.pow2_scale([1.75])[0] == 2.0 ** -8             # 1.75 * 2^8 = 448 exactly
+    assert fp8.pow2_scale([1.76])[0] == 2.0 ** -7
+    assert fp8.pow2_scale([0.0])[0] == 0.0
 
 
 def test_zero_row_and_exactly_representable_row():

@@ -84,6 +84,9 @@ FP8_MUTANTS = {
     "dequant_divides": ("return e4m3_decode(codes) * np.asarray(scales, dtype=np.float64)[:, None]",
                         "return e4m3_decode(codes) / np.asarray(scales, dtype=np.float64)[:, None]"),
     "y_off_by_one_percent": ("y = np.clip(y, -E4M3_MAX, E4M3_MAX)", "y = y * np.float32(1.01)"),
+    "scale_one_binade_high": ("e = np.where(m <= 0.875, E - 9, E - 8)", "e = np.where(m <= 0.875, E - 8, E - 7)"),
+    "scale_threshold_strict": ("e = np.where(m <= 0.875, E - 9, E - 8)", "e = np.where(m < 0.875, E - 9, E - 8)"),
+    "scale_not_power_of_two": ("scales = pow2_scale(amax)", "scales = (amax / np.float32(E4M3_MAX)).astype(np.float32)"),
 }
 
 
