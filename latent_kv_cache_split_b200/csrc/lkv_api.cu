@@ -127,9 +127,18 @@ lkv_status launch_combine(const TcParams& p, int units_per_req, int per_query_un
   c.hpg = p.hpg;
   c.out = p.out;
   c.lse = p.lse;
-  const dim3 cgrid(p.B * units_per_req, (p.R + kCombineWarps - 1) / kCombineWarps);
-  combine_kernel<<<cgrid, kCombineWarps * 32, 0, stream>>>(c);
-  return launch_err(cudaGetLastError());
+  // a programmatic dependent of the decode kernel: its launch overlaps the decode's run, and its
+  // blocks wait (griddepcontrol.wait) for the decode's completion before reading the partials
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.B * units_per_req, (p.R + kCombineWarps - 1) / kCombineWarps);
+  cfg.blockDim = dim3(kCombineWarps * 32);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return launch_err(cudaLaunchKernelEx(&cfg, combine_kernel, c));
 }
 
 struct TcLaunch {

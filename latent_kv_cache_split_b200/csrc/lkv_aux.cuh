@@ -176,6 +176,7 @@ struct CombineParams {
 constexpr int kCombineWarps = 4;
 
 __global__ void __launch_bounds__(kCombineWarps * 32) combine_kernel(const CombineParams p) {
+  griddep_wait();  // launched as a programmatic dependent of the decode kernel: its writes first
   __shared__ int lo, hi;
   const int u = blockIdx.x;
   const int tid = threadIdx.x;

@@ -323,6 +323,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (tid == 0) griddep_launch_dependents();  // the split combine may start launching
   const uint32_t tbase = sm.tmem_base;
   const WaitCtl wc{&sm.abort, p.err, p.wait_limit_ns};
 

@@ -59,6 +59,7 @@ struct GemmParams {
   void* out;
   int* err;
   unsigned long long wait_limit_ns;
+  int m_tiles;        // weight-resident kernel: row tiles per column tile (t1 * t2)
 };
 
 struct __align__(8) GemmSmem {
@@ -115,6 +116,24 @@ __device__ __forceinline__ void gemm_store32(const GemmParams& p, long long off,
 #pragma unroll
     for (int i = 0; i < 32; ++i)
       if (i < n) o[i] = static_cast<uint16_t>(h[i >> 1] >> (16 * (i & 1)));
+  }
+}
+
+// One epilogue warp's share of a finished tile: TMEM lane quadrant qd (row m of the tile), column
+// half `half`, from the accumulator at TMEM address `acc` to the result rows.
+__device__ __forceinline__ void gemm_store_tile(const GemmParams& p, const GemmTile& x, uint32_t acc, int qd, int half,
+                                                int m) {
+  const int hc = p.tn >> 1;
+  const int u1 = x.i1 * p.b1 + (m & (p.b1 - 1));
+  const int u2 = x.i2 * p.b2 + (m >> p.lg_b1);
+  const bool row_ok = u1 < p.n1 && u2 < p.n2;
+  const long long row_off = u1 * p.os1 + u2 * p.os2 + x.g * p.ocol;
+  for (int c = half * hc; c < (half + 1) * hc; c += 32) {
+    uint32_t v[32];
+    tmem_ld32(acc + (static_cast<uint32_t>(32 * qd) << 16) + c, v);
+    tmem_wait_ld();
+    const int col = x.nt * p.tn + c;
+    if (row_ok) gemm_store32(p, row_off + col, v, p.n_valid - col);
   }
 }
 
@@ -234,24 +253,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int qd = warp & 3;
     const int half = (warp - 2) >> 2;
     const int m = 32 * qd + lane;
-    const int hc = p.tn >> 1;
     int lt = 0;
     for (int t = blockIdx.x; t < p.total_tiles; t += gridDim.x, ++lt) {
       const GemmTile x = gemm_tile(p, t);
       const int buf = lt & 1;
       if (!mbar_wait(bar(sm.tfull[buf]), (lt >> 1) & 1, wc, GW_TFULL)) break;
       tc_fence_after();
-      const int u1 = x.i1 * p.b1 + (m & (p.b1 - 1));
-      const int u2 = x.i2 * p.b2 + (m >> p.lg_b1);
-      const bool row_ok = u1 < p.n1 && u2 < p.n2;
-      const long long row_off = u1 * p.os1 + u2 * p.os2 + x.g * p.ocol;
-      for (int c = half * hc; c < (half + 1) * hc; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(32 * qd) << 16) + 256u * buf + c, v);
-        tmem_wait_ld();
-        const int col = x.nt * p.tn + c;
-        if (row_ok) gemm_store32(p, row_off + col, v, p.n_valid - col);
-      }
+      gemm_store_tile(p, x, tmem + 256u * buf, qd, half, m);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(sm.tempty[buf]));
@@ -262,6 +270,206 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   if (warp == 0 && lane == 0)
     for (int i = sm.consumed; i < sm.fills; ++i) mbar_wait(bar(sm.full[i % S]), (i / S) & 1, wd, GW_DRAIN);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kGemmTmemCols);
+  }
+}
+
+// ------------------------------------------------------------------------------------------
+// Weight-resident form, for an MN-major B shared by every row (the expansion, or an output
+// projection with K <= 512): each CTA keeps its column tile's whole B (K x 128 columns) in shared
+// memory and streams only A, so a tile's shared-memory fill is its 128 rows of A (the measured TMA
+// fill of one SM, ~83 GB/s from L2, is what bounds the streaming form).  The tiles are ordered
+// column-tile-major and each CTA takes one contiguous range of them, so B is reloaded only when the
+// range crosses into the next column tile.  A streams in stages of two 64-wide K blocks (32 KB).
+// ------------------------------------------------------------------------------------------
+constexpr int kResTn = 128;                              // columns per tile
+constexpr int kResMaxK = 512;                            // K of the resident B
+constexpr int kResBBytes = kResMaxK * kResTn * 2;        // 128 KB
+constexpr int kResStages = 3;
+constexpr int kResStageBytes = 2 * kGemmABytes;          // two K blocks of A
+constexpr size_t kResSmemBytes = 1024 + kResBBytes + static_cast<size_t>(kResStages) * kResStageBytes;
+static_assert(kResSmemBytes <= 232448 - 1024, "shared memory budget");
+
+struct __align__(8) GemmResSmem {
+  uint64_t full[kResStages], empty[kResStages];
+  uint64_t tfull[2], tempty[2];
+  uint64_t bfull;     // the resident B of the current column tile landed
+  uint64_t bfree;     // the MMAs reading the previous column tile's B are done
+  uint64_t drain;
+  uint32_t tmem_base, abort, zero;
+  int fills, consumed, bloads;
+};
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    proj_gemm_resident_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                              const GemmParams p) {
+  extern __shared__ __align__(1024) uint8_t gemm_res_raw[];
+  __shared__ GemmResSmem sm;
+  uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gemm_res_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  const uint32_t bres = smem_u32(dsm);
+  const uint32_t ring = bres + kResBBytes;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr int S = kResStages;
+  auto bar = [](const uint64_t& b) { return smem_u32(&b); };
+  // this CTA's tiles [t0, t1) in column-tile-major order
+  const int t0 = static_cast<int>(static_cast<long long>(p.total_tiles) * blockIdx.x / gridDim.x);
+  const int t1 = static_cast<int>(static_cast<long long>(p.total_tiles) * (blockIdx.x + 1) / gridDim.x);
+  const int kpairs = (p.k_blocks + 1) >> 1;              // A stages per tile
+  const uint32_t batom = static_cast<uint32_t>(p.k_blocks) * 8192u;  // bytes of one 64-column atom of B
+  auto tile_of = [&](int t) {
+    GemmTile x;
+    x.nt = t / p.m_tiles;
+    const int mt = t % p.m_tiles;
+    x.i1 = mt % p.t1;
+    x.i2 = mt / p.t1;
+    x.g = 0;
+    return x;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s2 = 0; s2 < S; ++s2) {
+      mbar_init(bar(sm.full[s2]), 1);
+      mbar_init(bar(sm.empty[s2]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(sm.tfull[b]), 1);
+      mbar_init(bar(sm.tempty[b]), 8);
+    }
+    mbar_init(bar(sm.bfull), 1);
+    mbar_init(bar(sm.bfree), 1);
+    mbar_init(bar(sm.drain), 1);
+    sm.abort = 0;
+    sm.zero = 0;
+    sm.fills = 0;
+    sm.consumed = 0;
+    sm.bloads = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&sm.tmem_base), kGemmTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const WaitCtl wc{&sm.abort, p.err, p.wait_limit_ns};
+  const WaitCtl wd{&sm.zero, p.err, p.wait_limit_ns};
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&map_a);
+      tma_prefetch_desc(&map_b);
+      int it = 0, nb_loads = 0, cur_nt = -1;
+      bool ok = true;
+      for (int t = t0; ok && t < t1; ++t) {
+        const GemmTile x = tile_of(t);
+        if (x.nt != cur_nt) {
+          // the previous column tile's MMAs must be done with B before it is overwritten
+          if (nb_loads > 0 && !mbar_wait(bar(sm.bfree), (nb_loads - 1) & 1, wc, GW_EMPTY)) break;
+          mbar_arrive_expect_tx(bar(sm.bfull), static_cast<uint32_t>(2 * batom));
+          for (int a = 0; a < 2; ++a) {
+            const int c0 = x.nt * kResTn + 64 * a;
+            for (int kb = 0; kb < p.k_blocks; ++kb)
+              tma_load_3d(bres + a * batom + kb * 8192, &map_b, bar(sm.bfull), c0 % p.nb, kb * 64, c0 / p.nb);
+          }
+          ++nb_loads;
+          sm.bloads = nb_loads;
+          cur_nt = x.nt;
+        }
+        for (int kp = 0; kp < kpairs; ++kp, ++it) {
+          const int s2 = it % S;
+          if (!mbar_wait(bar(sm.empty[s2]), ((it / S) & 1) ^ 1, wc, GW_EMPTY)) {
+            ok = false;
+            break;
+          }
+          const int nkb = (2 * kp + 1 < p.k_blocks) ? 2 : 1;
+          const uint32_t fb = bar(sm.full[s2]);
+          mbar_arrive_expect_tx(fb, static_cast<uint32_t>(nkb * kGemmABytes));
+          for (int j = 0; j < nkb; ++j)
+            tma_load_3d(ring + s2 * kResStageBytes + j * kGemmABytes, &map_a, fb, (2 * kp + j) * 64, x.i1 * p.b1,
+                        x.i2 * p.b2);
+          sm.fills = it + 1;
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, kResTn, 0, 1);
+      const uint64_t bd0 = sdesc_sw128(bres, batom, 1024);  // MN-major: 64-column atoms batom apart
+      int it = 0, lt = 0, nb_seen = 0, cur_nt = -1;
+      bool issued = false, ok = true;
+      for (int t = t0; ok && t < t1; ++t, ++lt) {
+        const GemmTile x = tile_of(t);
+        if (x.nt != cur_nt) {
+          if (!mbar_wait(bar(sm.bfull), nb_seen & 1, wc, GW_FULL)) break;
+          ++nb_seen;
+          cur_nt = x.nt;
+        }
+        const int buf = lt & 1;
+        if (!mbar_wait(bar(sm.tempty[buf]), ((lt >> 1) & 1) ^ 1, wc, GW_TEMPTY)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + 256u * buf;
+        for (int kp = 0; kp < kpairs; ++kp, ++it) {
+          const int s2 = it % S;
+          if (!mbar_wait(bar(sm.full[s2]), (it / S) & 1, wc, GW_FULL)) {
+            ok = false;
+            break;
+          }
+          sm.consumed = it + 1;
+          tc_fence_after();
+          const int nkb = (2 * kp + 1 < p.k_blocks) ? 2 : 1;
+          for (int j = 0; j < nkb; ++j) {
+            const int kb = 2 * kp + j;
+            const uint64_t ad = sdesc_sw128(ring + s2 * kResStageBytes + j * kGemmABytes, 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_ss(d, desc_add(ad, kk * 32), desc_add(bd0, kb * 8192 + kk * 2048), idesc, (kb | kk) ? 1u : 0u);
+          }
+          issued = true;
+          umma_commit(bar(sm.empty[s2]));
+        }
+        if (!ok) break;
+        umma_commit(bar(sm.tfull[buf]));
+        if (t + 1 == t1 || tile_of(t + 1).nt != x.nt) umma_commit(bar(sm.bfree));
+      }
+      if (issued) {
+        umma_commit(bar(sm.drain));
+        mbar_wait(bar(sm.drain), 0, wd, GW_DRAIN);
+      }
+    }
+  } else {
+    // ---------------- epilogue ----------------
+    const int qd = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int m = 32 * qd + lane;
+    int lt = 0;
+    for (int t = t0; t < t1; ++t, ++lt) {
+      const GemmTile x = tile_of(t);
+      const int buf = lt & 1;
+      if (!mbar_wait(bar(sm.tfull[buf]), (lt >> 1) & 1, wc, GW_TFULL)) break;
+      tc_fence_after();
+      gemm_store_tile(p, x, tmem + 256u * buf, qd, half, m);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(sm.tempty[buf]));
+    }
+  }
+
+  // Copies the MMA never waited for (after an abort) must land before the CTA's shared memory goes.
+  __syncthreads();
+  if (warp == 0 && lane == 0) {
+    for (int i = sm.consumed; i < sm.fills; ++i) mbar_wait(bar(sm.full[i % S]), (i / S) & 1, wd, GW_DRAIN);
+    if (sm.bloads > 0) mbar_wait(bar(sm.bfull), (sm.bloads - 1) & 1, wd, GW_DRAIN);
+  }
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

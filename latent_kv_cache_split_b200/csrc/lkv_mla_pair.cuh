@@ -206,6 +206,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   __syncthreads();
   cluster_sync();  // both CTAs' barriers exist before any remote arrive or pair load
   tc_fence_after();
+  if (tid == 0) griddep_launch_dependents();  // the split combine may start launching
   const uint32_t tbase = sm.tmem_base;
   const WaitCtl wc{&sm.abort, p.err, p.wait_limit_ns};
 

@@ -71,12 +71,27 @@ lkv_status launch(const CUtensorMap& ma, const CUtensorMap& mb, GemmParams& p, i
     std::lock_guard<std::mutex> lock(mu);
     if (!attr_set[dev]) {
       if (cudaFuncSetAttribute(proj_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kGemmSmemBytes)) != cudaSuccess)
+                               static_cast<int>(kGemmSmemBytes)) != cudaSuccess ||
+          cudaFuncSetAttribute(proj_gemm_resident_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kResSmemBytes)) != cudaSuccess)
         return LKV_ERR_CUDA;
       attr_set[dev] = true;
     }
   }
   p.k_blocks = cdiv(k, 64);
+  // Weight-resident form: one B for every row (MN-major, not chosen per row or per column block),
+  // K <= 512, and at least one 128-column tile per SM to spread.
+  const long long res_tiles = static_cast<long long>(cdiv(p.n_valid, kResTn)) * p.t1 * p.t2;
+  if (p.b_mn && p.rows_per_b == 0 && p.groups == 1 && p.k_blocks * 64 <= kResMaxK && res_tiles >= num_sms &&
+      res_tiles <= INT_MAX) {
+    p.tn = kResTn;
+    p.n_tiles = cdiv(p.n_valid, kResTn);
+    p.m_tiles = p.t1 * p.t2;
+    p.total_tiles = static_cast<int>(res_tiles);
+    proj_gemm_resident_kernel<<<num_sms, kGemmThreads, kResSmemBytes, s>>>(ma, mb, p);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? LKV_OK : LKV_ERR_CUDA;
+  }
   const long long tiles = static_cast<long long>(p.n_tiles) * p.t1 * p.t2 * p.groups;
   if (tiles <= 0 || tiles > INT_MAX) return LKV_ERR_INVALID_ARG;
   p.total_tiles = static_cast<int>(tiles);

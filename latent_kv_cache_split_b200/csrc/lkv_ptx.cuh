@@ -133,6 +133,16 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
 }
 
 // ----------------------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with programmatic stream serialization may
+// begin launching once every CTA of the kernel before it has called griddep_launch_dependents (or
+// exited); it must call griddep_wait before reading anything that kernel writes.
+// ----------------------------------------------------------------------------------------
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// ----------------------------------------------------------------------------------------
 // Cluster helpers
 // ----------------------------------------------------------------------------------------
 __device__ __forceinline__ uint32_t cluster_ctarank() {

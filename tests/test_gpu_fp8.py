@@ -96,7 +96,8 @@ def test_append_fp8_short_request_is_recorded(L, gpu):
     torch.cuda.synchronize()
     assert L.check_device(clear=True) == L.SITE_BAD_LENGTH
     # request 0 (L = 1) is skipped; request 1 (L = 9) writes rows 1 + 9 - 2 + i = 8, 9
-    assert (cache[:8] == 0).all() and (cache[8:10, :r] == 0x7E).all()   # ones quantise to 448
+    # ones: scale 2^-8 (the smallest power of two with 1 / s <= 448), code of 256 = 0x78
+    assert (cache[:8] == 0).all() and (cache[8:10, :r] == 0x78).all()
 
 
 def test_fp8_argument_errors(L, gpu):

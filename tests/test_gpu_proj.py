@@ -120,6 +120,20 @@ def test_expand_full_cache_sampled_rows(L, gpu):
     _check(x[rows_t], oracle.expand_latent(_f64(cache[rows_t, :r]), _f64(w)))
 
 
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_output_projection_weight_resident(L, gpu, out_dtype):
+    """An output projection with K <= 512 and >= one 128-column tile per SM runs the weight-resident
+    form (B kept in shared memory per column tile, tiles split in contiguous ranges): every element
+    against the oracle."""
+    rng = np.random.default_rng(21)
+    o = _bf(rng.standard_normal((4097, 384)), gpu)
+    w = _bf(rng.standard_normal((384, 1000)) / 20, gpu)
+    y = L.output_projection(o, w, out_dtype=out_dtype, out=torch.full((4097, 1000), float("nan"), dtype=out_dtype,
+                                                                      device=gpu))
+    assert not torch.isnan(y).any()
+    _check(y, oracle.output_projection(_f64(o), _f64(w)))
+
+
 def test_projection_argument_errors(L, gpu):
     q = torch.zeros((4, 6, 8), dtype=torch.bfloat16, device=gpu)
     w = torch.zeros((4, 16, 8), dtype=torch.bfloat16, device=gpu)
@@ -189,15 +203,25 @@ def test_projection_throughput(L, gpu):
     wo = _bf(rng.standard_normal((128 * 128, 7168)) / 128, gpu)
     cases.append(("output projection 64 tok, 16384 -> 7168", lambda: L.output_projection(ob, wo),
                   2 * 64 * 16384 * 7168))
+    # Device time per call: 20 calls captured in one CUDA graph (the host cost of a call -- tensor
+    # maps, argument marshalling -- is then outside the timed replay).
+    s = torch.cuda.Stream()
     for name, fn, flops in cases:
-        for _ in range(3):
-            fn()
+        with torch.cuda.stream(s):
+            for _ in range(3):
+                fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            for _ in range(20):
+                fn()
+        g.replay()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
-        for _ in range(20):
-            fn()
+        g.replay()
         e1.record()
         torch.cuda.synchronize()
+        assert L.check_device() == 0
         ms = e0.elapsed_time(e1) / 20
         print(f"{name}: {ms * 1e3:.1f} us, {flops / ms / 1e9:.1f} TFLOP/s")
