@@ -47,18 +47,22 @@ NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 # The sources the decode kernels and their launch are built from (the projections' translation unit
 # and the header's declarations do not change what a decode launch reads or writes).
-DECODE_SOURCES = ("lkv_api.cu", "lkv_aux.cuh", "lkv_decode_tc.cuh", "lkv_mla_pair.cuh", "lkv_ptx.cuh", "lkv_sched.cuh",
-                  "lkv_tma_host.h")
+# Device sources of each decode kernel: a traffic figure measured with ncu is only reported while the
+# kernel it was measured on is unchanged (host code and the other kernels do not count).
+KERNEL_SOURCES = {
+    "mla": ("lkv_mla_pair.cuh", "lkv_ptx.cuh", "lkv_sched.cuh"),
+    "grouped": ("lkv_decode_tc.cuh", "lkv_ptx.cuh", "lkv_sched.cuh"),
+}
+DECODE_SOURCES = tuple(sorted({f for v in KERNEL_SOURCES.values() for f in v}))
 
 
-def kernel_source_hash() -> str:
-    """Hash of the decode kernels' CUDA sources: a traffic figure measured with ncu is only
-    reported while the kernels it was measured on are unchanged."""
+def kernel_source_hash(kind: str = "mla") -> str:
+    """Hash of the CUDA sources of the decode kernel that a workload of this kind launches
+    ("mla" for the CTA-pair kernel, anything else for the grouped kernel)."""
     h = hashlib.sha256()
-    files = [os.path.join(ROOT, "latent_kv_cache_split_b200", "csrc", f) for f in DECODE_SOURCES]
-    for f in files:
-        h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
+    for f in KERNEL_SOURCES["mla" if kind == "mla" else "grouped"]:
+        h.update(f.encode())
+        with open(os.path.join(ROOT, "latent_kv_cache_split_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
@@ -78,7 +82,7 @@ def measured_traffic(workload: str):
     if not os.path.exists(p):
         return None
     entry = json.load(open(p)).get(workload)
-    if not entry or entry.get("kernel_hash") != kernel_source_hash():
+    if not entry or entry.get("kernel_hash") != kernel_source_hash(synth.workload(workload).kind):
         return None
     return entry.get("dram_bytes_per_launch")
 
@@ -695,7 +699,7 @@ def bench_gpu(args, rank, world, local_rank):
             "tflops": tfl,
             "roofline": {"bound": bound, "achieved": achieved, "peak": peak,
                          "unit": "GB/s" if bound == "hbm" else "TFLOP/s", "frac": achieved / peak,
-                         "traffic": measured_traffic(w.name), "kernel_source_hash": kernel_source_hash(),
+                         "traffic": measured_traffic(w.name), "kernel_source_hash": kernel_source_hash(w.kind),
                          "peak_source": f"{how} (MEASURED_PEAKS.json burst)",
                          "nominal": {"hbm_gbs": NOMINAL_PEAKS["hbm_gbs"], "bf16_tflops": NOMINAL_PEAKS["bf16_tflops"],
                                      "frac": max(alg_bytes / (NOMINAL_PEAKS["hbm_gbs"] * 1e9),

@@ -60,6 +60,7 @@ struct GemmParams {
   int* err;
   unsigned long long wait_limit_ns;
   int m_tiles;        // weight-resident kernel: row tiles per column tile (t1 * t2)
+  int res_groups;     // weight-resident kernel: CTAs per column tile (grid = res_groups * n_tiles)
 };
 
 struct __align__(8) GemmSmem {
@@ -280,11 +281,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
 // ------------------------------------------------------------------------------------------
 // Weight-resident form, for an MN-major B shared by every row (the expansion, or an output
-// projection with K <= 512): each CTA keeps its column tile's whole B (K x 128 columns) in shared
-// memory and streams only A, so a tile's shared-memory fill is its 128 rows of A (the measured TMA
-// fill of one SM, ~83 GB/s from L2, is what bounds the streaming form).  The tiles are ordered
-// column-tile-major and each CTA takes one contiguous range of them, so B is reloaded only when the
-// range crosses into the next column tile.  A streams in stages of two 64-wide K blocks (32 KB).
+// projection with K <= 512): each CTA keeps one column tile's whole B (K x 128 columns) in shared
+// memory for the whole launch and streams only A, so a tile's shared-memory fill is its 128 rows of
+// A (the measured TMA fill of one SM, ~83 GB/s from L2, is what bounds the streaming form).  CTA i
+// owns column tile i % n_tiles and row tiles i / n_tiles, + res_groups, ...: the n_tiles CTAs that
+// need one row tile's A take it at about the same time, so it comes from HBM once and from L2 for
+// the rest.  A streams in stages of two 64-wide K blocks (32 KB).
 // ------------------------------------------------------------------------------------------
 constexpr int kResTn = 128;                              // columns per tile
 constexpr int kResMaxK = 512;                            // K of the resident B
@@ -297,8 +299,7 @@ static_assert(kResSmemBytes <= 232448 - 1024, "shared memory budget");
 struct __align__(8) GemmResSmem {
   uint64_t full[kResStages], empty[kResStages];
   uint64_t tfull[2], tempty[2];
-  uint64_t bfull;     // the resident B of the current column tile landed
-  uint64_t bfree;     // the MMAs reading the previous column tile's B are done
+  uint64_t bfull;     // the resident B landed
   uint64_t drain;
   uint32_t tmem_base, abort, zero;
   int fills, consumed, bloads;
@@ -317,15 +318,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int lane = threadIdx.x & 31;
   constexpr int S = kResStages;
   auto bar = [](const uint64_t& b) { return smem_u32(&b); };
-  // this CTA's tiles [t0, t1) in column-tile-major order
-  const int t0 = static_cast<int>(static_cast<long long>(p.total_tiles) * blockIdx.x / gridDim.x);
-  const int t1 = static_cast<int>(static_cast<long long>(p.total_tiles) * (blockIdx.x + 1) / gridDim.x);
+  // this CTA's column tile and first row tile; its row tiles step by res_groups
+  const int nt = blockIdx.x % p.n_tiles;
+  const int mt0 = blockIdx.x / p.n_tiles;
   const int kpairs = (p.k_blocks + 1) >> 1;              // A stages per tile
   const uint32_t batom = static_cast<uint32_t>(p.k_blocks) * 8192u;  // bytes of one 64-column atom of B
-  auto tile_of = [&](int t) {
+  auto tile_of = [&](int mt) {
     GemmTile x;
-    x.nt = t / p.m_tiles;
-    const int mt = t % p.m_tiles;
+    x.nt = nt;
     x.i1 = mt % p.t1;
     x.i2 = mt / p.t1;
     x.g = 0;
@@ -342,7 +342,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(bar(sm.tempty[b]), 8);
     }
     mbar_init(bar(sm.bfull), 1);
-    mbar_init(bar(sm.bfree), 1);
     mbar_init(bar(sm.drain), 1);
     sm.abort = 0;
     sm.zero = 0;
@@ -367,23 +366,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&map_a);
       tma_prefetch_desc(&map_b);
-      int it = 0, nb_loads = 0, cur_nt = -1;
+      int it = 0;
       bool ok = true;
-      for (int t = t0; ok && t < t1; ++t) {
-        const GemmTile x = tile_of(t);
-        if (x.nt != cur_nt) {
-          // the previous column tile's MMAs must be done with B before it is overwritten
-          if (nb_loads > 0 && !mbar_wait(bar(sm.bfree), (nb_loads - 1) & 1, wc, GW_EMPTY)) break;
-          mbar_arrive_expect_tx(bar(sm.bfull), static_cast<uint32_t>(2 * batom));
-          for (int a = 0; a < 2; ++a) {
-            const int c0 = x.nt * kResTn + 64 * a;
-            for (int kb = 0; kb < p.k_blocks; ++kb)
-              tma_load_3d(bres + a * batom + kb * 8192, &map_b, bar(sm.bfull), c0 % p.nb, kb * 64, c0 / p.nb);
-          }
-          ++nb_loads;
-          sm.bloads = nb_loads;
-          cur_nt = x.nt;
+      if (mt0 < p.m_tiles) {
+        // this column tile's B, once
+        mbar_arrive_expect_tx(bar(sm.bfull), static_cast<uint32_t>(2 * batom));
+        for (int a = 0; a < 2; ++a) {
+          const int c0 = nt * kResTn + 64 * a;
+          for (int kb = 0; kb < p.k_blocks; ++kb)
+            tma_load_3d(bres + a * batom + kb * 8192, &map_b, bar(sm.bfull), c0 % p.nb, kb * 64, c0 / p.nb);
         }
+        sm.bloads = 1;
+      }
+      for (int mt = mt0; ok && mt < p.m_tiles; mt += p.res_groups) {
+        const GemmTile x = tile_of(mt);
         for (int kp = 0; kp < kpairs; ++kp, ++it) {
           const int s2 = it % S;
           if (!mbar_wait(bar(sm.empty[s2]), ((it / S) & 1) ^ 1, wc, GW_EMPTY)) {
@@ -405,15 +401,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16(128, kResTn, 0, 1);
       const uint64_t bd0 = sdesc_sw128(bres, batom, 1024);  // MN-major: 64-column atoms batom apart
-      int it = 0, lt = 0, nb_seen = 0, cur_nt = -1;
-      bool issued = false, ok = true;
-      for (int t = t0; ok && t < t1; ++t, ++lt) {
-        const GemmTile x = tile_of(t);
-        if (x.nt != cur_nt) {
-          if (!mbar_wait(bar(sm.bfull), nb_seen & 1, wc, GW_FULL)) break;
-          ++nb_seen;
-          cur_nt = x.nt;
-        }
+      int it = 0, lt = 0;
+      bool issued = false;
+      bool ok = mt0 >= p.m_tiles || mbar_wait(bar(sm.bfull), 0, wc, GW_FULL);
+      for (int mt = mt0; ok && mt < p.m_tiles; mt += p.res_groups, ++lt) {
         const int buf = lt & 1;
         if (!mbar_wait(bar(sm.tempty[buf]), ((lt >> 1) & 1) ^ 1, wc, GW_TEMPTY)) break;
         tc_fence_after();
@@ -439,7 +430,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (!ok) break;
         umma_commit(bar(sm.tfull[buf]));
-        if (t + 1 == t1 || tile_of(t + 1).nt != x.nt) umma_commit(bar(sm.bfree));
       }
       if (issued) {
         umma_commit(bar(sm.drain));
@@ -452,8 +442,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int half = (warp - 2) >> 2;
     const int m = 32 * qd + lane;
     int lt = 0;
-    for (int t = t0; t < t1; ++t, ++lt) {
-      const GemmTile x = tile_of(t);
+    for (int mt = mt0; mt < p.m_tiles; mt += p.res_groups, ++lt) {
+      const GemmTile x = tile_of(mt);
       const int buf = lt & 1;
       if (!mbar_wait(bar(sm.tfull[buf]), (lt >> 1) & 1, wc, GW_TFULL)) break;
       tc_fence_after();

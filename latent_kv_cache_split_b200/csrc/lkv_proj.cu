@@ -80,15 +80,18 @@ lkv_status launch(const CUtensorMap& ma, const CUtensorMap& mb, GemmParams& p, i
   }
   p.k_blocks = cdiv(k, 64);
   // Weight-resident form: one B for every row (MN-major, not chosen per row or per column block),
-  // K <= 512, and at least one 128-column tile per SM to spread.
-  const long long res_tiles = static_cast<long long>(cdiv(p.n_valid, kResTn)) * p.t1 * p.t2;
-  if (p.b_mn && p.rows_per_b == 0 && p.groups == 1 && p.k_blocks * 64 <= kResMaxK && res_tiles >= num_sms &&
-      res_tiles <= INT_MAX) {
+  // K <= 512, at most one CTA per SM for each 128-column tile and at least two row tiles per CTA.
+  const int res_n = cdiv(p.n_valid, kResTn);
+  const long long res_m = static_cast<long long>(p.t1) * p.t2;
+  const int res_groups = res_n <= num_sms ? num_sms / res_n : 0;
+  if (p.b_mn && p.rows_per_b == 0 && p.groups == 1 && p.k_blocks * 64 <= kResMaxK && res_groups > 0 &&
+      res_m >= 2LL * res_groups && res_m <= INT_MAX) {
     p.tn = kResTn;
-    p.n_tiles = cdiv(p.n_valid, kResTn);
-    p.m_tiles = p.t1 * p.t2;
-    p.total_tiles = static_cast<int>(res_tiles);
-    proj_gemm_resident_kernel<<<num_sms, kGemmThreads, kResSmemBytes, s>>>(ma, mb, p);
+    p.n_tiles = res_n;
+    p.m_tiles = static_cast<int>(res_m);
+    p.res_groups = res_groups;
+    p.total_tiles = static_cast<int>(res_m * res_n);
+    proj_gemm_resident_kernel<<<res_groups * res_n, kGemmThreads, kResSmemBytes, s>>>(ma, mb, p);
     const cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? LKV_OK : LKV_ERR_CUDA;
   }

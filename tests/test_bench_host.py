@@ -52,11 +52,15 @@ def test_roofline_accounting_matches_the_pinned_oracle(name):
     assert flops == acc.step_flops(lengths, w.s_q, w.h_q, w.d_k, w.d_v, w.d_rope)
 
 
-def test_source_hash_covers_only_the_decode_sources():
-    h = bench.kernel_source_hash()
+def test_source_hash_covers_only_the_decode_kernel_sources():
+    h = bench.kernel_source_hash("mla")
     assert len(h) == 16
-    assert "lkv_proj.cu" not in bench.DECODE_SOURCES and "lkv_fp8.cu" not in bench.DECODE_SOURCES
-    assert bench.kernel_source_hash() == h                   # deterministic
+    for f in ("lkv_proj.cu", "lkv_fp8.cu", "lkv_api.cu", "lkv_gemm.cuh"):
+        assert f not in bench.DECODE_SOURCES
+    assert "lkv_decode_tc.cuh" not in bench.KERNEL_SOURCES["mla"]
+    assert "lkv_mla_pair.cuh" not in bench.KERNEL_SOURCES["grouped"]
+    assert bench.kernel_source_hash("mla") == h                   # deterministic
+    assert bench.kernel_source_hash("gqla") == bench.kernel_source_hash("gta") != h
 
 
 def test_roofline_entry_is_the_slower_of_bytes_and_flops():

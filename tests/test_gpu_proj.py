@@ -126,9 +126,9 @@ def test_output_projection_weight_resident(L, gpu, out_dtype):
     form (B kept in shared memory per column tile, tiles split in contiguous ranges): every element
     against the oracle."""
     rng = np.random.default_rng(21)
-    o = _bf(rng.standard_normal((4097, 384)), gpu)
+    o = _bf(rng.standard_normal((8193, 384)), gpu)
     w = _bf(rng.standard_normal((384, 1000)) / 20, gpu)
-    y = L.output_projection(o, w, out_dtype=out_dtype, out=torch.full((4097, 1000), float("nan"), dtype=out_dtype,
+    y = L.output_projection(o, w, out_dtype=out_dtype, out=torch.full((8193, 1000), float("nan"), dtype=out_dtype,
                                                                       device=gpu))
     assert not torch.isnan(y).any()
     _check(y, oracle.output_projection(_f64(o), _f64(w)))
