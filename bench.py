@@ -50,7 +50,7 @@ NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 # Device sources of each decode kernel: a traffic figure measured with ncu is only reported while the
 # kernel it was measured on is unchanged (host code and the other kernels do not count).
 KERNEL_SOURCES = {
-    "mla": ("lkv_mla_pair.cuh", "lkv_ptx.cuh", "lkv_sched.cuh"),
+    "mla": ("lkv_mla_pair.cuh", "lkv_decode_tc.cuh", "lkv_ptx.cuh", "lkv_sched.cuh"),  # with the shared TMEM row helpers
     "grouped": ("lkv_decode_tc.cuh", "lkv_ptx.cuh", "lkv_sched.cuh"),
 }
 DECODE_SOURCES = tuple(sorted({f for v in KERNEL_SOURCES.values() for f in v}))

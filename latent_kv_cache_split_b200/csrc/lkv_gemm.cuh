@@ -286,7 +286,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 // A (the measured TMA fill of one SM, ~83 GB/s from L2, is what bounds the streaming form).  CTA i
 // owns column tile i % n_tiles and row tiles i / n_tiles, + res_groups, ...: the n_tiles CTAs that
 // need one row tile's A take it at about the same time, so it comes from HBM once and from L2 for
-// the rest.  A streams in stages of two 64-wide K blocks (32 KB).
+// the rest.  A streams in stages of two 64-wide K blocks (32 KB).  (Asking L2 for the next row
+// tile's A ahead of time was measured slower.)
 // ------------------------------------------------------------------------------------------
 constexpr int kResTn = 128;                              // columns per tile
 constexpr int kResMaxK = 512;                            // K of the resident B

@@ -25,9 +25,13 @@
 // of its S lanes, so the four threads of a head (two lane halves x two column halves) agree on the
 // row max through a bounded shared-memory exchange.
 //
-// Shared memory per CTA: Q (9 chunks of 64 heads x 64 columns), P (4 chunks of 64 heads x 64 keys)
-// and a ring of 32 KB stages that carries, in the MMA's order, the QK chunks of tile n+1 and then
-// the PV chunks of tile n; every load is a 16 KB box of 128 rows x 64 columns.  Ring stages are counted on the even CTA's barriers (the pair load
+// Shared memory per CTA: Q (9 chunks of 64 heads x 64 columns), P for one 128-key value chunk
+// (2 chunks of 64 heads x 64 keys) and a ring of four 32 KB stages that carries, in the MMA's
+// order, the QK chunks of tile n+1 and then the PV chunks of tile n; every load is a 16 KB box of
+// 128 rows x 64 columns.  P holds one value chunk at a time: the softmax threads of the tile's
+// first chunk (in PV order) write theirs, the PV of that chunk runs, and only then do the threads
+// of the second chunk write theirs over it.  Half a P buffer is what makes room for the fourth
+// stage, and the ring's depth is what bounds this kernel (it fills ~41 GB/s per SM with three).  Ring stages are counted on the even CTA's barriers (the pair load
 // form), released to both CTAs by the MMA's multicast commit.
 #pragma once
 #include <cstdint>
@@ -47,11 +51,11 @@ constexpr int kPairTile = 256;             // keys per tile (N of the QK MMA)
 // two thirds of that rate).  Per 256-key tile a CTA fills 4 stages of two 64-column key chunks,
 // 1 stage with the RoPE key chunk, and 1 stage per 128-key value chunk and dims block: this CTA's
 // 128 dims of the block as two 64-dim boxes.
-constexpr int kPairStages = 3;             // ring stages
+constexpr int kPairStages = 4;             // ring stages
 constexpr int kPairStageBytes = 32768;
 constexpr int kPairChunkBytes = 16384;     // one box: 128 keys x 64 columns
 constexpr int kPairQBytes = 9 * 8192;      // 64 heads x (512 + 64) columns
-constexpr int kPairPBytes = 4 * 8192;      // 64 heads x 256 keys
+constexpr int kPairPBytes = 2 * 8192;      // 64 heads x 128 keys (one value chunk)
 constexpr int kPairQOff = 0;
 constexpr int kPairPOff = kPairQBytes;
 constexpr int kPairRingOff = kPairQBytes + kPairPBytes;
@@ -65,7 +69,7 @@ static_assert(kPairSmemBytes <= 232448 - 4096, "shared memory budget");
 #define LKV_WAIT_BASE_PAIR(x) (LKV_SITE_WAIT_BASE + (x))
 enum PairWaitSite {
   PW_EMPTY = 80, PW_FULL, PW_QFULL, PW_QFREE, PW_SFULL, PW_SFREE, PW_PFULL, PW_PVDONE, PW_OFREE, PW_VLAND,
-  PW_XCHG, PW_DRAIN
+  PW_XCHG, PW_DRAIN, PW_PLO, PW_PFULL2
 };
 
 struct __align__(16) PairSmem {
@@ -75,7 +79,10 @@ struct __align__(16) PairSmem {
   uint64_t q_free;              // each CTA: the last QK of the current unit is done
   uint64_t s_full[2];           // each CTA: QK of the tile in S buffer b is done
   uint64_t s_free[2];           // even CTA: all 16 softmax warps read S buffer b
-  uint64_t p_full;              // even CTA: all 16 softmax warps wrote P (and rescaled O)
+  uint64_t p_full;              // even CTA: all 16 softmax warps are done with the tile (P of its
+                                // first value chunk written, O rescaled, rows past the end cleared)
+  uint64_t p_lo_free;           // each CTA: the PV of the tile's first value chunk is done
+  uint64_t p_full2;             // even CTA: the 8 warps of the second value chunk wrote its P
   uint64_t pv_done;             // each CTA: PV of the tile is done (P free, O settled)
   uint64_t o_free;              // even CTA: the epilogue of the last unit read O
   uint64_t vland;               // each CTA: the chunk to clear past the cache end has landed
@@ -164,6 +171,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       mbar_init(smem_u32(&sm.s_free[b]), 16);
     }
     mbar_init(smem_u32(&sm.p_full), 16);
+    mbar_init(smem_u32(&sm.p_lo_free), 1);
+    mbar_init(smem_u32(&sm.p_full2), 8);
     mbar_init(smem_u32(&sm.pv_done), 1);
     mbar_init(smem_u32(&sm.o_free), 16);
     mbar_init(smem_u32(&sm.vland), 1);
@@ -322,7 +331,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       Segment sg, psg{};
       int pt = 0, pn = 0, pseg = 0;
       bool have_prev = false, ok = true;
-      int n = 0, ch = 0, seg = 0;
+      int n = 0, ch = 0, seg = 0, n2 = 0;  // n2: tiles with two value chunks so far
       auto full_wait = [&](int c) -> bool {
         return mbar_wait<true>(smem_u32(&sm.full[c % KS]), static_cast<uint32_t>((c / KS) & 1), wc,
                                LKV_WAIT_BASE_PAIR(PW_FULL));
@@ -353,15 +362,23 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           return false;
         tc_fence_after();
         for (int i = 0; i < 2 * nkc; ++i) {
-          const int kc = pair_pv_chunk(i, nkc, cross);
           const int b = i & 1;
+          if (i == 2) {
+            // the first value chunk's PV must be done before its P is overwritten by the second's
+            umma_pair_commit(smem_u32(&sm.p_lo_free), kBothCtas);
+            if (!mbar_wait<true>(smem_u32(&sm.p_full2), static_cast<uint32_t>(n2 & 1), wc,
+                                 LKV_WAIT_BASE_PAIR(PW_PFULL2)))
+              return false;
+            ++n2;
+            tc_fence_after();
+          }
           if (!full_wait(ch)) return false;
           tc_fence_after();
-          // P keys 128 kc + 16 kk: 64-key chunk 2 kc + kk / 4; V: two 64-dim boxes 16 KB apart
+          // P keys 16 kk of the current value chunk: 64-key chunk kk / 4; V: two 64-dim boxes 16 KB apart
           const uint64_t vd = sdesc_sw128(ring_base + (ch % KS) * kPairStageBytes, kPairChunkBytes, 1024);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk) {
-            const uint64_t pd = sdesc_sw128(p_base + (2 * kc + (kk >> 2)) * 8192, 16, 1024);
+            const uint64_t pd = sdesc_sw128(p_base + (kk >> 2) * 8192, 16, 1024);
             umma_pair_ss(tbase + 128 * b, desc_add(pd, (kk & 3) * 32), desc_add(vd, kk * 2048), id_pv,
                          (first && i < 2 && kk == 0) ? 0u : 1u);
           }
@@ -458,7 +475,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     float m_run = -INFINITY, l_run = 0.f, lb_run = 0.f;
     SegCursor cur = cur0;
     Segment sg;
-    int n = 0, ncross = 0;
+    int n = 0, ncross = 0, n2s = 0;  // n2s: tiles with two value chunks so far
     bool ok = true;
     while (ok && cur.next(sa, sg)) {
       for (int t = sg.tile_lo; ok && t < sg.tile_hi; ++t, ++n) {
@@ -534,14 +551,19 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           tc_fence_after();
           tmem_scale_row(trow + 128 * chh, 128, alpha);  // this lane's 128 columns of dims block chh
         }
-        // this thread's 64 keys of P: row m of key chunk 2 kh + chh (K-major, 128-byte swizzle)
-        {
-          uint8_t* prow = dsm + kPairPOff + (2 * kh + chh) * 8192 + m * 128;
+        // This thread's 64 keys of P belong to value chunk kh; the P buffer holds one chunk at a
+        // time, the tile's first in PV order (the last chunk when the tile crosses the cache end)
+        // now and the other after its PV.  Row m of 64-key chunk chh (K-major, 128-byte swizzle).
+        const int nkc_t = pair_pv_chunks(sg, t);
+        const int kc_first = pair_crosses_end(sg, t, T_end) ? nkc_t - 1 : 0;
+        auto write_p = [&]() {
+          uint8_t* prow = dsm + kPairPOff + chh * 8192 + m * 128;
 #pragma unroll
           for (int c = 0; c < 8; ++c)
             *reinterpret_cast<uint4*>(prow + ((c ^ (m & 7)) << 4)) =
                 make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-        }
+        };
+        if (kh == kc_first) write_p();
         fence_proxy_async_smem();
         if (pair_crosses_end(sg, t, T_end)) {
           // clear this CTA's latent rows past the cache end in the tile's last value chunk (two
@@ -568,6 +590,19 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         arrive_lead(sm.p_full);
+        if (nkc_t == 2) {
+          // the second value chunk's threads: their P once the first chunk's PV is done
+          if (kh != kc_first) {
+            if (!wait_all(smem_u32(&sm.p_lo_free), static_cast<uint32_t>(n2s & 1), LKV_WAIT_BASE_PAIR(PW_PLO))) {
+              ok = false;
+              break;
+            }
+            write_p();
+            fence_proxy_async_smem();
+            arrive_lead(sm.p_full2);
+          }
+          ++n2s;
+        }
         if (t != sg.tile_hi - 1) continue;
         // ---------------------------------------------------------- unit epilogue
         float lo[4], lbo[4];

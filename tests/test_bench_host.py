@@ -57,7 +57,6 @@ def test_source_hash_covers_only_the_decode_kernel_sources():
     assert len(h) == 16
     for f in ("lkv_proj.cu", "lkv_fp8.cu", "lkv_api.cu", "lkv_gemm.cuh"):
         assert f not in bench.DECODE_SOURCES
-    assert "lkv_decode_tc.cuh" not in bench.KERNEL_SOURCES["mla"]
     assert "lkv_mla_pair.cuh" not in bench.KERNEL_SOURCES["grouped"]
     assert bench.kernel_source_hash("mla") == h                   # deterministic
     assert bench.kernel_source_hash("gqla") == bench.kernel_source_hash("gta") != h
