@@ -469,4 +469,201 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// Split-K form, for few output tiles over a long K (a decode-size output projection: 64 tokens,
+// K = 16384): the S CTAs of a cluster (S = 2, 4 or 8) take one tile and a contiguous S-th of its K
+// blocks each.  Each CTA parks its fp32 partial tile in its own shared memory (the ring is free by
+// then); after a cluster barrier CTA c sums rows [c * 128 / S, (c + 1) * 128 / S) of all S partials
+// through distributed shared memory, in rank order (deterministic), and stores them.  Streaming
+// producer and MMA as in proj_gemm_kernel, one tile per cluster.
+// ------------------------------------------------------------------------------------------
+constexpr int kSplitRowPitch = 256 * 4 + 16;  // bytes per partial row (padded against bank conflicts)
+static_assert(128 * kSplitRowPitch <= kGemmStages * kGemmStageBytes, "partial tile fits the ring");
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    proj_gemm_splitk_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                            const GemmParams p, int splits) {
+  extern __shared__ __align__(1024) uint8_t gemm_sk_raw[];
+  __shared__ GemmSmem sm;
+  uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gemm_sk_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  const uint32_t ring = smem_u32(dsm);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr int S = kGemmStages;
+  auto bar = [](const uint64_t& b) { return smem_u32(&b); };
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int tile = blockIdx.x / splits;
+  const int kb0 = static_cast<int>(static_cast<long long>(p.k_blocks) * rank / splits);
+  const int kb1 = static_cast<int>(static_cast<long long>(p.k_blocks) * (rank + 1) / splits);
+  const GemmTile x = gemm_tile(p, tile);
+
+  if (threadIdx.x == 0) {
+    for (int s2 = 0; s2 < S; ++s2) {
+      mbar_init(bar(sm.full[s2]), 1);
+      mbar_init(bar(sm.empty[s2]), 1);
+    }
+    mbar_init(bar(sm.tfull[0]), 1);
+    mbar_init(bar(sm.drain), 1);
+    sm.abort = 0;
+    sm.zero = 0;
+    sm.fills = 0;
+    sm.consumed = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&sm.tmem_base), 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const WaitCtl wc{&sm.abort, p.err, p.wait_limit_ns};
+  const WaitCtl wd{&sm.zero, p.err, p.wait_limit_ns};
+  bool have = false;  // epilogue: this CTA's partial is in TMEM
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&map_a);
+      tma_prefetch_desc(&map_b);
+      const int row_b = p.rows_per_b ? (x.i1 * p.b1) / p.rows_per_b : 0;
+      const int c_tile = x.nt * p.tn;
+      for (int kb = kb0, it = 0; kb < kb1; ++kb, ++it) {
+        const int s2 = it % S;
+        if (!mbar_wait(bar(sm.empty[s2]), ((it / S) & 1) ^ 1, wc, GW_EMPTY)) break;
+        const uint32_t a_dst = ring + s2 * kGemmStageBytes;
+        const uint32_t b_dst = a_dst + kGemmABytes;
+        const uint32_t fb = bar(sm.full[s2]);
+        mbar_arrive_expect_tx(fb, kGemmABytes + p.b_bytes);
+        tma_load_3d(a_dst, &map_a, fb, kb * 64, x.i1 * p.b1, x.i2 * p.b2);
+        if (p.b_mn) {
+          for (int a = 0; a < (p.tn >> 6); ++a) {
+            const int c0 = c_tile + 64 * a;
+            tma_load_3d(b_dst + a * 8192, &map_b, fb, c0 % p.nb, kb * 64, x.g + row_b + c0 / p.nb);
+          }
+        } else {
+          tma_load_3d(b_dst, &map_b, fb, kb * 64, c_tile, x.g + row_b);
+        }
+        sm.fills = it + 1;
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(128, p.tn, 0, p.b_mn);
+      const uint32_t bstep = p.b_mn ? 2048u : 32u;
+      const uint32_t blbo = p.b_mn ? 8192u : 16u;
+      bool issued = false, ok = true;
+      for (int kb = kb0, it = 0; kb < kb1; ++kb, ++it) {
+        const int s2 = it % S;
+        if (!mbar_wait(bar(sm.full[s2]), (it / S) & 1, wc, GW_FULL)) {
+          ok = false;
+          break;
+        }
+        sm.consumed = it + 1;
+        tc_fence_after();
+        const uint32_t a_addr = ring + s2 * kGemmStageBytes;
+        const uint64_t ad = sdesc_sw128(a_addr, 16, 1024);
+        const uint64_t bd = sdesc_sw128(a_addr + kGemmABytes, blbo, 1024);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_ss(tmem, desc_add(ad, kk * 32), desc_add(bd, kk * bstep), idesc, (it | kk) ? 1u : 0u);
+        issued = true;
+        umma_commit(bar(sm.empty[s2]));
+      }
+      if (ok && issued) umma_commit(bar(sm.tfull[0]));
+      if (issued) {
+        umma_commit(bar(sm.drain));
+        mbar_wait(bar(sm.drain), 0, wd, GW_DRAIN);
+      }
+    }
+  } else {
+    // park this CTA's partial: TMEM lane quadrant qd, column half `half`
+    const int qd = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int m = 32 * qd + lane;
+    have = kb1 > kb0 && mbar_wait(bar(sm.tfull[0]), 0, wc, GW_TFULL);
+    have = __all_sync(0xffffffffu, have) != 0;
+    if (have) {
+      tc_fence_after();
+      const int hc = p.tn >> 1;
+      for (int c = half * hc; c < (half + 1) * hc; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem + (static_cast<uint32_t>(32 * qd) << 16) + c, v);
+        tmem_wait_ld();
+        float4* dst = reinterpret_cast<float4*>(dsm + m * kSplitRowPitch + c * 4);
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_float4(__uint_as_float(v[4 * i]), __uint_as_float(v[4 * i + 1]), __uint_as_float(v[4 * i + 2]),
+                               __uint_as_float(v[4 * i + 3]));
+      }
+    }
+  }
+  // Loads the MMA never waited for (after an abort) must land before the ring is reused.
+  __syncthreads();
+  if (warp == 0 && lane == 0)
+    for (int i = sm.consumed; i < sm.fills; ++i) mbar_wait(bar(sm.full[i % S]), (i / S) & 1, wd, GW_DRAIN);
+  __syncthreads();
+  // an empty K range (more splits than K blocks) parks zeros
+  if (warp >= 2 && kb1 <= kb0) {
+    const int m = 32 * (warp & 3) + lane;
+    const int half = (warp - 2) >> 2;
+    const int hc = p.tn >> 1;
+    for (int c = half * hc; c < (half + 1) * hc; c += 4)
+      *reinterpret_cast<float4*>(dsm + m * kSplitRowPitch + c * 4) = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  cluster_sync();  // every CTA's partial is parked
+  if (warp >= 2) {
+    // rows [r0, r0 + 128 / splits) of the tile, summed over the splits in rank order
+    const int rows = 128 / splits;
+    const int r0 = rank * rows;
+    const int t = threadIdx.x - 64;             // 0 .. 255
+    const int cpr = p.tn >> 2;                  // float4 columns per row
+    const uint32_t base = smem_u32(dsm);
+    for (int idx = t; idx < rows * cpr; idx += 256) {
+      const int rr = r0 + idx / cpr, c4 = idx % cpr;
+      const uint32_t off = base + static_cast<uint32_t>(rr * kSplitRowPitch + c4 * 16);
+      float4 acc = ld_cluster_f32x4(map_to_peer(off, 0u));
+      for (int k = 1; k < splits; ++k) {
+        const float4 v = ld_cluster_f32x4(map_to_peer(off, static_cast<uint32_t>(k)));
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
+      }
+      // the result row and column of this element group
+      const int u1 = x.i1 * p.b1 + (rr & (p.b1 - 1));
+      const int u2 = x.i2 * p.b2 + (rr >> p.lg_b1);
+      const int col = x.nt * p.tn + 4 * c4;
+      if (u1 >= p.n1 || u2 >= p.n2 || col >= p.n_valid) continue;
+      const long long o = u1 * p.os1 + u2 * p.os2 + x.g * p.ocol + col;
+      const int n = p.n_valid - col;
+      const float a4[4] = {acc.x, acc.y, acc.z, acc.w};
+      if (p.out_fp32) {
+        float* y = static_cast<float*>(p.out) + o;
+        if (p.vec_ok && n >= 4) {
+          *reinterpret_cast<float4*>(y) = acc;
+        } else {
+          for (int i = 0; i < 4 && i < n; ++i) y[i] = a4[i];
+        }
+      } else {
+        uint16_t* y = static_cast<uint16_t*>(p.out) + o;
+        const uint32_t lo = pack_bf16x2(acc.x, acc.y), hi = pack_bf16x2(acc.z, acc.w);
+        if (p.vec_ok && n >= 4) {
+          *reinterpret_cast<uint2*>(y) = make_uint2(lo, hi);
+        } else {
+          const uint32_t w2[2] = {lo, hi};
+          for (int i = 0; i < 4 && i < n; ++i) y[i] = static_cast<uint16_t>(w2[i >> 1] >> (16 * (i & 1)));
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  cluster_sync();  // no CTA leaves while a peer still reads its partial
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
 }  // namespace lkv

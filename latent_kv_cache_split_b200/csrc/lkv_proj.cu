@@ -73,7 +73,9 @@ lkv_status launch(const CUtensorMap& ma, const CUtensorMap& mb, GemmParams& p, i
       if (cudaFuncSetAttribute(proj_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(kGemmSmemBytes)) != cudaSuccess ||
           cudaFuncSetAttribute(proj_gemm_resident_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kResSmemBytes)) != cudaSuccess)
+                               static_cast<int>(kResSmemBytes)) != cudaSuccess ||
+          cudaFuncSetAttribute(proj_gemm_splitk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kGemmSmemBytes)) != cudaSuccess)
         return LKV_ERR_CUDA;
       attr_set[dev] = true;
     }
@@ -98,6 +100,32 @@ lkv_status launch(const CUtensorMap& ma, const CUtensorMap& mb, GemmParams& p, i
   const long long tiles = static_cast<long long>(p.n_tiles) * p.t1 * p.t2 * p.groups;
   if (tiles <= 0 || tiles > INT_MAX) return LKV_ERR_INVALID_ARG;
   p.total_tiles = static_cast<int>(tiles);
+  // Split-K form: fewer tiles than half the SMs over a long K (>= 2048; below that the cluster
+  // reduction costs more than it saves: a 512-wide un-absorb measured 10.5 against 8.4 us) -- the S
+  // CTAs of a cluster share a tile (S = 8, 4 or 2: the most that fit on the SMs with >= 4 K blocks
+  // each).
+  if (2 * tiles <= num_sms && p.k_blocks >= 32) {
+    int splits = 0;
+    for (int c = 8; c >= 2 && splits == 0; c >>= 1)
+      if (tiles * c <= num_sms && p.k_blocks >= 4 * c) splits = c;
+    if (splits) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3(static_cast<unsigned>(tiles * splits));
+      cfg.blockDim = dim3(kGemmThreads);
+      cfg.dynamicSmemBytes = kGemmSmemBytes;
+      cfg.stream = s;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = static_cast<unsigned>(splits);
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      const cudaError_t e = cudaLaunchKernelEx(&cfg, proj_gemm_splitk_kernel, ma, mb, p, splits);
+      if (e != cudaSuccess) cudaGetLastError();
+      return e == cudaSuccess ? LKV_OK : LKV_ERR_CUDA;
+    }
+  }
   const int grid = static_cast<int>(tiles < num_sms ? tiles : num_sms);
   proj_gemm_kernel<<<grid, kGemmThreads, kGemmSmemBytes, s>>>(ma, mb, p);
   const cudaError_t e = cudaGetLastError();
