@@ -666,4 +666,228 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// CTA-pair form of the weight-resident GEMM (tcgen05 cta_group::2): a pair computes 256 rows x 256
+// columns per tile, each CTA streaming its own 128 rows of A and holding its half (128 columns) of
+// the column tile's B for the whole launch.  One pair MMA multiplies each CTA's A rows by both
+// halves of B, so a CTA's A bytes carry twice the FLOPs of the one-CTA form (whose A stream, three
+// 32 KB stages beside the 128 KB B, bounds it).  For A with one row dimension (n2 = 1).  Pairs own
+// column tile pair % n_tiles and row tiles pair / n_tiles, + res_groups, ...; the A stages and B
+// are counted on the even CTA's barriers (pair-form TMA) and released to both CTAs by the MMA's
+// multicast commit, as in the MLA pair kernel.
+// ------------------------------------------------------------------------------------------
+constexpr int kPgTn = 256;
+constexpr int kPgStages = 3;
+constexpr int kPgStageBytes = 2 * kGemmABytes;
+constexpr size_t kPgSmemBytes = 1024 + kResBBytes + static_cast<size_t>(kPgStages) * kPgStageBytes;
+static_assert(kPgSmemBytes <= 232448 - 1024, "shared memory budget");
+enum PairGemmWaitSite { PG_EMPTY = LKV_SITE_WAIT_BASE + 130, PG_FULL, PG_TEMPTY, PG_TFULL, PG_BFULL, PG_DRAIN };
+constexpr uint16_t kPgBoth = 3, kPgEven = 1;  // multicast masks of a commit
+
+struct __align__(8) GemmPairSmem {
+  uint64_t full[kPgStages];   // even CTA: both CTAs' A of the stage landed
+  uint64_t empty[kPgStages];  // each CTA: the MMAs reading the stage are done (multicast commit)
+  uint64_t tfull[2];          // each CTA: accumulator b holds a finished tile (multicast commit)
+  uint64_t tempty[2];         // even CTA: the 16 epilogue warps of both CTAs read accumulator b
+  uint64_t bfull;             // even CTA: both CTAs' halves of B landed
+  uint64_t drain;             // even CTA: every MMA issued is complete
+  uint32_t tmem_base, abort;
+  int fills, b_issued;                  // this CTA's producer counts
+  int peer_fills, peer_b_issued;        // the odd CTA's, for the even CTA's drain
+  int stage_bytes[kPgStages];           // bytes per CTA of the last phase armed on each stage
+  int peer_stage_bytes[kPgStages];
+};
+
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    proj_gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b,
+                          const GemmParams p) {
+  extern __shared__ __align__(1024) uint8_t gemm_pair_raw[];
+  __shared__ GemmPairSmem sm;
+  uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gemm_pair_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  const uint32_t bres = smem_u32(dsm);
+  const uint32_t ring = bres + kResBBytes;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  constexpr int S = kPgStages;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = (rank == 0);
+  const int pair = blockIdx.x >> 1;
+  const int nt = pair % p.n_tiles;
+  const int mt0 = pair / p.n_tiles;
+  const int kpairs = (p.k_blocks + 1) >> 1;
+  const uint32_t batom = static_cast<uint32_t>(p.k_blocks) * 8192u;
+  auto bar = [](const uint64_t& b) { return smem_u32(&b); };
+  auto lead = [&](const uint64_t& b) -> uint32_t { return map_to_peer(smem_u32(&b), 0u); };
+
+  if (threadIdx.x == 0) {
+    for (int s2 = 0; s2 < S; ++s2) {
+      mbar_init(bar(sm.full[s2]), 1);
+      mbar_init(bar(sm.empty[s2]), 1);
+      sm.stage_bytes[s2] = 0;
+      sm.peer_stage_bytes[s2] = 0;
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar(sm.tfull[b]), 1);
+      mbar_init(bar(sm.tempty[b]), 16);
+    }
+    mbar_init(bar(sm.bfull), 1);
+    mbar_init(bar(sm.drain), 1);
+    sm.abort = 0;
+    sm.fills = 0;
+    sm.b_issued = 0;
+    sm.peer_fills = 0;
+    sm.peer_b_issued = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(&sm.tmem_base), kGemmTmemCols);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // both CTAs' barriers exist before any remote arrive or pair load
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+  const WaitCtl wc{&sm.abort, p.err, p.wait_limit_ns};
+
+  if (warp == 0) {
+    // ---------------- TMA producer (both CTAs) ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&map_a);
+      tma_prefetch_desc(&map_b);
+      int it = 0;
+      bool ok = true;
+      if (mt0 < p.m_tiles) {
+        // this CTA's half of the column tile's B: columns 256 nt + 128 rank .. +127, once
+        if (leader) mbar_arrive_expect_tx(bar(sm.bfull), 2u * 2u * batom);
+        for (int a = 0; a < 2; ++a) {
+          const int c0 = nt * kPgTn + 128 * static_cast<int>(rank) + 64 * a;
+          for (int kb = 0; kb < p.k_blocks; ++kb)
+            tma_load_3d_pair(bres + a * batom + kb * 8192, &map_b, lead(sm.bfull), c0 % p.nb, kb * 64, c0 / p.nb);
+        }
+        sm.b_issued = 1;
+      }
+      for (int mt = mt0; ok && mt < p.m_tiles; mt += p.res_groups) {
+        const int row = (2 * mt + static_cast<int>(rank)) * 128;  // this CTA's 128 rows of the pair tile
+        for (int kp = 0; kp < kpairs; ++kp, ++it) {
+          const int s2 = it % S;
+          if (!mbar_wait<true>(bar(sm.empty[s2]), ((it / S) & 1) ^ 1, wc, PG_EMPTY)) {
+            ok = false;
+            break;
+          }
+          const int nkb = (2 * kp + 1 < p.k_blocks) ? 2 : 1;
+          const int bytes = nkb * kGemmABytes;
+          if (leader) mbar_arrive_expect_tx(bar(sm.full[s2]), static_cast<uint32_t>(2 * bytes));
+          sm.stage_bytes[s2] = bytes;
+          for (int j = 0; j < nkb; ++j)
+            tma_load_3d_pair(ring + s2 * kPgStageBytes + j * kGemmABytes, &map_a, lead(sm.full[s2]), (2 * kp + j) * 64,
+                             row, 0);
+          sm.fills = it + 1;
+        }
+      }
+      if (!leader) {
+        st_cluster_u32(map_to_peer(smem_u32(&sm.peer_fills), 0u), static_cast<uint32_t>(sm.fills));
+        st_cluster_u32(map_to_peer(smem_u32(&sm.peer_b_issued), 0u), static_cast<uint32_t>(sm.b_issued));
+        for (int s2 = 0; s2 < S; ++s2)
+          st_cluster_u32(map_to_peer(smem_u32(&sm.peer_stage_bytes[s2]), 0u), static_cast<uint32_t>(sm.stage_bytes[s2]));
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (even CTA) ----------------
+    if (leader && lane == 0) {
+      const uint32_t idesc = idesc_bf16(256, kPgTn, 0, 1);   // 128 rows per CTA, B MN-major
+      const uint64_t bd0 = sdesc_sw128(bres, batom, 1024);
+      int it = 0, lt = 0;
+      bool issued = false;
+      bool ok = mt0 >= p.m_tiles || mbar_wait<true>(bar(sm.bfull), 0, wc, PG_BFULL);
+      for (int mt = mt0; ok && mt < p.m_tiles; mt += p.res_groups, ++lt) {
+        const int buf = lt & 1;
+        if (!mbar_wait<true>(bar(sm.tempty[buf]), ((lt >> 1) & 1) ^ 1, wc, PG_TEMPTY)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + 256u * buf;
+        for (int kp = 0; kp < kpairs; ++kp, ++it) {
+          const int s2 = it % S;
+          if (!mbar_wait<true>(bar(sm.full[s2]), (it / S) & 1, wc, PG_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nkb = (2 * kp + 1 < p.k_blocks) ? 2 : 1;
+          for (int j = 0; j < nkb; ++j) {
+            const int kb = 2 * kp + j;
+            const uint64_t ad = sdesc_sw128(ring + s2 * kPgStageBytes + j * kGemmABytes, 16, 1024);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_pair_ss(d, desc_add(ad, kk * 32), desc_add(bd0, kb * 8192 + kk * 2048), idesc, (kb | kk) ? 1u : 0u);
+          }
+          issued = true;
+          umma_pair_commit(bar(sm.empty[s2]), kPgBoth);
+        }
+        if (!ok) break;
+        umma_pair_commit(bar(sm.tfull[buf]), kPgBoth);
+      }
+      if (issued) {
+        umma_pair_commit(bar(sm.drain), kPgEven);
+        uint32_t zero = 0;
+        const WaitCtl dc{&zero, p.err, p.wait_limit_ns};
+        mbar_wait(bar(sm.drain), 0, dc, PG_DRAIN);
+      }
+    }
+  } else {
+    // ---------------- epilogue (both CTAs): this CTA's 128 rows x all 256 columns ----------------
+    const int qd = warp & 3;
+    const int half = (warp - 2) >> 2;
+    const int m = 32 * qd + lane;
+    int lt = 0;
+    for (int mt = mt0; mt < p.m_tiles; mt += p.res_groups, ++lt) {
+      const int buf = lt & 1;
+      const bool okw = __all_sync(0xffffffffu, mbar_wait<true>(bar(sm.tfull[buf]), (lt >> 1) & 1, wc, PG_TFULL)) != 0;
+      if (!okw) break;
+      tc_fence_after();
+      GemmTile x;
+      x.nt = nt;
+      x.i1 = 2 * mt + static_cast<int>(rank);
+      x.i2 = 0;
+      x.g = 0;
+      gemm_store_tile(p, x, tmem + 256u * buf, qd, half, m);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_pair(lead(sm.tempty[buf]));
+    }
+  }
+
+  // ---------------- teardown ----------------
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // the odd CTA's producer counts are visible; every remote arrive has been made
+  if (leader && warp == 0 && lane == 0) {
+    // Drain: no copy may still be landing in either CTA when they exit.  A phase one producer
+    // issued and the other did not (after a wait gave up) is completed for the missing side here.
+    uint32_t zero = 0;
+    const WaitCtl dc{&zero, p.err, p.wait_limit_ns};
+    const int nl = sm.fills, np = sm.peer_fills;
+    const int nmax = nl > np ? nl : np;
+    for (int i = (nmax > S ? nmax - S : 0); i < nmax; ++i) {
+      const uint32_t fb = bar(sm.full[i % S]);
+      if (i < nl && i >= np) mbar_complete_tx(fb, static_cast<uint32_t>(sm.stage_bytes[i % S]));
+      if (i >= nl && i < np) mbar_arrive_expect_tx(fb, static_cast<uint32_t>(sm.peer_stage_bytes[i % S]));
+      mbar_wait(fb, static_cast<uint32_t>((i / S) & 1), dc, PG_DRAIN);
+    }
+    if (sm.b_issued || sm.peer_b_issued) {
+      const uint32_t bb = bar(sm.bfull);
+      if (sm.b_issued && !sm.peer_b_issued) mbar_complete_tx(bb, 2u * batom);
+      if (!sm.b_issued && sm.peer_b_issued) mbar_arrive_expect_tx(bb, 2u * batom);
+      mbar_wait(bb, 0, dc, PG_DRAIN);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, kGemmTmemCols);
+  }
+}
+
 }  // namespace lkv

@@ -75,12 +75,42 @@ lkv_status launch(const CUtensorMap& ma, const CUtensorMap& mb, GemmParams& p, i
           cudaFuncSetAttribute(proj_gemm_resident_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(kResSmemBytes)) != cudaSuccess ||
           cudaFuncSetAttribute(proj_gemm_splitk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(kGemmSmemBytes)) != cudaSuccess)
+                               static_cast<int>(kGemmSmemBytes)) != cudaSuccess ||
+          cudaFuncSetAttribute(proj_gemm_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(kPgSmemBytes)) != cudaSuccess)
         return LKV_ERR_CUDA;
       attr_set[dev] = true;
     }
   }
   p.k_blocks = cdiv(k, 64);
+  // CTA-pair weight-resident form: as the one-CTA form below, with A of one row dimension and at
+  // least two 256-row tiles per pair.
+  const int pg_n = cdiv(p.n_valid, kPgTn);
+  const int pg_groups = pg_n <= num_sms / 2 ? (num_sms / 2) / pg_n : 0;
+  const long long pg_m = (static_cast<long long>(p.t1) + 1) / 2;
+  if (p.b_mn && p.rows_per_b == 0 && p.groups == 1 && p.n2 == 1 && p.k_blocks * 64 <= kResMaxK && pg_groups > 0 &&
+      pg_m >= 2LL * pg_groups && pg_m <= INT_MAX) {
+    p.tn = kPgTn;
+    p.n_tiles = pg_n;
+    p.m_tiles = static_cast<int>(pg_m);
+    p.res_groups = pg_groups;
+    p.total_tiles = static_cast<int>(pg_m * pg_n);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pg_groups * pg_n));
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = kPgSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, proj_gemm_pair_kernel, ma, mb, p);
+    if (e != cudaSuccess) cudaGetLastError();
+    return e == cudaSuccess ? LKV_OK : LKV_ERR_CUDA;
+  }
   // Weight-resident form: one B for every row (MN-major, not chosen per row or per column block),
   // K <= 512, at most one CTA per SM for each 128-column tile and at least two row tiles per CTA.
   const int res_n = cdiv(p.n_valid, kResTn);

@@ -134,6 +134,34 @@ def test_output_projection_weight_resident(L, gpu, out_dtype):
     _check(y, oracle.output_projection(_f64(o), _f64(w)))
 
 
+@pytest.mark.parametrize("T,G,r,d", [(9300, 8, 512, 128), (9301, 16, 320, 64)])
+def test_expand_cta_pair_form(L, gpu, T, G, r, d):
+    """Enough 256-row tiles for the CTA-pair form (two CTAs share each tile's MMAs, each holding half
+    of the column tile's weights): every element against the oracle, an odd number of 128-row
+    tiles, K not a multiple of 128 (a last stage of one K block)."""
+    rng = np.random.default_rng(T + r)
+    c = _bf(rng.standard_normal((T, r)), gpu)
+    w = _bf(rng.standard_normal((G, r, d)) / math.sqrt(r), gpu)
+    x = L.expand_latent(c, w, out=_nan_out((T, G, d), gpu))
+    torch.cuda.synchronize()
+    assert L.check_device() == 0
+    assert not torch.isnan(x).any()
+    _check(x, oracle.expand_latent(_f64(c), _f64(w)))
+
+
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_output_projection_cta_pair_form(L, gpu, out_dtype):
+    rng = np.random.default_rng(31)
+    o = _bf(rng.standard_normal((9300, 256)), gpu)
+    w = _bf(rng.standard_normal((256, 2048)) / 16, gpu)
+    y = L.output_projection(o, w, out_dtype=out_dtype, out=torch.full((9300, 2048), float("nan"), dtype=out_dtype,
+                                                                      device=gpu))
+    torch.cuda.synchronize()
+    assert L.check_device() == 0
+    assert not torch.isnan(y).any()
+    _check(y, oracle.output_projection(_f64(o), _f64(w)))
+
+
 def test_projection_argument_errors(L, gpu):
     q = torch.zeros((4, 6, 8), dtype=torch.bfloat16, device=gpu)
     w = torch.zeros((4, 16, 8), dtype=torch.bfloat16, device=gpu)
