@@ -51,7 +51,7 @@ NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 # kernel it was measured on is unchanged (host code and the other kernels do not count).
 KERNEL_SOURCES = {
     "mla": ("lkv_mla_pair.cuh", "lkv_decode_tc.cuh", "lkv_ptx.cuh", "lkv_sched.cuh"),  # with the shared TMEM row helpers
-    "grouped": ("lkv_decode_tc.cuh", "lkv_ptx.cuh", "lkv_sched.cuh"),
+    "grouped": ("lkv_decode_swap.cuh", "lkv_decode_tc.cuh", "lkv_ptx.cuh", "lkv_sched.cuh"),
 }
 DECODE_SOURCES = tuple(sorted({f for v in KERNEL_SOURCES.values() for f in v}))
 
@@ -67,10 +67,16 @@ def kernel_source_hash(kind: str = "mla") -> str:
     return h.hexdigest()[:16]
 
 
+SWAP_MAX_ROWS = 32  # GQLA / GTA units of at most this many query rows run keys-in-M
+
+
 def decode_kernel_name(w) -> str:
     """The tensor-core kernel a bf16 decode call of this workload launches."""
     if w.kind == "mla":
         return "mla_pair_kernel"
+    rows = (w.h_q // w.groups) * w.s_q
+    if w.kind in ("gqla", "gta") and rows <= SWAP_MAX_ROWS:
+        return "decode_swap_kernel<%s>" % ("true" if w.kind == "gta" else "false")
     return {"gqla": "decode_tc_kernel<MODE_GQLA>", "gla": "decode_tc_kernel<MODE_GLA>",
             "gta": "decode_tc_kernel<MODE_GTA>"}.get(w.kind, "decode_tc_kernel")
 

@@ -10,6 +10,7 @@
 #include "../../include/lkv.h"
 #include "lkv_aux.cuh"
 #include "lkv_decode_tc.cuh"
+#include "lkv_decode_swap.cuh"
 #include "lkv_mla_pair.cuh"
 #include "lkv_ptx.cuh"
 #include "lkv_tma_host.h"
@@ -66,7 +67,11 @@ lkv_status device_state(DeviceState** out) {
         cudaFuncSetAttribute(decode_tc_kernel<MODE_GTA8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(tc_smem_bytes(MODE_GTA8))) != cudaSuccess ||
         cudaFuncSetAttribute(mla_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(kPairSmemBytes)) != cudaSuccess)
+                             static_cast<int>(kPairSmemBytes)) != cudaSuccess ||
+        cudaFuncSetAttribute(decode_swap_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(swap_smem_bytes(false))) != cudaSuccess ||
+        cudaFuncSetAttribute(decode_swap_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(swap_smem_bytes(true))) != cudaSuccess)
       return LKV_ERR_CUDA;
     d.ready = true;
   }
@@ -149,7 +154,8 @@ struct TcLaunch {
   int per_query_units;
 };
 
-// Grouped decode (one CTA per range), then the split combine.
+// Grouped decode (one CTA per range), then the split combine.  GQLA and GTA units of at most 32
+// rows run with the keys in the MMA's M dimension (lkv_decode_swap.cuh); the rest row-major.
 lkv_status run_tc(TcLaunch& L, const DeviceState& d, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(L.p.P);
@@ -157,7 +163,15 @@ lkv_status run_tc(TcLaunch& L, const DeviceState& d, cudaStream_t stream) {
   cfg.dynamicSmemBytes = tc_smem_bytes(L.mode);
   cfg.stream = stream;
   cudaError_t e;
-  if (L.mode == MODE_GQLA) {
+  const bool swap = (L.mode == MODE_GQLA || L.mode == MODE_GTA) && L.p.R <= kSwapMaxRows;
+  if (swap) {
+    cfg.blockDim = dim3(kSwapThreads);
+    cfg.dynamicSmemBytes = swap_smem_bytes(L.mode == MODE_GTA);
+    if (L.mode == MODE_GTA)
+      e = cudaLaunchKernelEx(&cfg, decode_swap_kernel<true>, L.map_a, L.map_r, L.map_v, L.p);
+    else
+      e = cudaLaunchKernelEx(&cfg, decode_swap_kernel<false>, L.map_a, L.map_r, L.map_v, L.p);
+  } else if (L.mode == MODE_GQLA) {
     e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<MODE_GQLA>, L.map_a, L.map_r, L.map_v, L.p);
   } else if (L.mode == MODE_GTA) {
     e = cudaLaunchKernelEx(&cfg, decode_tc_kernel<MODE_GTA>, L.map_a, L.map_r, L.map_v, L.p);

@@ -1,0 +1,596 @@
+// Grouped decode with the keys in the MMA's M dimension, for units of at most 32 query rows
+// (GQLA groups, GTA tied groups; d_h = 128).
+//
+// Per group j the GQA path of the GQLA explainer (section 2) computes S = Q_j K_j^T over the
+// group's heads and O_j = softmax(S) V_j; GTA (GLA article, section "GTA") is the same with
+// K_j = V_j the tied state.  A unit holds hpg x s_q <= 32 rows, so the row-major form (S = Q K^T
+// with M = rows) fills 32 of the 128 rows of each tcgen05 MMA.  Here the products are transposed:
+//   S^T[key, row] = K[key, :] . Q[row, :]      M = 128 keys, N = 32 rows, K = 128 + 64 columns
+//   O^T[d, row]  += V^T[d, key] . P^T[key, row]  M = 128 value columns, N = 32 rows, K = 128 keys
+// so every MMA row is live and each MMA is a quarter of the row-major one.
+//
+// Warps: 0 TMA producer; 1 TMEM allocator and QK issuer; 2 PV issuer; 3 idle; 4-11 softmax /
+// epilogue.  Softmax warp w owns TMEM lane quadrant w % 4 and the 16 rows 16 h .. 16 h + 15,
+// h = (w - 4) / 4: its thread k (lane k of the quadrant) owns key k of the tile (lane k of S^T) for
+// those rows and value column d = k of O^T.  A row's tile max is a reduction over the 128 keys: a
+// reduce-scatter over the warp's lanes (16 shuffles, lane l ends with row l % 16), then the 4
+// quadrant warps' values through shared memory.  The row sums are kept per thread (one partial per
+// key lane and row) and reduced once, in the unit's epilogue.
+//
+// TMEM (128 columns): S^T buffers at columns 0 and 32 (128 keys x 32 rows, fp32), O^T at 64.
+// Shared memory: the key ring (two 64-column boxes of the group's key or tied state and the RoPE
+// key box per 128-key stage; in GQLA a separate value ring), the unit's Q as the K-major B operand
+// of QK (32 rows x 192 columns, three 128-byte-swizzled boxes) and two P^T buffers, the MN-major
+// B operand of PV (128 keys x 32 rows of bf16, 64-byte swizzle).
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+#include "lkv_ptx.cuh"
+#include "lkv_sched.cuh"
+#include "lkv_decode_tc.cuh"
+
+namespace lkv {
+
+constexpr int kSwapThreads = 384;
+constexpr int kSwapMaxRows = 32;  // N of every MMA: the unit's rows, zero-padded
+
+template <bool kTied>
+struct SwapCfg {
+  static constexpr int kTile = 128;                  // keys per tile = M of QK
+  static constexpr int kN = kSwapMaxRows;
+  static constexpr int kBoxBytes = kTile * 128;      // 128 keys x 64 bf16, 128-byte swizzle
+  static constexpr int kStageBytes = 3 * kBoxBytes;  // key (2 boxes) + RoPE key (1 box)
+  static constexpr int kStages = kTied ? 4 : 2;
+  static constexpr int kVStages = kTied ? 1 : 3;     // (no value ring when tied)
+  static constexpr int kVStageBytes = 2 * kBoxBytes;
+  static constexpr int kQBoxBytes = kN * 128;        // 32 rows x 64 bf16
+  static constexpr int kQBytes = 3 * kQBoxBytes;
+  static constexpr int kPBytes = kTile * kN * 2;     // 128 keys x 32 bf16
+  static constexpr size_t kRingBytes =
+      static_cast<size_t>(kStages) * kStageBytes + (kTied ? 0 : static_cast<size_t>(kVStages) * kVStageBytes);
+  static constexpr size_t kSmemBytes = 1024 + kRingBytes + kQBytes + 2 * kPBytes;
+  static constexpr uint32_t S0 = 0, O0 = 64;
+  static constexpr int kTmemCols = 128;
+  static constexpr int kSiteBase = LKV_SITE_WAIT_BASE + (kTied ? 240 : 260);  // wait sites of this kernel
+};
+static_assert(SwapCfg<true>::kSmemBytes <= 232448 - 4096, "shared memory budget");
+static_assert(SwapCfg<false>::kSmemBytes <= 232448 - 4096, "shared memory budget");
+
+template <int KS, int VS>
+struct __align__(16) SwapSmem {
+  uint64_t full[KS], empty[KS], vfull[VS], vempty[VS];
+  uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
+  uint64_t q_ready, o_free, drain;
+  uint64_t xb4[2];           // the 8 softmax warps posted one value per row (double-buffered)
+  float red[2][8][16];       // [buffer][softmax warp][row of its half]
+  float msub[8][16];         // per warp: the tile's row max (log2 units), subtracted in the exponent
+  float fac[8][16];          // per warp: 2^(tile max - running max) per row
+  float arow[8][16];         // per warp: O rescale factor per row, then 1 / l at the end
+  uint32_t tmem_base;
+  uint32_t abort;
+  long long t_begin, t_end, unit_t0;
+  int b0, k0;
+};
+
+template <bool kMax>
+__device__ __forceinline__ float rop(float a, float b) { return kMax ? fmaxf(a, b) : a + b; }
+
+// The same for 16 values (rows) per lane: a reduce-scatter over lanes differing in bits 3..0 leaves
+// lane l with row l % 16 over its 16-lane half; one exchange across the halves completes it.
+// 16 shuffles; lanes l and l + 16 end with the same value.
+template <bool kMax>
+__device__ __forceinline__ float warp_rows_reduce16(float (&v)[16], int lane) {
+#pragma unroll
+  for (int s = 8; s >= 1; s >>= 1) {
+    const bool up = (lane & s) != 0;
+#pragma unroll
+    for (int j = 0; j < s; ++j) {
+      const float send = up ? v[j] : v[j + s];
+      const float keep = up ? v[j + s] : v[j];
+      v[j] = rop<kMax>(keep, __shfl_xor_sync(0xffffffffu, send, s));
+    }
+  }
+  return rop<kMax>(v[0], __shfl_xor_sync(0xffffffffu, v[0], 16));
+}
+
+template <bool kTied>
+__global__ void __launch_bounds__(kSwapThreads, 1)
+    decode_swap_kernel(const __grid_constant__ CUtensorMap map_k,  // K (or the tied state) [rows, g*128], box 64 x 128
+                       const __grid_constant__ CUtensorMap map_r,  // RoPE key [rows, 64], box 64 x 128
+                       const __grid_constant__ CUtensorMap map_v,  // V [rows, g*128], box 64 x 128 (not tied)
+                       const TcParams p) {
+  using Cfg = SwapCfg<kTied>;
+  constexpr int TN = Cfg::kTile;
+  constexpr int KS = Cfg::kStages;
+  constexpr int VS = Cfg::kVStages;
+  constexpr int kBoxBytes = Cfg::kBoxBytes;
+  constexpr int kStageBytes = Cfg::kStageBytes;
+  constexpr uint32_t S0 = Cfg::S0, O0 = Cfg::O0;
+  constexpr int SB = Cfg::kSiteBase;
+
+  extern __shared__ __align__(1024) uint8_t swap_smem_raw[];
+  __shared__ SwapSmem<KS, VS> sm;
+  uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(swap_smem_raw) + 1023) &
+                                            ~static_cast<uintptr_t>(1023));
+  const uint32_t stage_base = smem_u32(dsm);
+  uint8_t* vring = dsm + KS * kStageBytes;
+  const uint32_t vring_base = smem_u32(vring);
+  uint8_t* qsm = dsm + Cfg::kRingBytes;
+  const uint32_t q_base = smem_u32(qsm);
+  uint8_t* psm = qsm + Cfg::kQBytes;
+  const uint32_t p_base = smem_u32(psm);
+
+  const int tid = threadIdx.x;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
+  const int range = blockIdx.x;
+
+  // Groups of a request run in lockstep on neighbouring ranges, as in decode_tc_kernel.
+  SchedArgs sa0;
+  sa0.cu = p.cu;
+  sa0.B = p.B;
+  sa0.s_q = p.s_q;
+  sa0.tile = TN;
+  sa0.units_per_req = p.G;
+  sa0.per_query_units = 0;
+  sa0.P = p.P;
+  const bool lockstep = lockstep_groups(sa0);
+  const SchedArgs sa = request_space(sa0);
+  const int sched_range = lockstep ? range / p.G : range;
+  const int kfix = lockstep ? range % p.G : 0;
+  auto next_seg = [&](SegCursor& c, Segment& sg) -> bool {
+    const bool r = c.next(sa, sg);
+    if (r && lockstep) {
+      sg.k = kfix;
+      sg.unit_id = sg.b * p.G + kfix;
+    }
+    return r;
+  };
+
+  if (tid == 0) {
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(smem_u32(&sm.full[s]), 1);
+      mbar_init(smem_u32(&sm.empty[s]), 1);
+    }
+    for (int s = 0; s < VS; ++s) {
+      mbar_init(smem_u32(&sm.vfull[s]), 1);
+      mbar_init(smem_u32(&sm.vempty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&sm.s_full[b]), 1);
+      mbar_init(smem_u32(&sm.s_free[b]), 8);  // the 8 softmax warps
+      mbar_init(smem_u32(&sm.p_full[b]), 8);
+      mbar_init(smem_u32(&sm.o_done[b]), 1);
+      mbar_init(smem_u32(&sm.xb4[b]), 8);
+    }
+    mbar_init(smem_u32(&sm.q_ready), 8);
+    mbar_init(smem_u32(&sm.o_free), 8);
+    mbar_init(smem_u32(&sm.drain), 2);  // one commit from each issuer
+    sm.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    bool malformed = false;
+    SegCursor c = locate_range(sa, sched_range, &malformed);
+    if (lane == 0) {
+      if (malformed && range == 0) record_error(p.err, LKV_SITE_BAD_LENGTH);
+      sm.t_begin = c.t_begin;
+      sm.t_end = c.t_end;
+      sm.unit_t0 = c.unit_t0;
+      sm.b0 = c.b;
+      sm.k0 = c.k;
+      p.seg_info[2 * range] = -1;
+      p.seg_info[2 * range + 1] = -1;
+      tma_prefetch_desc(&map_k);
+      tma_prefetch_desc(&map_r);
+      if (!kTied) tma_prefetch_desc(&map_v);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&sm.tmem_base), Cfg::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid == 0) griddep_launch_dependents();  // the split combine may start launching
+  const uint32_t tbase = sm.tmem_base;
+  const WaitCtl wc{&sm.abort, p.err, p.wait_limit_ns};
+
+  SegCursor cur0;
+  cur0.t_begin = sm.t_begin;
+  cur0.t_end = sm.t_end;
+  cur0.unit_t0 = sm.unit_t0;
+  cur0.b = sm.b0;
+  cur0.k = sm.k0;
+  cur0.produced = 0;
+
+  if (warp == 0) {
+    // ============================================================ TMA producer
+    if (lane == 0) {
+      SegCursor cur = cur0;
+      Segment sg;
+      int n = 0, nv = 0;
+      bool ok = true;
+      while (ok && next_seg(cur, sg)) {
+        for (int t = sg.tile_lo; t < sg.tile_hi; ++t) {
+          const int st = n % KS;
+          if (!mbar_wait(smem_u32(&sm.empty[st]), static_cast<uint32_t>(((n / KS) & 1) ^ 1), wc, SB + W_EMPTY)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = smem_u32(&sm.full[st]);
+          mbar_arrive_expect_tx(fb, kStageBytes);
+          const uint32_t dst = stage_base + st * kStageBytes;
+          const int row = sg.cu_b + t * TN;
+          const int c0 = 128 * sg.k;
+          tma_load_2d(dst, &map_k, fb, c0, row);
+          tma_load_2d(dst + kBoxBytes, &map_k, fb, c0 + 64, row);
+          tma_load_2d(dst + 2 * kBoxBytes, &map_r, fb, 0, row);
+          ++n;
+          if (!kTied) {
+            const int vs = nv % VS;
+            if (!mbar_wait(smem_u32(&sm.vempty[vs]), static_cast<uint32_t>(((nv / VS) & 1) ^ 1), wc, SB + W_EMPTY)) {
+              ok = false;
+              break;
+            }
+            const uint32_t vb = smem_u32(&sm.vfull[vs]);
+            mbar_arrive_expect_tx(vb, Cfg::kVStageBytes);
+            const uint32_t vdst = vring_base + vs * Cfg::kVStageBytes;
+            tma_load_2d(vdst, &map_v, vb, c0, row);
+            tma_load_2d(vdst + kBoxBytes, &map_v, vb, c0 + 64, row);
+            ++nv;
+          }
+        }
+      }
+      // no copy may still be landing when the CTA exits: wait for the last ones issued
+      uint32_t zero = 0;
+      const WaitCtl dc{&zero, p.err, p.wait_limit_ns};
+      for (int m = (n > KS ? n - KS : 0); m < n; ++m)
+        mbar_wait(smem_u32(&sm.full[m % KS]), static_cast<uint32_t>((m / KS) & 1), dc, SB + W_DRAIN);
+      if (!kTied)
+        for (int m = (nv > VS ? nv - VS : 0); m < nv; ++m)
+          mbar_wait(smem_u32(&sm.vfull[m % VS]), static_cast<uint32_t>((m / VS) & 1), dc, SB + W_DRAIN);
+    }
+  }
+  else if (warp == 1 || warp == 2) {
+    // ============================================================ MMA issuers
+    if (lane == 0) {
+      SegCursor cur = cur0;
+      Segment sg;
+      int n = 0, seg = 0;
+      bool ok = true;
+      if (warp == 1) {
+        // S^T[key, row] = K[key, :] . Q[row, :]: A = the key tile, K-major (boxes 0 and 1, then the
+        // RoPE box 2); B = Q, K-major (each row's 192 columns); M = 128 keys, N = 32 rows
+        const uint32_t id_qk = idesc_bf16(128, Cfg::kN, 0, 0);
+        const uint64_t qdesc = sdesc_sw128(q_base, 16, 1024);
+        while (ok && next_seg(cur, sg)) {
+          for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
+            const int st = n % KS;
+            const int sb = n & 1;
+            if (!mbar_wait(smem_u32(&sm.full[st]), static_cast<uint32_t>((n / KS) & 1), wc, SB + W_FULL) ||
+                (n >= 2 && !mbar_wait(smem_u32(&sm.s_free[sb]), static_cast<uint32_t>(((n - 2) >> 1) & 1), wc,
+                                      SB + W_SFREE)) ||
+                (t == sg.tile_lo &&
+                 !mbar_wait(smem_u32(&sm.q_ready), static_cast<uint32_t>(seg & 1), wc, SB + W_QREADY))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint64_t kdesc = sdesc_sw128(stage_base + st * kStageBytes, 16, 1024);
+#pragma unroll
+            for (int ks = 0; ks < 12; ++ks) {
+              const int bx = ks >> 2, kk = ks & 3;
+              umma_ss(tbase + S0 + Cfg::kN * sb, desc_add(kdesc, bx * kBoxBytes + kk * 32),
+                      desc_add(qdesc, bx * Cfg::kQBoxBytes + kk * 32), id_qk, ks ? 1u : 0u);
+            }
+            umma_commit(smem_u32(&sm.s_full[sb]));
+            if (!kTied) umma_commit(smem_u32(&sm.empty[st]));  // the key stage is free once QK is done
+          }
+          ++seg;
+        }
+      } else {
+        // O^T[d, row] += V^T[d, key] P^T[key, row]: A = the value tile read MN-major (d contiguous in
+        // two 64-wide boxes, LBO between them); B = P^T, MN-major (rows contiguous, 64-byte swizzle,
+        // 8-key atoms of 512 bytes); M = 128, N = 32, 16 keys per MMA
+        const uint32_t id_pv = idesc_bf16(128, Cfg::kN, 1, 1);
+        while (ok && next_seg(cur, sg)) {
+          for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
+            const int pb = n & 1;
+            const bool first = (t == sg.tile_lo);
+            if (!mbar_wait(smem_u32(&sm.p_full[pb]), static_cast<uint32_t>((n >> 1) & 1), wc, SB + W_PFULL) ||
+                (first && seg > 0 &&
+                 !mbar_wait(smem_u32(&sm.o_free), static_cast<uint32_t>((seg - 1) & 1), wc, SB + W_OFREE)) ||
+                (!kTied && !mbar_wait(smem_u32(&sm.vfull[n % VS]), static_cast<uint32_t>((n / VS) & 1), wc,
+                                      SB + W_FULL))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t vaddr = kTied ? stage_base + static_cast<uint32_t>(n % KS) * kStageBytes
+                                         : vring_base + static_cast<uint32_t>(n % VS) * Cfg::kVStageBytes;
+            const uint64_t adesc = sdesc_sw128(vaddr, kBoxBytes, 1024);
+            const uint64_t pdesc = sdesc_sw64(p_base + static_cast<uint32_t>(pb) * Cfg::kPBytes, 16, 512);
+#pragma unroll
+            for (int kk = 0; kk < TN / 16; ++kk)
+              umma_ss(tbase + O0, desc_add(adesc, kk * 2048), desc_add(pdesc, kk * 1024), id_pv,
+                      (first && kk == 0) ? 0u : 1u);
+            umma_commit(smem_u32(&sm.o_done[pb]));
+            umma_commit(kTied ? smem_u32(&sm.empty[n % KS]) : smem_u32(&sm.vempty[n % VS]));
+          }
+          ++seg;
+        }
+      }
+      // every MMA of this thread complete before TMEM is released (both issuers arrive)
+      umma_commit(smem_u32(&sm.drain));
+      uint32_t zero = 0;
+      const WaitCtl dc{&zero, p.err, p.wait_limit_ns};
+      mbar_wait(smem_u32(&sm.drain), 0, dc, SB + W_DRAIN);
+    }
+  }
+  else if (warp >= 4) {
+    // ============================================================ softmax / epilogue
+    const int sw = warp - 4;                 // softmax warp 0..7
+    const int q4 = warp & 3;                 // TMEM lane quadrant
+    const int hh = sw >> 2;                  // rows 16 hh .. 16 hh + 15
+    const int rb = 16 * hh;
+    const int k = q4 * 32 + lane;            // key of the tile = S^T lane; value column d of O^T
+    const int rl = lane & 15;                // after a row reduction: this lane's row, rb + rl
+    const uint32_t lb = static_cast<uint32_t>(q4 * 32);
+    auto wait_all = [&](uint32_t bar, uint32_t par, int site) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, par, wc, site)) != 0;
+    };
+    auto warp_arrive = [&](uint32_t bar) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar);
+    };
+    // every warp posts one value per row (lanes 0-15) and reads back the posts of the 4 warps of
+    // its row half (the 4 lane quadrants, i.e. all 128 keys)
+    int xc = 0;
+    auto xchg4 = [&](float v, float (&all)[4]) -> bool {
+      const int b = xc & 1;
+      if (lane < 16) sm.red[b][sw][lane] = v;
+      warp_arrive(smem_u32(&sm.xb4[b]));
+      const bool okx = wait_all(smem_u32(&sm.xb4[b]), static_cast<uint32_t>((xc >> 1) & 1), SB + W_XCHG);
+#pragma unroll
+      for (int w = 0; w < 4; ++w) all[w] = sm.red[b][4 * hh + w][rl];
+      ++xc;
+      return okx;
+    };
+    // the unit's Q (rows padded with zeros to 32) as the K-major B operand: 24 chunks of 16 bytes a row
+    auto load_q = [&](const Segment& sg) {
+      for (int idx = sw * 32 + lane; idx < Cfg::kN * 24; idx += 256) {
+        const int r = idx / 24, c = idx % 24;
+        const int bx = c >> 3, cc = c & 7;
+        uint4 x = make_uint4(0u, 0u, 0u, 0u);
+        if (r < p.R) {
+          const int i = r / p.hpg;
+          const int h = sg.k * p.hpg + (r - i * p.hpg);
+          const size_t qrow = (static_cast<size_t>(sg.b) * p.s_q + i) * p.h_q + h;
+          x = bx < 2 ? __ldg(reinterpret_cast<const uint4*>(p.q_nope + qrow * p.dq + 64 * bx) + cc)
+                     : __ldg(reinterpret_cast<const uint4*>(p.q_rope + qrow * 64) + cc);
+        }
+        *reinterpret_cast<uint4*>(qsm + bx * Cfg::kQBoxBytes + r * 128 + ((cc ^ (r & 7)) << 4)) = x;
+      }
+      fence_proxy_async_smem();
+      warp_arrive(smem_u32(&sm.q_ready));
+    };
+
+    const int qi0 = rb / p.hpg, rr0 = rb - qi0 * p.hpg;  // query and head offset of row rb
+    SegCursor cur = cur0;
+    Segment sg, nx;
+    bool ok = true;
+    int n = 0;
+    // running max of row rb + rl (log2 units); per row j of this warp, this thread's (key lane k)
+    // running sums of the fp32 weights (for the lse) and of the bf16 weights PV uses
+    float m_run = -INFINITY;
+    float lt[16], lbt[16];
+    bool have = next_seg(cur, sg);
+    if (have) load_q(sg);
+    while (ok && have) {
+      bool have_nx = false;
+      const int lim0 = sg.L - p.s_q;  // query i sees keys 0 .. lim0 + i of the request
+      for (int t = sg.tile_lo; t < sg.tile_hi; ++t, ++n) {
+        const int sb = n & 1, pb = n & 1;
+        if (!wait_all(smem_u32(&sm.s_full[sb]), static_cast<uint32_t>((n >> 1) & 1), SB + W_SFULL)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t a[16];
+        tmem_ld16(tm_addr(tbase, lb, S0 + Cfg::kN * sb + rb), a);
+        tmem_wait_ld();
+        tc_fence_before();
+        warp_arrive(smem_u32(&sm.s_free[sb]));
+        if (t == sg.tile_hi - 1 && (have_nx = next_seg(cur, nx))) load_q(nx);  // this unit's QKs are done
+        if (t == sg.tile_lo) {
+          m_run = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            lt[j] = 0.f;
+            lbt[j] = 0.f;
+          }
+        }
+        // row rb + j is query (rb + j) / hpg; rows >= R are padding
+        const int kg = t * TN + k;  // key index in the request
+        float sv[16];
+        {
+          int qi = qi0, rr = rr0;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const bool vis = (rb + j < p.R) && (kg <= lim0 + qi);
+            sv[j] = vis ? __uint_as_float(a[j]) : -INFINITY;
+            if (++rr == p.hpg) {
+              rr = 0;
+              ++qi;
+            }
+          }
+        }
+        // the tile's max per row over the 128 keys (raw scores: the scale is positive)
+        float mx[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) mx[j] = sv[j];
+        const float mw = warp_rows_reduce16<true>(mx, lane);
+        float all4[4];
+        if (!xchg4(mw, all4)) {
+          ok = false;
+          break;
+        }
+        const float mt = fmaxf(fmaxf(all4[0], all4[1]), fmaxf(all4[2], all4[3])) * p.sl2;
+        bool rescale = false;
+        float m_new = m_run;
+        if (mt > m_run + 8.f) {  // lazy rescale: keep the running max unless it grows by 2^8
+          m_new = mt;
+          rescale = (m_run != -INFINITY);
+        }
+        // exponents centred on the tile max (<= 0, so the fp16 argument of the best keys is exact
+        // or nearly so), times f = 2^(mt - m_new) <= 2^8 in fp32
+        if (lane < 16) {
+          sm.msub[sw][lane] = (mt == -INFINITY) ? 0.f : mt;
+          sm.fac[sw][lane] = (mt == -INFINITY) ? 0.f : ex2_approx(mt - m_new);
+          sm.arow[sw][lane] = rescale ? ex2_approx(m_run - m_new) : 1.f;
+        }
+        m_run = m_new;
+        __syncwarp();
+        const bool any_rescale = __any_sync(0xffffffffu, rescale) != 0;
+        // this key's weight for the warp's 16 rows: half of row k of P^T
+        uint32_t pw[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t h = ex2_f16x2(fmaf(sv[2 * j], p.sl2, -sm.msub[sw][2 * j]),
+                                       fmaf(sv[2 * j + 1], p.sl2, -sm.msub[sw][2 * j + 1]));
+          const float e0 = f16_lo(h) * sm.fac[sw][2 * j], e1 = f16_hi(h) * sm.fac[sw][2 * j + 1];
+          pw[j] = pack_bf16x2(e0, e1);
+          if (any_rescale) {
+            lt[2 * j] *= sm.arow[sw][2 * j];
+            lt[2 * j + 1] *= sm.arow[sw][2 * j + 1];
+            lbt[2 * j] *= sm.arow[sw][2 * j];
+            lbt[2 * j + 1] *= sm.arow[sw][2 * j + 1];
+          }
+          lt[2 * j] += e0;
+          lt[2 * j + 1] += e1;
+          lbt[2 * j] += __uint_as_float(pw[j] << 16);
+          lbt[2 * j + 1] += __uint_as_float(pw[j] & 0xFFFF0000u);
+        }
+        // P buffer pb was last read by PV(n - 2)
+        if (n >= 2 && !wait_all(smem_u32(&sm.o_done[pb]), static_cast<uint32_t>(((n - 2) >> 1) & 1), SB + W_ODONE)) {
+          ok = false;
+          break;
+        }
+        {
+          // row k of P^T is 64 bytes in the 64-byte swizzle (16-byte chunk c at c ^ ((k >> 1) & 3));
+          // this warp's rows are chunks 2 hh and 2 hh + 1
+          uint8_t* prow = psm + pb * Cfg::kPBytes + k * 64;
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+            *reinterpret_cast<uint4*>(prow + (((2 * hh + c) ^ ((k >> 1) & 3)) << 4)) =
+                make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+        }
+        // keys past the request belong to another request or to unwritten cache: their P is 0, but
+        // 0 * NaN would still poison O, so each such value row is cleared (box hh by row half hh)
+        const int in_unit = sg.keys - t * TN;
+        if (in_unit < TN) {
+          if (!kTied && !wait_all(smem_u32(&sm.vfull[n % VS]), static_cast<uint32_t>((n / VS) & 1), SB + W_FULL)) {
+            ok = false;
+            break;
+          }
+          if (k >= in_unit) {
+            uint8_t* vb = kTied ? dsm + (n % KS) * kStageBytes : vring + (n % VS) * Cfg::kVStageBytes;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(vb + hh * kBoxBytes + k * 128 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+        fence_proxy_async_smem();
+        if (any_rescale && t != sg.tile_lo) {
+          // O^T holds this unit's tiles up to n-1: wait for PV(n-1), then scale column r by alpha_r
+          if (!wait_all(smem_u32(&sm.o_done[pb ^ 1]), static_cast<uint32_t>(((n - 1) >> 1) & 1), SB + W_ODONE)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          uint32_t o[16];
+          tmem_ld16(tm_addr(tbase, lb, O0 + rb), o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * sm.arow[sw][j]);
+          tmem_st16(tm_addr(tbase, lb, O0 + rb), o);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        warp_arrive(smem_u32(&sm.p_full[pb]));
+        if (t != sg.tile_hi - 1) continue;
+        // ---------------------------------------------------------- unit epilogue
+        const float lw = warp_rows_reduce16<false>(lt, lane);
+        const float lbw = warp_rows_reduce16<false>(lbt, lane);
+        float lt4[4], lb4[4];
+        if (!xchg4(lw, lt4) || !xchg4(lbw, lb4)) {
+          ok = false;
+          break;
+        }
+        const float l_tot = (lt4[0] + lt4[1]) + (lt4[2] + lt4[3]);  // row rb + rl
+        const float lb_tot = (lb4[0] + lb4[1]) + (lb4[2] + lb4[3]);
+        const float inv_l = lb_tot > 0.f ? 1.f / lb_tot : 0.f;
+        const float lse_v = l_tot > 0.f ? (m_run + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
+        if (lane < 16) sm.arow[sw][lane] = inv_l;
+        __syncwarp();
+        if (!wait_all(smem_u32(&sm.o_done[pb]), static_cast<uint32_t>((n >> 1) & 1), SB + W_ODONE)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        uint32_t o[16];
+        tmem_ld16(tm_addr(tbase, lb, O0 + rb), o);
+        tmem_wait_ld();
+        const int d = k;
+        const size_t slot_row = static_cast<size_t>(2 * range + (sg.complete ? 0 : sg.slot)) * p.rmax;
+        {
+          int qi = qi0, rr = rr0;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (rb + j < p.R) {
+              const size_t orow = (static_cast<size_t>(sg.b) * p.s_q + qi) * p.h_q + sg.k * p.hpg + rr;
+              const float val = __uint_as_float(o[j]) * sm.arow[sw][j];
+              if (sg.complete)
+                p.out[orow * p.dv_total + d] = __float2bfloat16_rn(val);
+              else
+                p.part_o[(slot_row + rb + j) * p.dv_total + d] = val;
+            }
+            if (++rr == p.hpg) {
+              rr = 0;
+              ++qi;
+            }
+          }
+        }
+        if (q4 == 0 && lane < 16 && rb + lane < p.R) {
+          const int r = rb + lane;
+          const int i = r / p.hpg;
+          const size_t orow = (static_cast<size_t>(sg.b) * p.s_q + i) * p.h_q + sg.k * p.hpg + (r - i * p.hpg);
+          if (sg.complete)
+            p.lse[orow] = lse_v;
+          else
+            p.part_lse[slot_row + r] = lse_v;
+        }
+        if (!sg.complete && sw == 0 && lane == 0) p.seg_info[2 * range + sg.slot] = sg.unit_id;
+        tc_fence_before();
+        warp_arrive(smem_u32(&sm.o_free));
+      }
+      if (!ok) break;
+      have = have_nx;
+      if (have) sg = nx;
+    }
+  }
+  // ---------------------------------------------------------------- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, Cfg::kTmemCols);
+  }
+}
+
+// Host side: dynamic shared memory of the two forms.
+inline size_t swap_smem_bytes(bool tied) { return tied ? SwapCfg<true>::kSmemBytes : SwapCfg<false>::kSmemBytes; }
+
+}  // namespace lkv

@@ -60,6 +60,19 @@ def test_source_hash_covers_only_the_decode_kernel_sources():
     assert "lkv_mla_pair.cuh" not in bench.KERNEL_SOURCES["grouped"]
     assert bench.kernel_source_hash("mla") == h                   # deterministic
     assert bench.kernel_source_hash("gqla") == bench.kernel_source_hash("gta") != h
+    assert "lkv_decode_swap.cuh" in bench.KERNEL_SOURCES["grouped"]
+    assert "lkv_decode_swap.cuh" not in bench.KERNEL_SOURCES["mla"]
+
+
+def test_decode_kernel_name_follows_the_launch_rule():
+    """GQLA / GTA units of at most 32 query rows run keys-in-M; wider units, GLA and MLA do not."""
+    names = {n: bench.decode_kernel_name(synth.workload(n)) for n in synth.WORKLOADS}
+    assert names["mla_b64_l4096"] == "mla_pair_kernel"
+    assert names["gqla_g8_sq2_l8192"] == "decode_swap_kernel<false>"    # 16 heads x 2 queries
+    assert names["long_gqla_g8"] == "decode_swap_kernel<false>"
+    assert names["gta_g8_sq2_l8192"] == "decode_swap_kernel<true>"
+    assert names["gqa2_sq2_l8192"] == "decode_tc_kernel<MODE_GQLA>"     # 64 heads x 2 queries
+    assert names["long_gla2"] == "decode_tc_kernel<MODE_GLA>"
 
 
 def test_roofline_entry_is_the_slower_of_bytes_and_flops():

@@ -219,7 +219,9 @@ def test_gta_fp8_rows_past_the_cache_do_not_leak(L, gpu):
 
 def test_gta_fp8_agrees_with_bf16_gta_on_the_dequantised_states(L, gpu):
     """The FP8 decode and the bf16 GTA decode over the dequantised (bf16-exact) states compute on
-    the same values: outputs agree to the bf16 rounding of the results."""
+    the same values.  The two run different kernels (the FP8 rows row-major, bf16 GTA with the keys
+    in the MMA's M dimension), whose fp32 sums are taken in different orders, so they agree within
+    the bf16 parity gates rather than bit for bit."""
     w, d, rows, codes, scales, kpe = _fp8_gta_case([700, 64, 3], seed=7)
     deq = torch.from_numpy(fp8.dequantize_rows(codes, scales)).bfloat16()
     assert torch.equal(deq.double(), torch.from_numpy(fp8.dequantize_rows(codes, scales)))
@@ -229,7 +231,7 @@ def test_gta_fp8_agrees_with_bf16_gta_on_the_dequantised_states(L, gpu):
     out16, lse16 = L.gta_group_decode(d["q"].to(gpu), d["q_rope"].to(gpu), cache[:, :width], cache[:, width:],
                                       w.groups, d["cu_seqlens"].to(gpu), w.scale)
     torch.cuda.synchronize()
-    assert torch.equal(out8, out16) and torch.equal(lse8, lse16)
+    compare(out8, lse8, out16.double().cpu().numpy(), lse16.double().cpu().numpy(), label="fp8 vs bf16 GTA")
 
 
 def test_gta_fp8_argument_errors(L, gpu):
