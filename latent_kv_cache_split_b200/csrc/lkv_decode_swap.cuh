@@ -15,7 +15,8 @@
 // those rows and value column d = k of O^T.  A row's tile max is a reduction over the 128 keys: a
 // reduce-scatter over the warp's lanes (16 shuffles, lane l ends with row l % 16), then the 4
 // quadrant warps' values through shared memory.  The row sums are kept per thread (one partial per
-// key lane and row) and reduced once, in the unit's epilogue.
+// key lane and row) and reduced once, in the unit's epilogue.  A tile that every query sees whole,
+// with no padding row, skips the mask.
 //
 // TMEM (128 columns): S^T buffers at columns 0 and 32 (128 keys x 32 rows, fp32), O^T at 64.
 // Shared memory: the key ring (two 64-column boxes of the group's key or tied state and the RoPE
@@ -62,10 +63,10 @@ struct __align__(16) SwapSmem {
   uint64_t s_full[2], s_free[2], p_full[2], o_done[2];
   uint64_t q_ready, o_free, drain;
   uint64_t xb4[2];           // the 8 softmax warps posted one value per row (double-buffered)
-  float red[2][8][16];       // [buffer][softmax warp][row of its half]
-  float msub[8][16];         // per warp: the tile's row max (log2 units), subtracted in the exponent
-  float fac[8][16];          // per warp: 2^(tile max - running max) per row
-  float arow[8][16];         // per warp: O rescale factor per row, then 1 / l at the end
+  alignas(16) float red[2][8][16];  // [buffer][softmax warp][row of its half]
+  alignas(16) float msub[8][16];    // per warp: the tile's row max (log2 units), subtracted in the exponent
+  alignas(16) float fac[8][16];     // per warp: 2^(tile max - running max) per row
+  alignas(16) float arow[8][16];    // per warp: O rescale factor per row, then 1 / l at the end
   uint32_t tmem_base;
   uint32_t abort;
   long long t_begin, t_end, unit_t0;
@@ -383,9 +384,10 @@ __global__ void __launch_bounds__(kSwapThreads, 1)
     bool ok = true;
     int n = 0;
     // running max of row rb + rl (log2 units); per row j of this warp, this thread's (key lane k)
-    // running sums of the fp32 weights (for the lse) and of the bf16 weights PV uses
+    // running sum of the fp32 weights: it gives the lse and normalises the output (the bf16 weights
+    // PV multiplies sum to it within their rounding; tracking their own sum cost 4 % more time)
     float m_run = -INFINITY;
-    float lt[16], lbt[16];
+    float lt[16];
     bool have = next_seg(cur, sg);
     if (have) load_q(sg);
     while (ok && have) {
@@ -407,15 +409,16 @@ __global__ void __launch_bounds__(kSwapThreads, 1)
         if (t == sg.tile_lo) {
           m_run = -INFINITY;
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            lt[j] = 0.f;
-            lbt[j] = 0.f;
-          }
+          for (int j = 0; j < 16; ++j) lt[j] = 0.f;
         }
-        // row rb + j is query (rb + j) / hpg; rows >= R are padding
+        // row rb + j is query (rb + j) / hpg; rows >= R are padding.  A tile whose last key every
+        // query sees, with no padding row, needs no mask (the common case).
         const int kg = t * TN + k;  // key index in the request
         float sv[16];
-        {
+        if ((t + 1) * TN - 1 <= lim0 && p.R == kSwapMaxRows) {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) sv[j] = __uint_as_float(a[j]);
+        } else {
           int qi = qi0, rr = rr0;
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
@@ -455,23 +458,29 @@ __global__ void __launch_bounds__(kSwapThreads, 1)
         __syncwarp();
         const bool any_rescale = __any_sync(0xffffffffu, rescale) != 0;
         // this key's weight for the warp's 16 rows: half of row k of P^T
+        float msub[16], fac[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float4 m4 = reinterpret_cast<const float4*>(sm.msub[sw])[j];
+          const float4 f4 = reinterpret_cast<const float4*>(sm.fac[sw])[j];
+          msub[4 * j] = m4.x, msub[4 * j + 1] = m4.y, msub[4 * j + 2] = m4.z, msub[4 * j + 3] = m4.w;
+          fac[4 * j] = f4.x, fac[4 * j + 1] = f4.y, fac[4 * j + 2] = f4.z, fac[4 * j + 3] = f4.w;
+        }
+        if (any_rescale) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float4 a4 = reinterpret_cast<const float4*>(sm.arow[sw])[j];
+            lt[4 * j] *= a4.x, lt[4 * j + 1] *= a4.y, lt[4 * j + 2] *= a4.z, lt[4 * j + 3] *= a4.w;
+          }
+        }
         uint32_t pw[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-          const uint32_t h = ex2_f16x2(fmaf(sv[2 * j], p.sl2, -sm.msub[sw][2 * j]),
-                                       fmaf(sv[2 * j + 1], p.sl2, -sm.msub[sw][2 * j + 1]));
-          const float e0 = f16_lo(h) * sm.fac[sw][2 * j], e1 = f16_hi(h) * sm.fac[sw][2 * j + 1];
+          const uint32_t h = ex2_f16x2(fmaf(sv[2 * j], p.sl2, -msub[2 * j]), fmaf(sv[2 * j + 1], p.sl2, -msub[2 * j + 1]));
+          const float e0 = f16_lo(h) * fac[2 * j], e1 = f16_hi(h) * fac[2 * j + 1];
           pw[j] = pack_bf16x2(e0, e1);
-          if (any_rescale) {
-            lt[2 * j] *= sm.arow[sw][2 * j];
-            lt[2 * j + 1] *= sm.arow[sw][2 * j + 1];
-            lbt[2 * j] *= sm.arow[sw][2 * j];
-            lbt[2 * j + 1] *= sm.arow[sw][2 * j + 1];
-          }
           lt[2 * j] += e0;
           lt[2 * j + 1] += e1;
-          lbt[2 * j] += __uint_as_float(pw[j] << 16);
-          lbt[2 * j + 1] += __uint_as_float(pw[j] & 0xFFFF0000u);
         }
         // P buffer pb was last read by PV(n - 2)
         if (n >= 2 && !wait_all(smem_u32(&sm.o_done[pb]), static_cast<uint32_t>(((n - 2) >> 1) & 1), SB + W_ODONE)) {
@@ -523,15 +532,13 @@ __global__ void __launch_bounds__(kSwapThreads, 1)
         if (t != sg.tile_hi - 1) continue;
         // ---------------------------------------------------------- unit epilogue
         const float lw = warp_rows_reduce16<false>(lt, lane);
-        const float lbw = warp_rows_reduce16<false>(lbt, lane);
-        float lt4[4], lb4[4];
-        if (!xchg4(lw, lt4) || !xchg4(lbw, lb4)) {
+        float lt4[4];
+        if (!xchg4(lw, lt4)) {
           ok = false;
           break;
         }
         const float l_tot = (lt4[0] + lt4[1]) + (lt4[2] + lt4[3]);  // row rb + rl
-        const float lb_tot = (lb4[0] + lb4[1]) + (lb4[2] + lb4[3]);
-        const float inv_l = lb_tot > 0.f ? 1.f / lb_tot : 0.f;
+        const float inv_l = l_tot > 0.f ? 1.f / l_tot : 0.f;
         const float lse_v = l_tot > 0.f ? (m_run + __log2f(l_tot)) * 0.69314718055994531f : -INFINITY;
         if (lane < 16) sm.arow[sw][lane] = inv_l;
         __syncwarp();
