@@ -52,15 +52,16 @@ NOMINAL_PEAKS = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 KERNEL_SOURCES = {
     "mla": ("lkv_mla_pair.cuh", "lkv_decode_tc.cuh", "lkv_ptx.cuh", "lkv_sched.cuh"),  # with the shared TMEM row helpers
     "grouped": ("lkv_decode_swap.cuh", "lkv_decode_tc.cuh", "lkv_ptx.cuh", "lkv_sched.cuh"),
+    "gla": ("lkv_decode_swap_wide.cuh", "lkv_decode_swap.cuh", "lkv_decode_tc.cuh", "lkv_ptx.cuh", "lkv_sched.cuh"),
 }
 DECODE_SOURCES = tuple(sorted({f for v in KERNEL_SOURCES.values() for f in v}))
 
 
 def kernel_source_hash(kind: str = "mla") -> str:
     """Hash of the CUDA sources of the decode kernel that a workload of this kind launches
-    ("mla" for the CTA-pair kernel, anything else for the grouped kernel)."""
+    ("mla" for the CTA-pair kernel, "gla" for the GLA kernels, anything else for the grouped one)."""
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES["mla" if kind == "mla" else "grouped"]:
+    for f in KERNEL_SOURCES[kind if kind in ("mla", "gla") else "grouped"]:
         h.update(f.encode())
         with open(os.path.join(ROOT, "latent_kv_cache_split_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
@@ -68,6 +69,7 @@ def kernel_source_hash(kind: str = "mla") -> str:
 
 
 SWAP_MAX_ROWS = 32  # GQLA / GTA units of at most this many query rows run keys-in-M
+WIDE_MAX_ROWS = 64  # GLA units of at most this many query rows run keys-in-M
 
 
 def decode_kernel_name(w) -> str:
@@ -77,6 +79,8 @@ def decode_kernel_name(w) -> str:
     rows = (w.h_q // w.groups) * w.s_q
     if w.kind in ("gqla", "gta") and rows <= SWAP_MAX_ROWS:
         return "decode_swap_kernel<%s>" % ("true" if w.kind == "gta" else "false")
+    if w.kind == "gla" and rows <= WIDE_MAX_ROWS:
+        return "decode_swap_wide_kernel"
     return {"gqla": "decode_tc_kernel<MODE_GQLA>", "gla": "decode_tc_kernel<MODE_GLA>",
             "gta": "decode_tc_kernel<MODE_GTA>"}.get(w.kind, "decode_tc_kernel")
 

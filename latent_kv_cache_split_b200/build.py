@@ -19,7 +19,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "liblkv.so")
 SOURCES = ["lkv_api.cu", "lkv_proj.cu", "lkv_fp8.cu"]
-HEADERS = ["lkv_ptx.cuh", "lkv_sched.cuh", "lkv_decode_tc.cuh", "lkv_decode_swap.cuh", "lkv_mla_pair.cuh", "lkv_gemm.cuh", "lkv_aux.cuh", "lkv_tma_host.h"]
+HEADERS = ["lkv_ptx.cuh", "lkv_sched.cuh", "lkv_decode_tc.cuh", "lkv_decode_swap.cuh", "lkv_decode_swap_wide.cuh", "lkv_mla_pair.cuh", "lkv_gemm.cuh", "lkv_aux.cuh", "lkv_tma_host.h"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

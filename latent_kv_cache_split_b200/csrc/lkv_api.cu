@@ -11,6 +11,7 @@
 #include "lkv_aux.cuh"
 #include "lkv_decode_tc.cuh"
 #include "lkv_decode_swap.cuh"
+#include "lkv_decode_swap_wide.cuh"
 #include "lkv_mla_pair.cuh"
 #include "lkv_ptx.cuh"
 #include "lkv_tma_host.h"
@@ -71,7 +72,9 @@ lkv_status device_state(DeviceState** out) {
         cudaFuncSetAttribute(decode_swap_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(swap_smem_bytes(false))) != cudaSuccess ||
         cudaFuncSetAttribute(decode_swap_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(swap_smem_bytes(true))) != cudaSuccess)
+                             static_cast<int>(swap_smem_bytes(true))) != cudaSuccess ||
+        cudaFuncSetAttribute(decode_swap_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(WideCfg::kSmemBytes)) != cudaSuccess)
       return LKV_ERR_CUDA;
     d.ready = true;
   }
@@ -146,6 +149,9 @@ lkv_status launch_combine(const TcParams& p, int units_per_req, int per_query_un
   return launch_err(cudaLaunchKernelEx(&cfg, combine_kernel, c));
 }
 
+// GLA units of at most 64 rows run the keys-in-M kernel (lkv_decode_swap_wide.cuh).
+inline bool gla_keys_in_m(int mode, int R) { return mode == MODE_GLA && R <= kWideMaxRows; }
+
 struct TcLaunch {
   int mode;
   CUtensorMap map_a, map_r, map_v;
@@ -155,7 +161,8 @@ struct TcLaunch {
 };
 
 // Grouped decode (one CTA per range), then the split combine.  GQLA and GTA units of at most 32
-// rows run with the keys in the MMA's M dimension (lkv_decode_swap.cuh); the rest row-major.
+// rows and GLA units of at most 64 run with the keys in the MMA's M dimension (lkv_decode_swap.cuh,
+// lkv_decode_swap_wide.cuh); the rest row-major.
 lkv_status run_tc(TcLaunch& L, const DeviceState& d, cudaStream_t stream) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(L.p.P);
@@ -164,7 +171,11 @@ lkv_status run_tc(TcLaunch& L, const DeviceState& d, cudaStream_t stream) {
   cfg.stream = stream;
   cudaError_t e;
   const bool swap = (L.mode == MODE_GQLA || L.mode == MODE_GTA) && L.p.R <= kSwapMaxRows;
-  if (swap) {
+  if (gla_keys_in_m(L.mode, L.p.R)) {
+    cfg.blockDim = dim3(kSwapThreads);
+    cfg.dynamicSmemBytes = WideCfg::kSmemBytes;
+    e = cudaLaunchKernelEx(&cfg, decode_swap_wide_kernel, L.map_a, L.map_r, L.p);
+  } else if (swap) {
     cfg.blockDim = dim3(kSwapThreads);
     cfg.dynamicSmemBytes = swap_smem_bytes(L.mode == MODE_GTA);
     if (L.mode == MODE_GTA)
@@ -694,9 +705,11 @@ lkv_status lkv_gla_group_decode(const void* q, const void* q_rope, const void* c
   if (!workspace || !al16(workspace) || workspace_bytes < w.total) return LKV_ERR_WORKSPACE;
   TcLaunch L;
   L.mode = MODE_GLA;
+  // 128-key tiles for the keys-in-M kernel, 64-key tiles for the rows-in-M one
+  const uint32_t box_rows = gla_keys_in_m(MODE_GLA, R) ? WideCfg::kTile : ModeCfg<MODE_GLA>::kTile;
   if (!make_tmap_bf16(&L.map_a, clat, static_cast<uint64_t>(n_lat) * r_g, cache_rows,
-                      clat_row_stride * 2, 64, ModeCfg<MODE_GLA>::kTile) ||
-      !make_tmap_bf16(&L.map_r, kpe, d_rope, cache_rows, kpe_row_stride * 2, 64, ModeCfg<MODE_GLA>::kTile))
+                      clat_row_stride * 2, 64, box_rows) ||
+      !make_tmap_bf16(&L.map_r, kpe, d_rope, cache_rows, kpe_row_stride * 2, 64, box_rows))
     return LKV_ERR_CUDA;
   L.map_v = L.map_a;
   uint8_t* ws = static_cast<uint8_t*>(workspace);

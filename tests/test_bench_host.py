@@ -62,17 +62,20 @@ def test_source_hash_covers_only_the_decode_kernel_sources():
     assert bench.kernel_source_hash("gqla") == bench.kernel_source_hash("gta") != h
     assert "lkv_decode_swap.cuh" in bench.KERNEL_SOURCES["grouped"]
     assert "lkv_decode_swap.cuh" not in bench.KERNEL_SOURCES["mla"]
+    assert "lkv_decode_swap_wide.cuh" in bench.KERNEL_SOURCES["gla"]
+    assert "lkv_decode_swap_wide.cuh" not in bench.KERNEL_SOURCES["grouped"]
+    assert bench.kernel_source_hash("gla") not in (h, bench.kernel_source_hash("gqla"))
 
 
 def test_decode_kernel_name_follows_the_launch_rule():
-    """GQLA / GTA units of at most 32 query rows run keys-in-M; wider units, GLA and MLA do not."""
+    """GQLA / GTA units of at most 32 query rows and GLA units of at most 64 run keys-in-M."""
     names = {n: bench.decode_kernel_name(synth.workload(n)) for n in synth.WORKLOADS}
     assert names["mla_b64_l4096"] == "mla_pair_kernel"
     assert names["gqla_g8_sq2_l8192"] == "decode_swap_kernel<false>"    # 16 heads x 2 queries
     assert names["long_gqla_g8"] == "decode_swap_kernel<false>"
     assert names["gta_g8_sq2_l8192"] == "decode_swap_kernel<true>"
     assert names["gqa2_sq2_l8192"] == "decode_tc_kernel<MODE_GQLA>"     # 64 heads x 2 queries
-    assert names["long_gla2"] == "decode_tc_kernel<MODE_GLA>"
+    assert names["long_gla2"] == "decode_swap_wide_kernel"              # 64 heads x 1 query
 
 
 def test_roofline_entry_is_the_slower_of_bytes_and_flops():
