@@ -1,8 +1,9 @@
 """GPU parity of the keys-in-M decode kernels (GQLA / GTA units of at most 32 rows, GLA units of at
 most 64) on the unit shapes the benchmark workloads do not reach: two queries per unit with the
 second starting inside a softmax warp's rows, and padding rows (fewer live rows than the MMA's N).
-(The entry points take s_q = 1 or 2.)  Each case against the fp64 oracle with the usual bf16 gates, ragged lengths that span
-several 128-key tiles, a request shorter than a tile and one of exactly s_q keys."""
+(The entry points take s_q = 1 or 2.)  Each case against the fp64 oracle with the usual bf16
+gates, ragged lengths that span several 128-key tiles, a request shorter than a tile and one of
+exactly s_q keys."""
 import pytest
 import torch
 
