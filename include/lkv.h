@@ -74,7 +74,8 @@ const char* lkv_status_string(int status);
  * (request, unit) pairs are laid end to end and cut into `ranges` equal runs, one per
  * persistent CTA (MLA: per CTA pair).  A unit is one query token of a request for MLA,
  * one group of a request for GQLA / GLA.  Returns the number of ranges, or -1 on bad input.
- *   kind: 0 = MLA absorbed, 1 = GQLA, 2 = GLA, 3 = GTA (partitioned like GQLA).
+ *   kind: 0 = MLA absorbed, 1 = GQLA, 2 = GLA, 3 = GTA (partitioned like GQLA), 4 = GLA whose
+ *   units have at most 64 rows (s_q * h_q / groups <= 64: the ranges of kind 2).
  *   num_sms: SMs available on the device.
  */
 int lkv_plan_ranges(int kind, int batch, int s_q, int groups, int num_sms);
@@ -83,7 +84,8 @@ int lkv_plan_ranges(int kind, int batch, int s_q, int groups, int num_sms);
  * Host-only view of the same partition (no CUDA call): for host-side cu_seqlens_host [batch+1]
  * and `num_ranges` ranges, writes one record of 8 int32 per segment, in processing order:
  *   (range, request, unit, tile_lo, tile_hi, complete, slot, unit_id)
- * tiles are 256 keys (MLA), 128 keys (GQLA, GTA) or 64 keys (GLA); slot is -1 for a segment that covers its whole unit, else the partial
+ * tiles are 256 keys (MLA), 128 keys (GQLA, GTA, GLA units of at most 64 rows: kind 4) or 64 keys
+ * (GLA units of more rows: kind 2); slot is -1 for a segment that covers its whole unit, else the partial
  * slot (0 = first segment of its range, 1 = last).  Returns the number of segments (records
  * past max_out are counted but not written), or -1 on bad input.
  */

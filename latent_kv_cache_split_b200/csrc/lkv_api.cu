@@ -276,14 +276,22 @@ const char* lkv_status_string(int s) {
 }
 
 int lkv_plan_ranges(int kind, int batch, int s_q, int groups, int num_sms) {
-  if (kind == 3) kind = 1;  // GTA runs the GQLA kernel
+  if (kind == 3) kind = 1;  // GTA is partitioned like GQLA
+  if (kind == 4) kind = 2;  // GLA with 128-key tiles: the same ranges
   if (kind < 0 || kind > 2) return -1;
   return plan_ranges(kind, batch, s_q, kind == 0 ? 1 : groups, num_sms);
 }
 
+static_assert(WideCfg::kTile == ModeCfg<MODE_GQLA>::kTile, "kind 4 describes the keys-in-M GLA tiles");
+
 int lkv_plan_segments(int kind, const int32_t* cu_seqlens_host, int batch, int s_q, int groups,
                       int num_ranges, int32_t* out, int max_out) {
   if (kind == 3) kind = 1;
+  // kind 4: GLA units of at most 64 rows, which the keys-in-M kernel walks in 128-key tiles
+  const int tile = kind == 0 ? kPairTile
+                 : (kind == 1 || kind == 4) ? ModeCfg<MODE_GQLA>::kTile
+                                            : ModeCfg<MODE_GLA>::kTile;
+  if (kind == 4) kind = 2;
   if (kind < 0 || kind > 2 || !cu_seqlens_host || batch <= 0 || s_q <= 0 || num_ranges <= 0 ||
       (kind != 0 && groups <= 0) || max_out < 0 || (max_out > 0 && !out))
     return -1;
@@ -294,7 +302,7 @@ int lkv_plan_segments(int kind, const int32_t* cu_seqlens_host, int batch, int s
   a.units_per_req = kind == 0 ? s_q : groups;
   a.per_query_units = kind == 0 ? 1 : 0;
   a.P = num_ranges;
-  a.tile = kind == 0 ? kPairTile : (kind == 1 ? ModeCfg<MODE_GQLA>::kTile : ModeCfg<MODE_GLA>::kTile);
+  a.tile = tile;
   const bool lockstep = lockstep_groups(a);
   const SchedArgs ar = request_space(a);
   int n = 0;
@@ -332,6 +340,7 @@ size_t lkv_mla_decode_workspace_size(int batch, int s_q, int h_q, int r_kv, int 
 size_t lkv_group_decode_workspace_size(int kind, int batch, int s_q, int h_q, int groups, int d_v,
                                        int num_sms) {
   if (kind == 3) kind = 1;
+  if (kind == 4) kind = 2;
   if (kind != 1 && kind != 2) return 0;
   const int P = plan_ranges(kind, batch, s_q, groups, num_sms);
   if (P <= 0 || h_q <= 0 || groups <= 0 || h_q % groups || d_v <= 0) return 0;

@@ -54,6 +54,7 @@ def test_version_and_status_strings(lkv):
     (1, 1, 1, 8, 144),      # one request: every block is a slice of it
     (3, 64, 2, 8, 144),     # GTA runs the GQLA kernel and partition
     (1, 64, 2, 2, 128),     # GQA-2: 128 equal units nearly fill 148 SMs: one range per unit
+    (4, 8, 1, 2, 148),      # GLA units of 64 rows: the ranges of kind 2
 ])
 def test_plan_ranges(lkv, kind, B, s_q, G, want):
     assert lkv.plan_ranges(kind, B, s_q, G, 148) == want
@@ -72,14 +73,15 @@ def test_workspace_sizes(lkv):
     g = lkv.group_decode_workspace_size(1, 64, 2, 128, 8, 128, 148)
     assert g >= 2 * 144 * 32 * 128 * 4
     assert lkv.group_decode_workspace_size(3, 64, 2, 128, 8, 128, 148) == g   # GTA: the GQLA layout
-    assert lkv.group_decode_workspace_size(4, 1, 1, 128, 8, 128, 148) == 0
+    assert lkv.group_decode_workspace_size(4, 8, 1, 128, 2, 256, 148) == lkv.group_decode_workspace_size(2, 8, 1, 128, 2, 256, 148) > 0
+    assert lkv.group_decode_workspace_size(5, 1, 1, 128, 8, 128, 148) == 0
     assert lkv.group_decode_workspace_size(1, 1, 1, 128, 7, 128, 148) == 0
 
 
 def _check_partition(segs, cu, kind, s_q, G, P):
     """Every tile of every unit is covered exactly once; slot rules hold."""
     B = len(cu) - 1
-    T = {0: 256, 1: 128, 2: 64}[kind]   # keys per tile: MLA pair kernel, GQLA / GTA, GLA
+    T = {0: 256, 1: 128, 2: 64, 4: 128}[kind]   # keys per tile: MLA pair, GQLA / GTA, GLA, GLA keys-in-M
     upr = s_q if kind == 0 else G
     covered = {}
     by_range = {}
@@ -113,7 +115,8 @@ def _check_partition(segs, cu, kind, s_q, G, P):
 
 
 @pytest.mark.parametrize("kind,s_q,G,P", [(0, 1, 1, 74), (0, 2, 1, 74), (1, 2, 8, 148), (2, 1, 2, 148),
-                                         (0, 1, 1, 3), (1, 1, 4, 5), (1, 2, 8, 144), (1, 1, 4, 8)])
+                                         (0, 1, 1, 3), (1, 1, 4, 5), (1, 2, 8, 144), (1, 1, 4, 8),
+                                         (4, 1, 2, 148), (4, 2, 4, 148)])
 def test_partition_covers_every_tile_once(lkv, kind, s_q, G, P):
     rng = np.random.default_rng(kind * 10 + s_q + P)
     for trial in range(4):
