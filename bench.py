@@ -737,14 +737,21 @@ def bench_gpu(args, rank, world, local_rank):
 _INPUT_CACHE = {}
 
 
-def cpu_baseline(w, budget_s: float):
-    """The oracle as it stands on the host cores, on a bounded sample of the workload."""
+def cpu_baseline(w, budget_s: float, one_thread: bool = True):
+    """The oracle as it stands on the host cores, on a bounded sample of the workload; with
+    one_thread, also its time on one core (BLAS limited to one thread) on a smaller sample."""
     import oracle
     if w.name not in _INPUT_CACHE:
         _INPUT_CACHE[w.name] = synth.make_inputs(w)
     d = _INPUT_CACHE[w.name]
     cu = d["cu_seqlens"].numpy().astype(np.int64)
     order = list(range(w.batch))
+    single = None
+    if one_thread:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            single = cpu_baseline(w, max(0.5, budget_s / 4), one_thread=False)
+        single = {k: single[k] for k in ("value", "sample", "seconds")}
     t0 = time.perf_counter()
     done = 0
     for b in order:
@@ -767,9 +774,12 @@ def cpu_baseline(w, budget_s: float):
         if time.perf_counter() - t0 > budget_s:
             break
     dt = time.perf_counter() - t0
-    return {"value": done * w.s_q / dt, "unit": "tokens/s", "cores": os.cpu_count(),
-            "kind": "oracle", "sample": f"{done} of {w.batch} requests of {w.name} (fp64 numpy oracle)",
-            "seconds": dt}
+    res = {"value": done * w.s_q / dt, "unit": "tokens/s", "cores": os.cpu_count(),
+           "kind": "oracle", "sample": f"{done} of {w.batch} requests of {w.name} (fp64 numpy oracle)",
+           "seconds": dt}
+    if single is not None:
+        res["one_thread"] = single
+    return res
 
 
 def bench_reference(args, rank, world):
@@ -778,8 +788,8 @@ def bench_reference(args, rank, world):
     w = synth.workload(args.workload)
     budget = max(1.0, 150.0 / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
-        cpu_baseline(w, budget)
-    vals = [cpu_baseline(w, budget) for _ in range(args.steps)]
+        cpu_baseline(w, budget, one_thread=False)
+    vals = [cpu_baseline(w, budget, one_thread=(i == args.steps - 1)) for i in range(args.steps)]
     v = float(np.mean([x["value"] for x in vals]))
     cb = dict(vals[-1])
     cb["value"] = v
@@ -802,7 +812,7 @@ def main():
     ap.add_argument("--workload", default="mla_b64_l4096", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="lkv", choices=["lkv", "reference"])
     ap.add_argument("--cpu-budget", type=float, default=20.0)
-    ap.add_argument("--side-iters", type=int, default=10,
+    ap.add_argument("--side-iters", type=int, default=50,
                     help="calls per workload for the flushed per-workload timings (0: skip them)")
     ap.add_argument("--side-cpu-budget", type=float, default=1.5,
                     help="seconds of CPU-oracle work per side workload")

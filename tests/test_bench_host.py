@@ -14,7 +14,7 @@ from oracle import accounting as acc
 def test_reference_line_keeps_the_contract(monkeypatch):
     calls = []
 
-    def fake_baseline(w, budget):
+    def fake_baseline(w, budget, one_thread=True):
         calls.append(budget)
         return {"value": 12.5, "unit": "tokens/s", "cores": 4, "kind": "oracle",
                 "sample": f"1 of {w.batch} requests of {w.name} (fp64 numpy oracle)", "seconds": 0.1}
