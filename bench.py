@@ -127,15 +127,24 @@ def job_throughput(tokens_per_rank: int, ms_this_rank: float, world: int, device
     return tokens_per_rank * world / (ms * 1e-3), ms
 
 
-def workload_accounting(w, lengths):
-    """Algorithmic bytes (cache rows once, q, out, lse) and FLOPs (visible query-key pairs)."""
+def fp8_row_bytes(width: int, d_rope: int) -> int:
+    """Bytes of one FP8 cache row: width e4m3 codes, the fp32 scale padded to 16 bytes, the bf16
+    RoPE key, rounded up to 16 bytes (656 for the 512-wide MLA latent, 1168 for GTA's 8 x 128)."""
+    return 16 * ((width + 16 + 2 * d_rope + 15) // 16)
+
+
+def workload_accounting(w, lengths, fp8: bool = False):
+    """Algorithmic bytes (cache rows once, q, out, lse) and FLOPs (visible query-key pairs).
+    fp8: the latent / tied-state rows are FP8 cache rows (fp8_row_bytes per token)."""
     lengths = np.asarray(lengths, dtype=np.int64)
     elem = 2 if w.dtype == "bf16" else 4
-    if w.kind in ("mla", "gla", "gta"):
-        row = w.groups * w.d_k + w.d_rope
+    if fp8:
+        if w.kind not in ("mla", "gla", "gta"):
+            raise ValueError("FP8 rows hold a latent or tied-state cache")
+        cache_bytes = int(lengths.sum()) * fp8_row_bytes(w.groups * w.d_k, w.d_rope)
     else:
-        row = w.groups * (w.d_k + w.d_v) + w.d_rope
-    cache_bytes = int(lengths.sum()) * row * elem
+        row = (w.groups * w.d_k if w.kind in ("mla", "gla", "gta") else w.groups * (w.d_k + w.d_v)) + w.d_rope
+        cache_bytes = int(lengths.sum()) * row * elem
     io_bytes = w.batch * w.s_q * w.h_q * ((w.d_k + w.d_rope) * elem + w.d_v * elem + 4)
     vis = sum(int((lengths - w.s_q + i + 1).sum()) for i in range(w.s_q))
     flops = vis * 2 * w.h_q * (w.d_k + w.d_rope + w.d_v)
@@ -149,10 +158,11 @@ SIDE_WORKLOADS = ("tiny_fp32_mla", "gqla_g8_sq2_l8192", "varlen_mla_sq1", "varle
 L2_FLUSH_BYTES = 256 << 20   # twice the 126 MB L2
 
 
-def roofline_entry(w, lengths, dec_ms, peaks, how):
+def roofline_entry(w, lengths, dec_ms, peaks, how, fp8: bool = False):
     """Algorithmic bytes / FLOPs of one decode call and the fraction of the roofline time
-    max(bytes / HBM peak, FLOPs / tensor peak) that a call of dec_ms milliseconds achieves."""
-    cache_bytes, io_bytes, flops = workload_accounting(w, lengths)
+    max(bytes / HBM peak, FLOPs / tensor peak) that a call of dec_ms milliseconds achieves.
+    fp8: the cache is FP8 rows (no ncu traffic figure is recorded for that kernel)."""
+    cache_bytes, io_bytes, flops = workload_accounting(w, lengths, fp8=fp8)
     alg_bytes = cache_bytes + io_bytes
     dec_s = dec_ms * 1e-3
     gbs = alg_bytes / dec_s / 1e9
@@ -164,7 +174,7 @@ def roofline_entry(w, lengths, dec_ms, peaks, how):
     peak = peaks["hbm_gbs"] if bound == "hbm" else peaks["bf16_tflops"]
     nominal = max(alg_bytes / (NOMINAL_PEAKS["hbm_gbs"] * 1e9), flops / (NOMINAL_PEAKS["bf16_tflops"] * 1e12)) / dec_s
     return {"bound": bound, "achieved": achieved, "peak": peak, "unit": "GB/s" if bound == "hbm" else "TFLOP/s",
-            "frac": achieved / peak, "traffic": measured_traffic(w.name),
+            "frac": achieved / peak, "traffic": None if fp8 else measured_traffic(w.name),
             "peak_source": f"{how} (MEASURED_PEAKS.json burst)", "nominal": {"frac": nominal},
             "roofline_ms": max(t_hbm, t_tc) * 1e3, "algorithmic_bytes": alg_bytes, "algorithmic_flops": flops,
             "kv_gbs": gbs, "tflops": tfl}
@@ -398,6 +408,81 @@ def bench_side_workloads(lkv, dev, names, iters: int, cpu_budget: float):
         del d, out, lse, decode
         torch.cuda.empty_cache()
     return res
+
+
+# The GTA workload with its tied states stored as FP8 cache rows (e4m3 codes, a power-of-two fp32
+# scale per token, the bf16 RoPE key), quantised on the device by the library before timing.
+FP8_BASE = "gta_g8_sq2_l8192"
+FP8_NAME = "gta_g8_sq2_l8192_fp8"
+
+
+def cpu_baseline_fp8(w, d, rows, lkv, budget_s: float):
+    """The oracle's FP8 GTA decode (dequantise, then the plain attention) on the host cores, on a
+    bounded sample (whole requests) of the device-quantised rows."""
+    import oracle
+    width = w.groups * w.d_k
+    codes_v, scales_v, kpe_v = lkv.fp8_cache_fields(rows, width, w.d_rope)
+    cu = d["cu_seqlens"].cpu().numpy().astype(np.int64)
+    t0 = time.perf_counter()
+    done = keys = 0
+    for b in range(w.batch):
+        c0, c1 = int(cu[b]), int(cu[b + 1])
+        one = np.array([0, c1 - c0], dtype=np.int64)
+        oracle.fp8.gta_group_decode_fp8(d["q"][b:b + 1].cpu(), d["q_rope"][b:b + 1].cpu(),
+                                        codes_v[c0:c1].contiguous().cpu().numpy(),
+                                        scales_v[c0:c1].contiguous().cpu().numpy(),
+                                        kpe_v[c0:c1].contiguous().cpu(), w.groups, one, w.scale)
+        done += 1
+        keys += c1 - c0
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": done * w.s_q / dt, "unit": "tokens/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{done} of {w.batch} requests ({keys} cached tokens) of {FP8_NAME} (fp64 numpy oracle "
+                      "over the dequantised rows)", "seconds": dt}
+
+
+def bench_fp8_gta(lkv, dev, iters: int, cpu_budget: float):
+    """lkv_gta_group_decode_fp8 on the GTA workload's shape (64 requests of 8192 keys, s_q = 2,
+    g = 8): the device-drawn bf16 tied states and RoPE key quantised into FP8 rows by
+    lkv_quantize_latent_fp8, then each decode call timed after an L2 flush like the other workloads.
+    The roofline counts the FP8 rows' bytes (1168 per token against 2176 in bf16)."""
+    w = synth.workload(FP8_BASE)
+    peaks, how = load_peaks()
+    nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+    stream = torch.cuda.current_stream(dev)
+    d = device_inputs(w, dev)
+    width = w.groups * w.d_k
+    rows = lkv.quantize_latent_fp8(d.pop("cache"), width)
+    torch.cuda.empty_cache()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    ws = torch.empty(lkv.group_decode_workspace_size(lkv.KIND_GTA, w.batch, w.s_q, w.h_q, w.groups, w.d_v, nsm),
+                     dtype=torch.uint8, device=dev)
+    out = torch.empty((w.batch, w.s_q, w.h_q, w.d_v), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.batch, w.s_q, w.h_q), dtype=torch.float32, device=dev)
+    cu = d["cu_seqlens"]
+
+    def decode(qq, qqr, o, l):
+        lkv.gta_group_decode_fp8(qq, qqr, rows, w.groups, cu, w.scale, out=o, lse=l, workspace=ws)
+
+    for _ in range(3):
+        decode(d["q"], d["q_rope"], out, lse)
+    if lkv.check_device() != 0:
+        raise RuntimeError(f"device error during warm-up of {FP8_NAME}")
+    ms = time_flushed(decode, (d["q"], d["q_rope"], out, lse), stream, flush, iters)
+    if lkv.check_device() != 0:
+        raise RuntimeError(f"device error while timing {FP8_NAME}")
+    med = float(np.median(ms))
+    return {"decode_ms": med, "decode_ms_min": float(min(ms)), "decode_ms_max": float(max(ms)), "calls": iters,
+            "tokens_per_s": w.batch * w.s_q / (med * 1e-3),
+            "dtype": "bf16 (cache rows e4m3 + power-of-two scale, dequantised in shared memory)",
+            "kernel": "decode_tc_kernel<MODE_GTA8> + split combine (one lkv_gta_group_decode_fp8 call)",
+            "shape": {"kind": "gta", "batch": w.batch, "s_q": w.s_q, "h_q": w.h_q, "groups": w.groups,
+                      "d_k": w.d_k, "d_v": w.d_v, "d_rope": w.d_rope, "seqlen": w.seqlen,
+                      "fp8_row_bytes": fp8_row_bytes(width, w.d_rope),
+                      "total_cached_tokens": int(d["lengths"].sum())},
+            "roofline": roofline_entry(w, d["lengths"], med, peaks, how, fp8=True),
+            "cpu_baseline": cpu_baseline_fp8(w, d, rows, lkv, cpu_budget)}
 
 
 class ClockSampler:
@@ -663,6 +748,13 @@ def bench_gpu(args, rank, world, local_rank):
     # Group-axis TP of the GQLA step over all ranks (every rank takes the same collective steps).
     del d
     tp_res = bench_tp(lkv, dev, rank, world, args.tp_steps, 3) if args.tp_steps > 0 else None
+
+    # The FP8 GTA decode last, its failure recorded in the line rather than ending the run.
+    if side is not None:
+        try:
+            side[FP8_NAME] = bench_fp8_gta(lkv, dev, args.side_iters, args.side_cpu_budget)
+        except Exception as e:  # noqa: BLE001 -- reported, not hidden
+            side[FP8_NAME] = {"error": f"{type(e).__name__}: {e}"[:300]}
 
     tokens = B * S * world
     cache_bytes, io_bytes, flops = workload_accounting(w, lengths)

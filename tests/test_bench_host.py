@@ -137,3 +137,43 @@ def test_tp_local_inputs_hold_one_ranks_groups_and_heads(world, rank):
     assert d["w_o"].shape == (w.h_q // world * w.d_v, 64)
     assert d["cu_seqlens"].tolist() == [0, 40, 80]
     assert all(t.dtype == torch.bfloat16 for k, t in d.items() if k not in ("lengths", "cu_seqlens"))
+
+
+def test_fp8_accounting_counts_the_fp8_rows():
+    """The FP8 GTA entry's roofline counts one FP8 row per token (codes, 16-byte scale field, bf16
+    RoPE key), the size the library's own row-size call gives, and the bf16 query / output bytes."""
+    import latent_kv_cache_split_b200 as lkv
+    assert bench.fp8_row_bytes(512, 64) == 656 == lkv.fp8_cache_row_bytes(512, 64)
+    assert bench.fp8_row_bytes(1024, 64) == 1168 == lkv.fp8_cache_row_bytes(1024, 64)
+    w = synth.workload(bench.FP8_BASE)
+    lengths = np.full(w.batch, w.seqlen, dtype=np.int64)
+    c16, io16, f16 = bench.workload_accounting(w, lengths)
+    c8, io8, f8 = bench.workload_accounting(w, lengths, fp8=True)
+    assert c8 == int(lengths.sum()) * 1168 and c16 == int(lengths.sum()) * 2176
+    assert (io8, f8) == (io16, f16)
+    r = bench.roofline_entry(w, lengths, 1.0, {"hbm_gbs": 1000.0, "bf16_tflops": 100.0}, "test", fp8=True)
+    assert r["algorithmic_bytes"] == c8 + io8 and r["traffic"] is None
+    with pytest.raises(ValueError):
+        bench.workload_accounting(synth.workload("gqla_g8_sq2_l8192"), lengths, fp8=True)
+
+
+def test_cpu_baseline_fp8_reads_the_rows_fields():
+    """The FP8 entry's CPU baseline splits the rows into codes, scales and RoPE key with the
+    library's field views and runs the oracle's FP8 GTA decode on them: the same result as the
+    oracle on the quantised fields it was built from."""
+    import torch
+    import latent_kv_cache_split_b200 as lkv
+    from oracle import fp8
+    w = synth.workload(bench.FP8_BASE, batch=2, seqlen=None, len_lo=20, len_hi=40)
+    d = bench.device_inputs(w, torch.device("cpu"))
+    width = w.groups * w.d_k
+    codes, scales = fp8.quantize_rows(d["cache"][:, :width].float().numpy())
+    rows = torch.zeros((codes.shape[0], bench.fp8_row_bytes(width, w.d_rope)), dtype=torch.uint8)
+    rows[:, :width] = torch.from_numpy(codes)
+    rows[:, width:width + 4] = torch.from_numpy(scales.view(np.uint8).reshape(-1, 4))
+    rows[:, width + 16:width + 16 + 2 * w.d_rope] = d["cache"][:, width:].contiguous().view(torch.uint8)
+    c_v, s_v, k_v = lkv.fp8_cache_fields(rows, width, w.d_rope)
+    assert np.array_equal(c_v.numpy(), codes) and np.array_equal(s_v.numpy(), scales)
+    assert torch.equal(k_v, d["cache"][:, width:])
+    cb = bench.cpu_baseline_fp8(w, d, rows, lkv, 0.0)       # budget spent after the first request
+    assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["sample"].startswith("1 of 2 requests")
