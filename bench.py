@@ -442,6 +442,16 @@ def cpu_baseline_fp8(w, d, rows, lkv, budget_s: float):
                       "over the dequantised rows)", "seconds": dt}
 
 
+def add_guarded(side: dict, name: str, fn):
+    """side[name] = fn(); an exception is recorded there as {"error": "<type>: <message>"} instead of
+    ending the run (the entry is reported, not hidden)."""
+    try:
+        side[name] = fn()
+    except Exception as e:  # noqa: BLE001
+        side[name] = {"error": f"{type(e).__name__}: {e}"[:300]}
+    return side[name]
+
+
 def bench_fp8_gta(lkv, dev, iters: int, cpu_budget: float):
     """lkv_gta_group_decode_fp8 on the GTA workload's shape (64 requests of 8192 keys, s_q = 2,
     g = 8): the device-drawn bf16 tied states and RoPE key quantised into FP8 rows by
@@ -751,10 +761,7 @@ def bench_gpu(args, rank, world, local_rank):
 
     # The FP8 GTA decode last, its failure recorded in the line rather than ending the run.
     if side is not None:
-        try:
-            side[FP8_NAME] = bench_fp8_gta(lkv, dev, args.side_iters, args.side_cpu_budget)
-        except Exception as e:  # noqa: BLE001 -- reported, not hidden
-            side[FP8_NAME] = {"error": f"{type(e).__name__}: {e}"[:300]}
+        add_guarded(side, FP8_NAME, lambda: bench_fp8_gta(lkv, dev, args.side_iters, args.side_cpu_budget))
 
     tokens = B * S * world
     cache_bytes, io_bytes, flops = workload_accounting(w, lengths)

@@ -177,3 +177,15 @@ def test_cpu_baseline_fp8_reads_the_rows_fields():
     assert torch.equal(k_v, d["cache"][:, width:])
     cb = bench.cpu_baseline_fp8(w, d, rows, lkv, 0.0)       # budget spent after the first request
     assert cb["kind"] == "oracle" and cb["value"] > 0 and cb["sample"].startswith("1 of 2 requests")
+
+
+def test_a_failing_guarded_entry_is_recorded_not_raised():
+    side = {"x": {"decode_ms": 1.0}}
+
+    def boom():
+        raise RuntimeError("device error while timing gta_g8_sq2_l8192_fp8")
+
+    r = bench.add_guarded(side, bench.FP8_NAME, boom)
+    assert r == side[bench.FP8_NAME] and r["error"].startswith("RuntimeError: device error")
+    assert bench.add_guarded(side, "y", lambda: {"decode_ms": 2.0}) == {"decode_ms": 2.0}
+    assert side["x"] == {"decode_ms": 1.0}
