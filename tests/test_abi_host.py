@@ -81,7 +81,7 @@ def test_workspace_sizes(lkv):
 def _check_partition(segs, cu, kind, s_q, G, P):
     """Every tile of every unit is covered exactly once; slot rules hold."""
     B = len(cu) - 1
-    T = {0: 256, 1: 128, 2: 64, 4: 128}[kind]   # keys per tile: MLA pair, GQLA / GTA, GLA, GLA keys-in-M
+    T = {0: 256, 1: 128, 2: 64, 3: 128, 4: 128}[kind]   # keys per tile: MLA pair, GQLA, GLA, GTA, GLA keys-in-M
     upr = s_q if kind == 0 else G
     covered = {}
     by_range = {}
@@ -116,7 +116,7 @@ def _check_partition(segs, cu, kind, s_q, G, P):
 
 @pytest.mark.parametrize("kind,s_q,G,P", [(0, 1, 1, 74), (0, 2, 1, 74), (1, 2, 8, 148), (2, 1, 2, 148),
                                          (0, 1, 1, 3), (1, 1, 4, 5), (1, 2, 8, 144), (1, 1, 4, 8),
-                                         (4, 1, 2, 148), (4, 2, 4, 148)])
+                                         (4, 1, 2, 148), (4, 2, 4, 148), (3, 2, 8, 144), (3, 1, 4, 148)])
 def test_partition_covers_every_tile_once(lkv, kind, s_q, G, P):
     rng = np.random.default_rng(kind * 10 + s_q + P)
     for trial in range(4):
