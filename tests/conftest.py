@@ -27,3 +27,15 @@ def gpu():
         pytest.skip("no CUDA device")
     import torch
     return torch.device("cuda:0")
+
+
+@pytest.fixture(scope="session")
+def lkv_built():
+    """The binding with liblkv.so built in-tree first (nvcc cross-compiles; no GPU needed to load it)."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("lkv_build", os.path.join(ROOT, "latent_kv_cache_split_b200", "build.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+    import latent_kv_cache_split_b200 as L
+    return L

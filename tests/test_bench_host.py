@@ -139,10 +139,10 @@ def test_tp_local_inputs_hold_one_ranks_groups_and_heads(world, rank):
     assert all(t.dtype == torch.bfloat16 for k, t in d.items() if k not in ("lengths", "cu_seqlens"))
 
 
-def test_fp8_accounting_counts_the_fp8_rows():
+def test_fp8_accounting_counts_the_fp8_rows(lkv_built):
     """The FP8 GTA entry's roofline counts one FP8 row per token (codes, 16-byte scale field, bf16
     RoPE key), the size the library's own row-size call gives, and the bf16 query / output bytes."""
-    import latent_kv_cache_split_b200 as lkv
+    lkv = lkv_built
     assert bench.fp8_row_bytes(512, 64) == 656 == lkv.fp8_cache_row_bytes(512, 64)
     assert bench.fp8_row_bytes(1024, 64) == 1168 == lkv.fp8_cache_row_bytes(1024, 64)
     w = synth.workload(bench.FP8_BASE)
@@ -157,13 +157,13 @@ def test_fp8_accounting_counts_the_fp8_rows():
         bench.workload_accounting(synth.workload("gqla_g8_sq2_l8192"), lengths, fp8=True)
 
 
-def test_cpu_baseline_fp8_reads_the_rows_fields():
+def test_cpu_baseline_fp8_reads_the_rows_fields(lkv_built):
     """The FP8 entry's CPU baseline splits the rows into codes, scales and RoPE key with the
     library's field views and runs the oracle's FP8 GTA decode on them: the same result as the
     oracle on the quantised fields it was built from."""
     import torch
-    import latent_kv_cache_split_b200 as lkv
     from oracle import fp8
+    lkv = lkv_built
     w = synth.workload(bench.FP8_BASE, batch=2, seqlen=None, len_lo=20, len_hi=40)
     d = bench.device_inputs(w, torch.device("cpu"))
     width = w.groups * w.d_k
